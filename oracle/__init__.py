@@ -1,0 +1,40 @@
+"""CPU oracle for the mixed-precision FMHA forward.
+
+TEST INFRASTRUCTURE ONLY. Nothing on the product path may import this
+package: only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline
+leg of ``bench.py`` use it. It shares no code, table or constant with the
+CUDA library, and it imports nothing from it.
+
+What it computes (plain, slow, obviously correct):
+
+* ``e4m3``      -- the OCP 8-bit float E4M3 ("E4M3FN") codec, written from the
+                   format definition (bias 7, no infinities, max 448).
+* ``quant``     -- block quantization: amax -> scale = amax/R -> INT8 or E4M3
+                   codes, in IEEE float32 exactly as stated (one division for
+                   the scale, one per element for the code).
+* ``attention`` -- scaled-dot-product attention in float64 on dequantized
+                   operands, with causal / 128x128 block masks, GQA and a
+                   paged-KV gather.
+
+Sources (page titles; sections):
+
+* "FlashInfer DiT optimization: SageAttention and Int8/FP8 mixed-precision
+  kernels" (flashinfer PR #2711), sections 2 (SageAttention scale factors) and
+  "Why" item 2 (block-wise scaling beats per-tensor for outlier-heavy maps).
+* "FlashInfer FP8/BF16 mixed-precision attention for Blackwell" (flashinfer
+  PR #5900), introduction (dense context FMHA, QK-BF16/PV-FP8 and all-FP8).
+* "FlashInfer block-sparse attention with PrimTS" (flashinfer PR #4474),
+  section 2 (block-sparse API over contiguous and paged K/V).
+
+The pages never write the attention formula down; the oracle uses the
+textbook definition O = softmax(scale * Q K^T) V. Every reading taken where
+the pages are silent is listed in the module that takes it.
+
+Parity pins: every function here is pinned by ``tests/test_oracle_*.py``
+against brute force, closed forms, invariants or an independent library
+routine. The one thing left unpinned is the GPU's internal quantization of
+the softmax output P (not an operand, so not modelled here): "parity
+unpinned" beyond the stated tolerance.
+"""
+
+from . import e4m3, quant, attention  # noqa: F401
