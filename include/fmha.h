@@ -1,0 +1,196 @@
+/*
+ * fmha.h -- C ABI of libfmha.so: mixed-precision fused multi-head attention
+ * forward for NVIDIA B200 (sm_100a), plus the block quantizer that produces
+ * its 8-bit operands.
+ *
+ * Sources (page titles; sections):
+ *  [DiT-Sage]  "FlashInfer DiT optimization: SageAttention and Int8/FP8
+ *              mixed-precision kernels" (flashinfer PR #2711): section 1
+ *              (kernel key over separate Q/K/V/O dtypes and the four
+ *              SageAttention scale-factor granularities), section 2 (scale
+ *              factors for Q, K, P and V passed to the kernel and applied
+ *              after the Int8/FP8 BMM1 and BMM2), "Why" items 1-3.
+ *  [BW-FP8]    "FlashInfer FP8/BF16 mixed-precision attention for Blackwell"
+ *              (flashinfer PR #5900): introduction (dense context FMHA with
+ *              QK-BF16/PV-FP8 and all-FP8), section 3 (lazy O correction,
+ *              exp2 on MUFU and FMA).
+ *  [PrimTS-BS] "FlashInfer block-sparse attention with PrimTS" (flashinfer
+ *              PR #4474): section 2 (block-sparse attention over contiguous
+ *              and paged K/V through a page table).
+ *  [Cake-MLA]  "FlashInfer DeepSeek-V4 sparse-MLA: Cake backend" (flashinfer
+ *              PR #5686): section 1 (output written through a TMA descriptor
+ *              passed to the kernel as a grid constant).
+ *
+ * Conventions for every call
+ *  - All tensor pointers are DEVICE pointers owned by the caller. The library
+ *    never allocates device memory for a call and keeps no state between
+ *    calls except one device-global error word per device.
+ *  - Calls are asynchronous on `stream` (NULL = legacy default stream). The
+ *    only host synchronisation is in fmha_get_device_error().
+ *  - Argument errors are detected on the host and returned before anything
+ *    is launched; nothing is written. fmha_last_error_message() then holds a
+ *    one-line reason (thread-local).
+ *  - A device-side wait that runs out (a lost signal inside a kernel) never
+ *    traps or hangs: the kernel records FMHA_ERR_TIMEOUT in the device error
+ *    word and returns; fmha_get_device_error() reports it.
+ *  - Tensors are token-major "NHD": element (b, s, h, d) lives at
+ *    ptr + b*stride_b + s*stride_s + h*stride_h + d (strides in ELEMENTS,
+ *    d contiguous). Base pointers and strides must be 16-byte aligned
+ *    (TMA requirement); otherwise FMHA_ERR_INVALID_ARG.
+ *  - Indexing uses 64-bit offsets throughout.
+ */
+#ifndef FMHA_H_
+#define FMHA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+struct CUstream_st; /* cudaStream_t is `struct CUstream_st *` */
+
+typedef enum {
+  FMHA_OK = 0,
+  FMHA_ERR_INVALID_ARG = 1, /* bad pointer, size, stride, alignment or scale layout */
+  FMHA_ERR_UNSUPPORTED = 2, /* valid request this build does not implement (dtype tuple, D, page size) */
+  FMHA_ERR_CUDA = 3,        /* a CUDA runtime / driver call failed (message has the CUDA error) */
+  FMHA_ERR_TIMEOUT = 4,     /* a kernel's bounded wait ran out (reported by fmha_get_device_error) */
+  FMHA_ERR_DEVICE_INDEX = 5 /* a kernel met an out-of-range page index (reported by fmha_get_device_error) */
+} fmha_status;
+
+/* Element types. BF16/FP16 are IEEE-style 16-bit floats, E4M3 is the OCP
+ * 8-bit float (bias 7, max 448, no infinities), INT8 is two's complement. */
+typedef enum { FMHA_BF16 = 0, FMHA_FP16 = 1, FMHA_FP32 = 2, FMHA_E4M3 = 3, FMHA_INT8 = 4 } fmha_dtype;
+
+/* Scale-factor granularity ([DiT-Sage] sections 1-2). A scale factor is the
+ * fp32 DEQUANTIZATION multiplier: real value = code * scale. Layouts (fp32,
+ * contiguous), for a tensor of shape [B, S, H, D]:
+ *   FMHA_SF_NONE            no scale (1.0); ptr may be NULL
+ *   FMHA_SF_PER_TENSOR      [1]
+ *   FMHA_SF_PER_HEAD        [B, H]
+ *   FMHA_SF_PER_TOKEN_BLOCK [B, H, ceil(S / rows_per_block)]
+ *   FMHA_SF_PER_CHANNEL     [B, H, D]                                      */
+typedef enum {
+  FMHA_SF_NONE = 0,
+  FMHA_SF_PER_TENSOR = 1,
+  FMHA_SF_PER_HEAD = 2,
+  FMHA_SF_PER_TOKEN_BLOCK = 3,
+  FMHA_SF_PER_CHANNEL = 4
+} fmha_sf_kind;
+
+typedef struct {
+  void* ptr;        /* device pointer to element (0,0,0,0) */
+  int32_t dtype;    /* fmha_dtype */
+  int32_t reserved; /* must be 0 */
+  int64_t stride_b, stride_s, stride_h; /* element strides; d is contiguous */
+} fmha_tensor;
+
+typedef struct {
+  float* ptr;             /* device pointer, layout per `kind` */
+  int32_t kind;           /* fmha_sf_kind */
+  int32_t rows_per_block; /* tokens per block for FMHA_SF_PER_TOKEN_BLOCK, else ignored */
+} fmha_sf;
+
+/* Arguments of one attention call.
+ *   q [B, Sq, Hq, D], k [B, Skv, Hkv, D], v [B, Skv, Hkv, D], o [B, Sq, Hq, D].
+ *   Query head h attends to KV head h / (Hq / Hkv) (grouped-query attention).
+ *   O_i = sum_j softmax_j(softmax_scale * q_i . k_j) v_j over the visible keys
+ *   j, where q, k, v are the DEQUANTIZED operands (code * scale).
+ * Scale factors ([DiT-Sage] section 2): sf_q, sf_k, sf_v dequantize the
+ * 8-bit operands; sf_q / sf_k are applied to QK^T before the softmax, sf_v to
+ * the PV product in the epilogue. Allowed: sf_q PER_TENSOR / PER_HEAD /
+ * PER_TOKEN_BLOCK (any rows_per_block >= 1); sf_k PER_TENSOR / PER_HEAD /
+ * PER_TOKEN_BLOCK (rows_per_block a multiple of 32); sf_v PER_TENSOR /
+ * PER_HEAD / PER_CHANNEL. For BF16 operands the kind must be FMHA_SF_NONE.
+ * sf_p scales the softmax output P when P is cast to E4M3 for the PV product
+ * (8-bit V only): P is stored as E4M3(p / sf_p) and the product is multiplied
+ * back by sf_p. Allowed: NONE (= an internal power-of-two scale chosen for
+ * precision), PER_TENSOR, or PER_TOKEN_BLOCK over query rows [B, Hq,
+ * ceil(Sq / rows_per_block)] with rows_per_block a multiple of 128. Values
+ * must be positive and finite.
+ *   softmax_scale <= 0 selects 1/sqrt(D).
+ *   causal != 0: key j is visible to query i iff j <= i + (Skv - Sq)
+ *   (bottom-right aligned).
+ *   lse (nullable): fp32 [B, Hq, Sq], natural-log log-sum-exp of the scaled
+ *   scores; -inf for a row with no visible key (whose O row is 0).
+ * Supported (q, k, v, o) dtype tuples: (BF16, BF16, BF16, BF16),
+ * (BF16, BF16, E4M3, BF16) ("QK-BF16/PV-FP8", [BW-FP8]),
+ * (E4M3, E4M3, E4M3, BF16) ("all-FP8", [BW-FP8]), (INT8, INT8, E4M3, BF16)
+ * ("SageAttention", [DiT-Sage]). D must be 64 or 128 (128 for 8-bit Q/K).   */
+typedef struct {
+  fmha_tensor q, k, v, o;
+  fmha_sf sf_q, sf_k, sf_v, sf_p;
+  int32_t B, Hq, Hkv, Sq, Skv, D;
+  float softmax_scale;
+  int32_t causal;
+  float* lse;
+} fmha_args;
+
+/* Block quantizer: amax -> scale = amax / R -> codes ([DiT-Sage] section 2,
+ * "Why" item 2).
+ *   src: BF16 [B, S, H, D]; dst: INT8 (R = 127) or E4M3 (R = 448), same shape.
+ *   sf:  output scales, kind PER_TENSOR / PER_HEAD / PER_TOKEN_BLOCK /
+ *        PER_CHANNEL (layouts above).
+ * Per block: amax = max |x|; scale = fp32(amax) / fp32(R) (IEEE division;
+ * 1.0 when amax == 0); code = RN(fp32(x) / scale) (IEEE division), INT8
+ * rounded half-to-even and clamped to [-127, 127], E4M3 rounded to nearest
+ * even with saturation to +-448. Inputs must be finite.
+ * PER_TOKEN_BLOCK needs no workspace. The other kinds reduce amax across the
+ * whole grid and need `workspace`: a device buffer of at least
+ * fmha_quantize_workspace_bytes(...) bytes, 4-byte aligned, owned by the
+ * caller, not shared with a concurrent call; its contents on entry do not
+ * matter. workspace may be NULL when that size is 0.                        */
+fmha_status fmha_quantize_blockwise(const fmha_tensor* src, const fmha_tensor* dst, const fmha_sf* sf,
+                                    int32_t B, int32_t S, int32_t H, int32_t D,
+                                    void* workspace, size_t workspace_bytes, struct CUstream_st* stream);
+
+/* Workspace bytes fmha_quantize_blockwise needs for this granularity and shape. */
+size_t fmha_quantize_workspace_bytes(int32_t sf_kind, int32_t B, int32_t S, int32_t H, int32_t D);
+
+/* Dense attention (optionally causal) over contiguous K/V ([BW-FP8] intro). */
+fmha_status fmha_fwd(const fmha_args* args, struct CUstream_st* stream);
+
+/* Attention restricted by a 128x128 block mask ([PrimTS-BS] section 2).
+ *   mask: uint8, element (b, h_kv, i, j) at mask[b*mask_stride_b +
+ *   h_kv*mask_stride_h + i*ceil(Skv/128) + j], nonzero = the 128x128 block of
+ *   query rows [128i, 128i+128) x keys [128j, 128j+128) is visible (ANDed with
+ *   causal). Strides may be 0 to broadcast. Fully hidden rows give O = 0.    */
+fmha_status fmha_fwd_block_sparse(const fmha_args* args, const uint8_t* mask, int64_t mask_stride_b,
+                                  int64_t mask_stride_h, struct CUstream_st* stream);
+
+/* Attention over a paged K/V cache ([PrimTS-BS] section 2).
+ *   args->k / args->v describe the page POOL: element (page, t, h, d) at
+ *   ptr + page*stride_b + t*stride_s + h*stride_h + d, num_pages pages of
+ *   page_size tokens. Token s of sequence b is row s % page_size of pool page
+ *   page_table[b*max_pages_per_seq + s / page_size] (int32, device).
+ *   page_size must be 16, 32, 64 or 128. Every sequence has Skv tokens.
+ *   mask: optional block mask as in fmha_fwd_block_sparse (NULL = dense).
+ *   A page index outside [0, num_pages) reads zeros and is reported as
+ *   FMHA_ERR_DEVICE_INDEX by fmha_get_device_error().                       */
+fmha_status fmha_fwd_paged(const fmha_args* args, const int32_t* page_table, int32_t num_pages,
+                           int32_t page_size, int32_t max_pages_per_seq, const uint8_t* mask,
+                           int64_t mask_stride_b, int64_t mask_stride_h, struct CUstream_st* stream);
+
+/* Synchronises `stream`, then returns and clears the current device's error
+ * word: FMHA_OK, FMHA_ERR_TIMEOUT or FMHA_ERR_DEVICE_INDEX (or FMHA_ERR_CUDA if
+ * the synchronisation itself failed). */
+fmha_status fmha_get_device_error(struct CUstream_st* stream);
+
+/* Static string naming a status code. */
+const char* fmha_status_string(fmha_status status);
+
+/* One-line reason for the last non-OK status returned on this host thread. */
+const char* fmha_last_error_message(void);
+
+/* Test hook: sets the bound on every device-side wait, in GPU clock cycles,
+ * for launches made after the call (0 restores the default of about one
+ * second). Lets a test make a wait run out quickly. Process-wide.          */
+void fmha_set_wait_timeout_cycles(uint64_t cycles);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FMHA_H_ */

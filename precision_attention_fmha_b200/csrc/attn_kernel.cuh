@@ -1,0 +1,628 @@
+// attn_kernel.cuh -- warp-specialised FMHA forward for sm_100a.
+//
+// Computes O = softmax(scale * Q K^T) V on dequantized operands with an
+// online-softmax pass over 128-key tiles ("FlashInfer FP8/BF16 mixed-precision
+// attention for Blackwell", introduction and section 1: QK (BMM1) -> softmax ->
+// PV (BMM2); "FlashInfer DiT optimization: SageAttention and Int8/FP8
+// mixed-precision kernels", section 2: Q/K/P/V scale factors applied after the
+// 8-bit BMMs).
+//
+// One CTA owns two 128-row query tiles X = 0, 1 that share every K/V tile
+// (either two consecutive query blocks of one head, or the same query block
+// of two query heads that read the same KV head). 320 threads, one CTA/SM:
+//   warps 0-3  softmax for tile 0 (TMEM lanes 0-127: one query row per thread)
+//   warps 4-7  softmax for tile 1
+//   warp  8    tensor-core issue (one thread): S = Q K^T and O += P V
+//   warp  9    TMA producer (one thread): Q once, then K_j, V_j into a ring
+// TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D,256+2D).
+// The softmax writes P (BF16 or E4M3) over the first columns of its S tile and
+// the PV product reads P straight from TMEM, so P never touches shared memory.
+// Because the issue thread orders S_X(j+1) after PV_X(j), the arrival of
+// S_X(j+1) also proves PV_X(j) finished; the softmax warps therefore rescale O
+// themselves (only when the running row max grows by more than 2^tau, the
+// "lazy correction" of the Blackwell page, section 3) before releasing P_X(j+1).
+// The epilogue scales O by 1/l (and the V / P scale factors), converts to BF16,
+// stages 64-column halves in the dead Q buffer and writes them with TMA stores
+// ("FlashInfer DeepSeek-V4 sparse-MLA: Cake backend", section 1: output through
+// a TMA descriptor passed as a grid constant).
+//
+// Every wait is bounded: on expiry the thread sets the device error word and a
+// CTA-wide abort flag; all roles then fall through to a teardown that drains
+// in-flight TMA loads and MMAs before TMEM is freed. Nothing traps.
+#pragma once
+
+#include "fmha_internal.h"
+#include "ptx_sm100.cuh"
+
+namespace fmha {
+
+template <int D_, int QK_, int PV_, bool PAGED_>
+struct AttnCfg {
+  static constexpr int D = D_, QK = QK_, PV = PV_;
+  static constexpr bool PAGED = PAGED_;
+  static constexpr int BM = 128, BN = 128;
+  static constexpr int QK_ELEM = QK == QK_BF16 ? 2 : 1;
+  static constexpr int V_ELEM = PV == PV_BF16 ? 2 : 1;
+  static constexpr int QK_ROW_BYTES = D * QK_ELEM;
+  static constexpr int QK_CHUNKS = QK_ROW_BYTES / 128;  // 128-byte swizzle columns along D
+  static constexpr int QK_CHUNK_ELEMS = 128 / QK_ELEM;
+  static constexpr int V_CHUNKS = D * V_ELEM / 128;
+  static constexpr int V_CHUNK_ELEMS = 128 / V_ELEM;
+  static_assert(QK_ROW_BYTES % 128 == 0 && (D * V_ELEM) % 128 == 0, "rows must be whole 128-byte atoms");
+  static constexpr int CHUNK_BYTES = 128 * 128;  // one 128-row x 128-byte swizzled column block
+  static constexpr int Q_TILE = BM * QK_ROW_BYTES;
+  static constexpr int K_TILE = BN * QK_ROW_BYTES;
+  static constexpr int V_TILE = BN * D * V_ELEM;
+  static constexpr int SLOT = K_TILE > V_TILE ? K_TILE : V_TILE;
+  static constexpr int MISC_BYTES = 1024;
+  static constexpr int SMEM_CAP = 232448;  // 227 KB opt-in maximum per CTA
+  static constexpr int STAGES_FIT = (SMEM_CAP - 1024 - MISC_BYTES - 2 * Q_TILE) / SLOT;
+  static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
+  static_assert(STAGES >= 3, "the K/V ring needs at least three slots");
+  static constexpr int SMEM_BYTES = 1024 + 2 * Q_TILE + STAGES * SLOT + MISC_BYTES;
+  static constexpr int QK_STEPS = QK_ROW_BYTES / 32;  // one MMA covers 32 bytes of K (16 bf16 / 32 8-bit)
+  static constexpr int PV_K = PV == PV_BF16 ? 16 : 32;
+  static constexpr int PV_STEPS = BN / PV_K;
+  static constexpr int O_STAGE_BUFS = Q_TILE / CHUNK_BYTES;  // 16 KB staging buffers inside a Q buffer
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t IDESC_QK = QK == QK_BF16   ? ptx::make_idesc(1, 1, 1, 0, 0, BN, BM)
+                                       : QK == QK_E4M3 ? ptx::make_idesc(1, 0, 0, 0, 0, BN, BM)
+                                                       : ptx::make_idesc(2, 1, 1, 0, 0, BN, BM);
+  static constexpr uint32_t IDESC_PV =
+      PV == PV_BF16 ? ptx::make_idesc(1, 1, 1, 0, 1, D, BM) : ptx::make_idesc(1, 0, 0, 0, 1, D, BM);
+  static constexpr int THREADS = 320;
+};
+
+struct alignas(8) AttnMisc {
+  uint64_t q_full;
+  uint64_t s_full[2];
+  uint64_t p_full[2];
+  uint64_t o_full;
+  uint64_t drain;
+  uint64_t kv_full[8];
+  uint64_t kv_empty[8];
+  uint32_t tmem_base;
+  volatile uint32_t abort;
+  float sf_v[128];
+};
+
+struct TileInfo {
+  int h;      // query head
+  int q0;     // first query row
+  int qblk;   // 128-row query block index
+  int n_kv;   // KV tiles [0, n_kv) not excluded by causality / length
+  bool valid;
+};
+
+// Bounded mbarrier wait. Returns false on timeout (recorded) or CTA abort.
+struct Waiter {
+  volatile uint32_t* abort_flag;
+  uint32_t* err;
+  uint64_t budget;
+  __device__ __forceinline__ bool wait(uint32_t bar, uint32_t parity) const {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (true) {
+      if (ptx::mbar_try_wait(bar, parity)) return true;
+      if (*abort_flag) return false;
+      if (static_cast<uint64_t>(clock64() - t0) > budget) {
+        *abort_flag = 1u;
+        atomicOr(err, kErrTimeout);
+        return false;
+      }
+    }
+  }
+  // Teardown wait: ignores the abort flag (used to drain in-flight async work).
+  __device__ __forceinline__ bool drain(uint32_t bar, uint32_t parity) const {
+    const long long t0 = clock64();
+    while (!ptx::mbar_try_wait(bar, parity)) {
+      if (static_cast<uint64_t>(clock64() - t0) > budget) {
+        atomicOr(err, kErrTimeout);
+        return false;
+      }
+    }
+    return true;
+  }
+};
+
+__device__ __forceinline__ bool keep_tile(const AttnParams& p, const TileInfo& t, int b, int hkv, int u) {
+  if (u >= t.n_kv) return false;
+  if (p.mask == nullptr) return true;
+  return p.mask[b * p.mask_sb + hkv * p.mask_sh + static_cast<int64_t>(t.qblk) * p.n_kv_blocks + u] != 0;
+}
+
+__device__ __forceinline__ float sf_lookup(const float* sf, int kind, int64_t bh, int nblk, int idx_in_seq,
+                                           int rpb) {
+  switch (kind) {
+    case FMHA_SF_PER_TENSOR: return sf[0];
+    case FMHA_SF_PER_HEAD: return sf[bh];
+    case FMHA_SF_PER_TOKEN_BLOCK: return sf[bh * nblk + idx_in_seq / rpb];
+    default: return 1.f;
+  }
+}
+
+// ------------------------------------------------------------ TMA producer --
+template <class C>
+__device__ void attn_load_role(const AttnParams& p, const TileInfo (&t)[2], int b, int hkv, uint8_t* const (&sQ)[2],
+                               uint8_t* sSlots, AttnMisc* misc, const CUtensorMap* tmQ, const CUtensorMap* tmK,
+                               const CUtensorMap* tmV, const Waiter& w) {
+  using namespace ptx;
+  const uint32_t q_full = smem_addr(&misc->q_full);
+  uint32_t qbytes = 0;
+  for (int x = 0; x < 2; ++x) qbytes += t[x].valid ? C::Q_TILE : 0;
+  mbar_arrive_expect_tx(q_full, qbytes);
+  for (int x = 0; x < 2; ++x) {
+    if (!t[x].valid) continue;
+#pragma unroll
+    for (int c = 0; c < C::QK_CHUNKS; ++c)
+      tma_load_4d(smem_addr(sQ[x]) + c * C::CHUNK_BYTES, tmQ, q_full, c * C::QK_CHUNK_ELEMS, t[x].h, t[x].q0, b);
+  }
+  const uint64_t pol = policy_evict_last();  // K/V tiles are re-read by every CTA of this head
+  int last_phase[8];
+#pragma unroll
+  for (int s = 0; s < 8; ++s) last_phase[s] = -1;
+  int slot_it = 0;
+  const int n_u = max(t[0].n_kv, t[1].n_kv);
+  bool ok = true;
+  for (int u = 0; u < n_u && ok; ++u) {
+    if (!keep_tile(p, t[0], b, hkv, u) && !keep_tile(p, t[1], b, hkv, u)) continue;
+    for (int kv = 0; kv < 2; ++kv) {  // K then V
+      const int s = slot_it % C::STAGES;
+      const uint32_t ph = (slot_it / C::STAGES) & 1;
+      ++slot_it;
+      if (!w.wait(smem_addr(&misc->kv_empty[s]), ph ^ 1)) { ok = false; break; }
+      const uint32_t full = smem_addr(&misc->kv_full[s]);
+      const int chunks = kv == 0 ? C::QK_CHUNKS : C::V_CHUNKS;
+      const int chunk_elems = kv == 0 ? C::QK_CHUNK_ELEMS : C::V_CHUNK_ELEMS;
+      const CUtensorMap* tm = kv == 0 ? tmK : tmV;
+      const uint32_t dst = smem_addr(sSlots + s * C::SLOT);
+      mbar_arrive_expect_tx(full, kv == 0 ? C::K_TILE : C::V_TILE);
+      last_phase[s] = static_cast<int>(ph);
+      if constexpr (!C::PAGED) {
+        for (int c = 0; c < chunks; ++c)
+          tma_load_4d_hint(dst + c * C::CHUNK_BYTES, tm, full, c * chunk_elems, hkv, u * C::BN, b, pol);
+      } else {
+        const int per = C::BN / p.page_size;
+        for (int pp = 0; pp < per; ++pp) {
+          const int lp = (u * C::BN) / p.page_size + pp;  // logical page of this sequence
+          int page = p.num_pages;                          // out of range: TMA fills zeros
+          if (lp * p.page_size < p.Skv) {
+            const int e = p.page_table[static_cast<int64_t>(b) * p.max_pages_per_seq + lp];
+            if (e >= 0 && e < p.num_pages)
+              page = e;
+            else
+              atomicOr(p.err, kErrPageIndex);
+          }
+          for (int c = 0; c < chunks; ++c)
+            tma_load_4d_hint(dst + c * C::CHUNK_BYTES + pp * p.page_size * 128, tm, full, c * chunk_elems, hkv, 0,
+                             page, pol);
+        }
+      }
+    }
+  }
+  if (*w.abort_flag) {  // let every issued copy land before shared memory goes away
+    w.drain(q_full, 0);
+    for (int s = 0; s < C::STAGES; ++s)
+      if (last_phase[s] >= 0) w.drain(smem_addr(&misc->kv_full[s]), static_cast<uint32_t>(last_phase[s]));
+  }
+}
+
+// ------------------------------------------------------- tensor-core issue --
+template <class C>
+__device__ __forceinline__ void issue_qk(uint32_t tmem_d, uint32_t q_smem, uint32_t k_smem) {
+#pragma unroll
+  for (int s = 0; s < C::QK_STEPS; ++s) {
+    const uint32_t off = (s / 4) * C::CHUNK_BYTES + (s % 4) * 32;
+    const uint64_t a = ptx::smem_desc(q_smem + off, 16, 1024, 2);
+    const uint64_t bd = ptx::smem_desc(k_smem + off, 16, 1024, 2);
+    if constexpr (C::QK == QK_BF16)
+      ptx::mma_ss_f16(tmem_d, a, bd, C::IDESC_QK, s > 0);
+    else if constexpr (C::QK == QK_E4M3)
+      ptx::mma_ss_f8(tmem_d, a, bd, C::IDESC_QK, s > 0);
+    else
+      ptx::mma_ss_i8(tmem_d, a, bd, C::IDESC_QK, s > 0);
+  }
+}
+
+template <class C>
+__device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint32_t v_smem, bool accumulate) {
+#pragma unroll
+  for (int s = 0; s < C::PV_STEPS; ++s) {
+    // V is MN-major (d contiguous): K-step s starts PV_K rows down; the 64/128-wide
+    // d columns are CHUNK_BYTES apart (leading byte offset), 8-row groups 1 KB apart.
+    const uint64_t bd = ptx::smem_desc(v_smem + s * C::PV_K * 128, C::CHUNK_BYTES, 1024, 2);
+    const uint32_t a = tmem_p + s * 8;  // 8 TMEM columns = 16 bf16 / 32 e4m3 of P
+    if constexpr (C::PV == PV_BF16)
+      ptx::mma_ts_f16(tmem_o, a, bd, C::IDESC_PV, (accumulate || s > 0) ? 1u : 0u);
+    else
+      ptx::mma_ts_f8(tmem_o, a, bd, C::IDESC_PV, (accumulate || s > 0) ? 1u : 0u);
+  }
+}
+
+template <class C>
+__device__ void attn_mma_role(const AttnParams& p, const TileInfo (&t)[2], int b, int hkv, uint8_t* const (&sQ)[2],
+                              uint8_t* sSlots, AttnMisc* misc, uint32_t tmem, const Waiter& w) {
+  using namespace ptx;
+  const uint32_t s_col[2] = {0u, 128u};
+  const uint32_t o_col[2] = {256u, 256u + C::D};
+  int pend[2] = {-1, -1};
+  int pv_cnt[2] = {0, 0};
+  int prev_v = -1;
+  int slot_it = 0;
+  const int n_u = max(t[0].n_kv, t[1].n_kv);
+  bool ok = w.wait(smem_addr(&misc->q_full), 0);
+  tc_fence_after();
+  for (int u = 0; u < n_u && ok; ++u) {
+    const bool kx[2] = {keep_tile(p, t[0], b, hkv, u), keep_tile(p, t[1], b, hkv, u)};
+    if (!kx[0] && !kx[1]) continue;
+    const int ks = slot_it % C::STAGES;
+    const uint32_t kph = (slot_it / C::STAGES) & 1;
+    ++slot_it;
+    const int vs = slot_it % C::STAGES;
+    const uint32_t vph = (slot_it / C::STAGES) & 1;
+    ++slot_it;
+    bool k_ready = false;
+    for (int x = 0; x < 2 && ok; ++x) {
+      if (pend[x] >= 0) {  // PV of the previous tile first: S_x(u) overwrites P_x
+        if (!(ok = w.wait(smem_addr(&misc->p_full[x]), pv_cnt[x] & 1))) break;
+        tc_fence_after();
+        issue_pv<C>(tmem + o_col[x], tmem + s_col[x], smem_addr(sSlots + pend[x] * C::SLOT), pv_cnt[x] > 0);
+        ++pv_cnt[x];
+        pend[x] = -1;
+      }
+      if (kx[x]) {
+        if (!k_ready) {
+          if (!(ok = w.wait(smem_addr(&misc->kv_full[ks]), kph))) break;
+          tc_fence_after();
+          k_ready = true;
+        }
+        issue_qk<C>(tmem + s_col[x], smem_addr(sQ[x]), smem_addr(sSlots + ks * C::SLOT));
+        tc_commit(smem_addr(&misc->s_full[x]));
+      }
+    }
+    if (!ok) break;
+    tc_commit(smem_addr(&misc->kv_empty[ks]));                     // K_u free once the S MMAs finish
+    if (prev_v >= 0) tc_commit(smem_addr(&misc->kv_empty[prev_v]));  // previous V: its PVs are issued
+    if (!(ok = w.wait(smem_addr(&misc->kv_full[vs]), vph))) break;
+    tc_fence_after();
+    pend[0] = kx[0] ? vs : -1;
+    pend[1] = kx[1] ? vs : -1;
+    prev_v = vs;
+  }
+  for (int x = 0; x < 2 && ok; ++x) {
+    if (pend[x] < 0) continue;
+    if (!(ok = w.wait(smem_addr(&misc->p_full[x]), pv_cnt[x] & 1))) break;
+    tc_fence_after();
+    issue_pv<C>(tmem + o_col[x], tmem + s_col[x], smem_addr(sSlots + pend[x] * C::SLOT), pv_cnt[x] > 0);
+  }
+  if (ok) tc_commit(smem_addr(&misc->o_full));
+  // Drain: arrives when every MMA issued above has completed.
+  tc_commit(smem_addr(&misc->drain));
+  w.drain(smem_addr(&misc->drain), 0);
+}
+
+// --------------------------------------------------------------- softmax ----
+template <class C>
+__device__ void attn_softmax_role(const AttnParams& p, const TileInfo& t, int x, int b, int hkv, uint8_t* sQx,
+                                  AttnMisc* misc, uint32_t tmem, const CUtensorMap* tmO, const Waiter& w) {
+  using namespace ptx;
+  constexpr uint32_t FULL = 0xffffffffu;
+  const int warp = (threadIdx.x >> 5) & 3;  // TMEM lane quadrant of this warp
+  const int lane = threadIdx.x & 31;
+  const int r = warp * 32 + lane;  // row within the tile
+  const int row = t.q0 + r;        // query row
+  const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+  const uint32_t tS = tmem + lane_off + (x ? 128u : 0u);
+  const uint32_t tO = tmem + lane_off + (x ? 256u + C::D : 256u);
+  const int wg_tid = threadIdx.x & 127;
+  const int64_t bhq = static_cast<int64_t>(b) * p.Hq + t.h;
+  const int64_t bhk = static_cast<int64_t>(b) * p.Hkv + hkv;
+
+  // Row factor: softmax scale * log2(e) * Q scale of this row.
+  float cq = p.scale_log2;
+  if (C::QK != QK_BF16) cq *= sf_lookup(p.sf_q, p.sf_q_kind, bhq, p.sf_q_nblk, min(row, p.Sq - 1), p.sf_q_rpb);
+  const float ck_uniform =
+      p.sf_k_kind == FMHA_SF_PER_TOKEN_BLOCK ? 1.f : sf_lookup(p.sf_k, p.sf_k_kind, bhk, 1, 0, 1);
+
+  // P encoding: E4M3 P holds p * g with g = 1 / sf_p; the lazy-rescale
+  // threshold tau keeps the stale-max bound 2^tau * g <= 448. BF16 P: g = 1, tau = 8.
+  float log2g = 0.f;
+  float tau = 8.f;
+  if constexpr (C::PV == PV_E4M3) {
+    float sfp = 1.f / 16.f;
+    if (p.sf_p_kind == FMHA_SF_PER_TENSOR) sfp = p.sf_p[0];
+    if (p.sf_p_kind == FMHA_SF_PER_TOKEN_BLOCK) sfp = p.sf_p[bhq * p.sf_p_nblk + t.q0 / p.sf_p_rpb];
+    log2g = -__log2f(sfp);
+    tau = fminf(8.f, fmaxf(0.f, floorf(__log2f(448.f * sfp))));
+  }
+
+  float m = -INFINITY;  // running row max (log2 units, scaled)
+  float l = 0.f;        // running row sum of the stored P (times g)
+  int it = 0;
+  bool ok = true;
+  for (int u = 0; u < t.n_kv; ++u) {
+    if (!keep_tile(p, t, b, hkv, u)) continue;
+    ok = __all_sync(FULL, w.wait(smem_addr(&misc->s_full[x]), it & 1));
+    if (!ok) break;
+    tc_fence_after();
+    uint32_t s[4][32];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, s[c]);
+    tmem_wait_ld();
+#pragma unroll
+    for (int c = 0; c < 4; ++c) reg_fence(s[c]);
+
+    // Column factors: K scale per 32-key chunk (token-block K scales), times cq.
+    const int kv0 = u * C::BN;
+    float ck[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      float f = ck_uniform;
+      if (C::QK != QK_BF16 && p.sf_k_kind == FMHA_SF_PER_TOKEN_BLOCK)
+        f = p.sf_k[bhk * p.sf_k_nblk + min(kv0 + 32 * c, p.Skv - 1) / p.sf_k_rpb];
+      ck[c] = f * cq;
+    }
+    // Raw scores as fp32 (INT8 products are exact s32 < 2^22: magic-number conversion).
+    float f[4][32];
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        if constexpr (C::QK == QK_INT8)
+          f[c][j] = __int_as_float(static_cast<int>(s[c][j]) + 0x4B400000) - 12582912.f;
+        else
+          f[c][j] = __uint_as_float(s[c][j]);
+      }
+    // Mask keys past the sequence end and (causal) past the diagonal.
+    int lim = p.Skv - kv0;
+    if (p.causal) lim = min(lim, row + 1 + (p.Skv - p.Sq) - kv0);
+    if (lim < C::BN) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          if (32 * c + j >= lim) f[c][j] = -INFINITY;
+    }
+    float m_tile = -INFINITY;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      float mc = f[c][0];
+#pragma unroll
+      for (int j = 1; j < 32; ++j) mc = fmaxf(mc, f[c][j]);
+      m_tile = fmaxf(m_tile, mc * ck[c]);
+    }
+    const float m_new = fmaxf(m, m_tile);
+    float alpha = 1.f;
+    bool resc = false;
+    if (it == 0) {
+      m = m_new;
+    } else if (m_new > m + tau) {
+      alpha = ex2(m - m_new);
+      resc = true;
+      m = m_new;
+      l *= alpha;
+    }
+    if (__any_sync(FULL, resc)) {  // lazy O correction, whole warp (tcgen05.ld/st are warp-wide)
+#pragma unroll 1
+      for (int c = 0; c < C::D / 32; ++c) {
+        uint32_t o[32];
+        tmem_ld32(tO + 32 * c, o);
+        tmem_wait_ld();
+        reg_fence(o);
+#pragma unroll
+        for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+        tmem_st32(tO + 32 * c, o);
+      }
+    }
+    const float mb = (m == -INFINITY ? 0.f : m) - log2g;
+    float rs = 0.f;
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+#pragma unroll
+      for (int j = 0; j < 32; ++j) {
+        f[c][j] = ex2(fmaf(f[c][j], ck[c], -mb));
+        rs += f[c][j];
+      }
+    l += rs;
+    if constexpr (C::PV == PV_BF16) {
+      uint32_t pk[2][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int j = 0; j < 16; ++j) pk[c >> 1][(c & 1) * 16 + j] = pack_bf16x2(f[c][2 * j], f[c][2 * j + 1]);
+      tmem_st32(tS, pk[0]);
+      tmem_st32(tS + 32, pk[1]);
+    } else {
+      uint32_t pk[32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          pk[c * 8 + j] =
+              pack_e4m3x2(f[c][4 * j], f[c][4 * j + 1]) | (pack_e4m3x2(f[c][4 * j + 2], f[c][4 * j + 3]) << 16);
+      tmem_st32(tS, pk);
+    }
+    tmem_wait_st();
+    tc_fence_before();
+    mbar_arrive(smem_addr(&misc->p_full[x]));
+    ++it;
+  }
+
+  // ---- epilogue ----
+  bool have_o = false;
+  if (ok) ok = __all_sync(FULL, w.wait(smem_addr(&misc->q_full), 0));  // Q buffer (our staging) has landed
+  if (ok && it > 0) {
+    ok = __all_sync(FULL, w.wait(smem_addr(&misc->o_full), 0));
+    tc_fence_after();
+    have_o = ok;
+  }
+  float sfv = 1.f;
+  if (C::PV == PV_E4M3 && p.sf_v_kind != FMHA_SF_PER_CHANNEL) sfv = sf_lookup(p.sf_v, p.sf_v_kind, bhk, 1, 0, 1);
+  const float inv_l = l > 0.f ? sfv / l : 0.f;
+  const uint32_t stage0 = smem_addr(sQx);
+#pragma unroll 1
+  for (int c64 = 0; c64 < C::D / 64; ++c64) {
+    uint32_t o[2][32];
+    if (have_o) {
+      tmem_ld32(tO + 64 * c64, o[0]);
+      tmem_ld32(tO + 64 * c64 + 32, o[1]);
+      tmem_wait_ld();
+      reg_fence(o[0]);
+      reg_fence(o[1]);
+    }
+    uint32_t pk[32];
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      float a = have_o ? __uint_as_float(o[j >> 4][(2 * j) & 31]) * inv_l : 0.f;
+      float bb = have_o ? __uint_as_float(o[j >> 4][(2 * j + 1) & 31]) * inv_l : 0.f;
+      if (C::PV == PV_E4M3 && p.sf_v_kind == FMHA_SF_PER_CHANNEL) {
+        a *= misc->sf_v[64 * c64 + 2 * j];
+        bb *= misc->sf_v[64 * c64 + 2 * j + 1];
+      }
+      pk[j] = pack_bf16x2(a, bb);
+    }
+    const int buf = c64 % C::O_STAGE_BUFS;
+    if (c64 >= C::O_STAGE_BUFS) {  // buffer reuse: the previous store must have read it
+      if (wg_tid == 0) bulk_wait_read0();
+      named_bar_sync(1 + x, 128);
+    }
+    const uint32_t base = stage0 + buf * C::CHUNK_BYTES + r * 128;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const uint32_t addr = base + ((k ^ (r & 7)) << 4);
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[4 * k]), "r"(pk[4 * k + 1]),
+                   "r"(pk[4 * k + 2]), "r"(pk[4 * k + 3])
+                   : "memory");
+    }
+    fence_proxy_async_smem();
+    named_bar_sync(1 + x, 128);
+    if (wg_tid == 0 && ok) {
+      tma_store_4d(tmO, stage0 + buf * C::CHUNK_BYTES, 64 * c64, t.h, t.q0, b);
+      bulk_commit();
+    }
+  }
+  if (p.lse != nullptr && row < p.Sq && ok) {
+    const float lse = l > 0.f ? (m + __log2f(l) - log2g) * 0.69314718055994531f : -INFINITY;
+    p.lse[bhq * p.Sq + row] = lse;
+  }
+  if (wg_tid == 0) bulk_wait0();
+}
+
+// ------------------------------------------------------------------ kernel --
+template <class C>
+__global__ void __launch_bounds__(C::THREADS, 1)
+    attn_fwd_kernel(const __grid_constant__ AttnParams p, const __grid_constant__ CUtensorMap tmQ,
+                    const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
+                    const __grid_constant__ CUtensorMap tmO) {
+  using namespace ptx;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* const sQ[2] = {smem, smem + C::Q_TILE};
+  uint8_t* sSlots = smem + 2 * C::Q_TILE;
+  AttnMisc* misc = reinterpret_cast<AttnMisc*>(sSlots + C::STAGES * C::SLOT);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // ---- work item -> (b, heads, query rows) ----
+  int b, hkv;
+  TileInfo t[2];
+  {
+    int item = blockIdx.x;
+    if (p.pair_mode == PAIR_ROWS) {
+      int pr = item % p.n_units;
+      item /= p.n_units;
+      const int h = item % p.Hq;
+      b = item / p.Hq;
+      if (p.causal) pr = p.n_units - 1 - pr;  // heaviest causal tiles first
+      for (int x = 0; x < 2; ++x) {
+        t[x].h = h;
+        t[x].qblk = 2 * pr + x;
+      }
+    } else {
+      int qb = item % p.n_units;
+      item /= p.n_units;
+      const int hp = item % (p.Hq / 2);
+      b = item / (p.Hq / 2);
+      if (p.causal) qb = p.n_units - 1 - qb;
+      for (int x = 0; x < 2; ++x) {
+        t[x].h = 2 * hp + x;
+        t[x].qblk = qb;
+      }
+    }
+    hkv = t[0].h / p.group;
+    for (int x = 0; x < 2; ++x) {
+      t[x].q0 = t[x].qblk * C::BM;
+      t[x].valid = t[x].q0 < p.Sq;
+      int n = p.n_kv_blocks;
+      if (p.causal) {
+        const int last = min(t[x].q0 + C::BM - 1, p.Sq - 1) + (p.Skv - p.Sq);
+        n = last < 0 ? 0 : min(p.n_kv_blocks, last / C::BN + 1);
+      }
+      t[x].n_kv = t[x].valid ? n : 0;
+    }
+  }
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_addr(&misc->q_full), 1);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(smem_addr(&misc->s_full[x]), 1);
+      mbar_init(smem_addr(&misc->p_full[x]), 128);
+    }
+    mbar_init(smem_addr(&misc->o_full), 1);
+    mbar_init(smem_addr(&misc->drain), 1);
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(smem_addr(&misc->kv_full[s]), 1);
+      mbar_init(smem_addr(&misc->kv_empty[s]), 1);
+    }
+    misc->abort = 0u;
+    fence_barrier_init();
+  }
+  if (C::PV == PV_E4M3 && p.sf_v_kind == FMHA_SF_PER_CHANNEL && threadIdx.x < C::D)
+    misc->sf_v[threadIdx.x] = p.sf_v[(static_cast<int64_t>(b) * p.Hkv + hkv) * C::D + threadIdx.x];
+  if (warp == 8) {
+    tmem_alloc(smem_addr(&misc->tmem_base), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 9 && lane == 0) {
+    prefetch_tmap(&tmQ);
+    prefetch_tmap(&tmK);
+    prefetch_tmap(&tmV);
+    prefetch_tmap(&tmO);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = misc->tmem_base;
+  const Waiter w{&misc->abort, p.err, p.wait_cycles};
+
+  if (warp < 8) {
+    const int x = warp >> 2;
+    if (t[x].valid) attn_softmax_role<C>(p, t[x], x, b, hkv, sQ[x], misc, tmem, &tmO, w);
+  } else if (warp == 8) {
+    if (lane == 0) attn_mma_role<C>(p, t, b, hkv, sQ, sSlots, misc, tmem, w);
+    __syncwarp();
+  } else {
+    if (lane == 0) attn_load_role<C>(p, t, b, hkv, sQ, sSlots, misc, &tmQ, &tmK, &tmV, w);
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 8) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+template <class C>
+cudaError_t launch_attention_t(const AttnParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
+                               const CUtensorMap& tv, const CUtensorMap& to, cudaStream_t stream) {
+  auto kern = attn_fwd_kernel<C>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  const int head_units = p.pair_mode == PAIR_ROWS ? p.Hq : p.Hq / 2;
+  const long long blocks = static_cast<long long>(p.n_units) * head_units * p.B;
+  kern<<<static_cast<unsigned>(blocks), C::THREADS, C::SMEM_BYTES, stream>>>(p, tq, tk, tv, to);
+  return cudaGetLastError();
+}
+
+}  // namespace fmha

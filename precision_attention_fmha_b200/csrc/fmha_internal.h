@@ -1,0 +1,66 @@
+// fmha_internal.h -- structures shared by the host launchers and the kernels
+// of libfmha.so. Not part of the public ABI (that is include/fmha.h).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/fmha.h"
+
+namespace fmha {
+
+// Device error word bits (one word per device, see api.cu).
+enum : uint32_t { kErrTimeout = 1u, kErrPageIndex = 2u };
+
+// Default bound on one device-side wait (GPU clock cycles, ~1 s at 2 GHz).
+constexpr uint64_t kDefaultWaitCycles = 2000000000ull;
+
+// Operand kinds of the two tensor-core products.
+enum QkKind : int { QK_BF16 = 0, QK_E4M3 = 1, QK_INT8 = 2 };
+enum PvKind : int { PV_BF16 = 0, PV_E4M3 = 1 };
+
+// How a CTA's two 128-row query tiles are chosen.
+enum PairMode : int {
+  PAIR_ROWS = 0,   // query blocks 2i and 2i+1 of one head
+  PAIR_HEADS = 1,  // one query block of heads 2j and 2j+1 (same KV head)
+};
+
+struct AttnParams {
+  int32_t B, Hq, Hkv, Sq, Skv, group;
+  int32_t n_q_blocks;   // ceil(Sq / 128)
+  int32_t n_kv_blocks;  // ceil(Skv / 128)
+  int32_t pair_mode;
+  int32_t n_units;      // work items per (b, head unit): pairs of q blocks (PAIR_ROWS) or q blocks (PAIR_HEADS)
+  int32_t causal;
+  float scale_log2;     // softmax_scale * log2(e)
+  // scale factors (dequantization multipliers), kinds from fmha_sf_kind
+  const float* sf_q; int32_t sf_q_kind; int32_t sf_q_rpb; int32_t sf_q_nblk;
+  const float* sf_k; int32_t sf_k_kind; int32_t sf_k_rpb; int32_t sf_k_nblk;
+  const float* sf_v; int32_t sf_v_kind;
+  const float* sf_p; int32_t sf_p_kind; int32_t sf_p_rpb; int32_t sf_p_nblk;
+  float* lse;           // nullable [B, Hq, Sq]
+  // block mask (nullable): byte (b, hkv, i, j) at mask[b*mask_sb + hkv*mask_sh + i*n_kv_blocks + j]
+  const uint8_t* mask; int64_t mask_sb, mask_sh;
+  // paged K/V (page_table == nullptr: contiguous)
+  const int32_t* page_table; int32_t num_pages, page_size, max_pages_per_seq;
+  uint32_t* err;        // device error word
+  uint64_t wait_cycles; // bound on one wait
+};
+
+struct QuantParams {
+  const uint16_t* src; int64_t s_sb, s_ss, s_sh;  // bf16 bits
+  uint8_t* dst; int64_t d_sb, d_ss, d_sh;         // int8 / e4m3 bytes
+  float* sf; int32_t kind; int32_t rpb; int32_t nblk;
+  int32_t B, S, H, D;
+  uint32_t* ws;          // amax accumulators (float bits) for the grid-wide kinds
+  int32_t rows_per_cta;  // grid-wide kinds: token rows per CTA
+};
+
+// Launchers (defined in the .cu files). They return cudaSuccess or the launch error.
+cudaError_t launch_attention(int qk_kind, int pv_kind, int D, bool paged, const AttnParams& p,
+                             const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                             const CUtensorMap& to, cudaStream_t stream);
+cudaError_t launch_quantize(bool to_e4m3, const QuantParams& p, cudaStream_t stream);
+
+}  // namespace fmha
