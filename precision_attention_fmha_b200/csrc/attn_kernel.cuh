@@ -415,33 +415,41 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo& t, int x,
       }
     }
     const float mb = (m == -INFINITY ? 0.f : m) - log2g;
-    float rs = 0.f;
 #pragma unroll
     for (int c = 0; c < 4; ++c)
 #pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        f[c][j] = ex2(fmaf(f[c][j], ck[c], -mb));
-        rs += f[c][j];
-      }
-    l += rs;
+      for (int j = 0; j < 32; ++j) f[c][j] = ex2(fmaf(f[c][j], ck[c], -mb));
+    float rs = 0.f;
     if constexpr (C::PV == PV_BF16) {
       uint32_t pk[2][32];
 #pragma unroll
       for (int c = 0; c < 4; ++c)
 #pragma unroll
-        for (int j = 0; j < 16; ++j) pk[c >> 1][(c & 1) * 16 + j] = pack_bf16x2(f[c][2 * j], f[c][2 * j + 1]);
+        for (int j = 0; j < 16; ++j) {
+          pk[c >> 1][(c & 1) * 16 + j] = pack_bf16x2(f[c][2 * j], f[c][2 * j + 1]);
+          rs += f[c][2 * j] + f[c][2 * j + 1];
+        }
       tmem_st32(tS, pk[0]);
       tmem_st32(tS + 32, pk[1]);
     } else {
+      // The row sum adds the E4M3-rounded values actually stored, so the
+      // normalised weights sum to one and a dominant key returns its value.
       uint32_t pk[32];
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+      for (int c = 0; c < 4; ++c) {
+        uint32_t acc = 0u;  // f16x2 zero
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          pk[c * 8 + j] =
-              pack_e4m3x2(f[c][4 * j], f[c][4 * j + 1]) | (pack_e4m3x2(f[c][4 * j + 2], f[c][4 * j + 3]) << 16);
+        for (int j = 0; j < 8; ++j) {
+          const uint32_t lo = pack_e4m3x2(f[c][4 * j], f[c][4 * j + 1]);
+          const uint32_t hi = pack_e4m3x2(f[c][4 * j + 2], f[c][4 * j + 3]);
+          pk[c * 8 + j] = lo | (hi << 16);
+          acc = hadd2(acc, hadd2(e4m3x2_to_f16x2(lo), e4m3x2_to_f16x2(hi)));
+        }
+        rs += f16x2_sum(acc);
+      }
       tmem_st32(tS, pk);
     }
+    l += rs;
     tmem_wait_st();
     tc_fence_before();
     mbar_arrive(smem_addr(&misc->p_full[x]));

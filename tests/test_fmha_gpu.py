@@ -76,7 +76,9 @@ def run_dense(mode, B, Hq, Hkv, Sq, Skv, D, causal, seed, with_lse=False):
     g, rq, rk, rv = prepare(mode, q.contiguous(), k.contiguous(), v.contiguous())
     scale = 1 / math.sqrt(D)
     lse = torch.full((B, Hq, Sq), float("nan"), device=DEV) if with_lse else None
-    sf_p = Scale(torch.ones(B, Hq, math.ceil(Sq / 128), device=DEV), "per_token_block", 128) if mode == "sage" else None
+    sf_p = None
+    if mode == "sage":  # per-row-block P scale: P is stored as 16 p (lazy-rescale bound 2^4 * 16 <= 448)
+        sf_p = Scale(torch.full((B, Hq, math.ceil(Sq / 128)), 1 / 16, device=DEV), "per_token_block", 128)
     o = fmha.fmha_fwd(g["q"], g["k"], g["v"], sf_q=g["sf_q"], sf_k=g["sf_k"], sf_v=g["sf_v"], sf_p=sf_p,
                       softmax_scale=scale, causal=causal, lse=lse)
     fmha.get_device_error()
