@@ -114,7 +114,10 @@ typedef struct {
  *   causal != 0: key j is visible to query i iff j <= i + (Skv - Sq)
  *   (bottom-right aligned).
  *   lse (nullable): fp32 [B, Hq, Sq], natural-log log-sum-exp of the scaled
- *   scores; -inf for a row with no visible key (whose O row is 0).
+ *   scores; -inf for a row with no visible key (whose O row is 0). When P is
+ *   cast to E4M3 (8-bit V) the sum runs over the stored, rounded P values --
+ *   the same normaliser O uses, so partial results merge exactly -- and lse
+ *   then differs from the exact value by at most ln(1 + 2^-4) ~ 0.061.
  * Supported (q, k, v, o) dtype tuples: (BF16, BF16, BF16, BF16),
  * (BF16, BF16, E4M3, BF16) ("QK-BF16/PV-FP8", [BW-FP8]),
  * (E4M3, E4M3, E4M3, BF16) ("all-FP8", [BW-FP8]), (INT8, INT8, E4M3, BF16)

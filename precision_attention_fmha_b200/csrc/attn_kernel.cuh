@@ -9,11 +9,13 @@
 //
 // One CTA owns two 128-row query tiles X = 0, 1 that share every K/V tile
 // (either two consecutive query blocks of one head, or the same query block
-// of two query heads that read the same KV head). 320 threads, one CTA/SM:
+// of two query heads that read the same KV head). 384 threads, one CTA/SM:
 //   warps 0-3  softmax for tile 0 (TMEM lanes 0-127: one query row per thread)
 //   warps 4-7  softmax for tile 1
 //   warp  8    tensor-core issue (one thread): S = Q K^T and O += P V
 //   warp  9    TMA producer (one thread): Q once, then K_j, V_j into a ring
+//   warps 10-11 idle (they complete the third warpgroup, whose registers are
+//              handed to the softmax warpgroups with setmaxnreg)
 // TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D,256+2D).
 // The softmax writes P (BF16 or E4M3) over the first columns of its S tile and
 // the PV product reads P straight from TMEM, so P never touches shared memory.
@@ -70,7 +72,12 @@ struct AttnCfg {
                                                        : ptx::make_idesc(2, 1, 1, 0, 0, BN, BM);
   static constexpr uint32_t IDESC_PV =
       PV == PV_BF16 ? ptx::make_idesc(1, 1, 1, 0, 1, D, BM) : ptx::make_idesc(1, 0, 0, 0, 1, D, BM);
-  static constexpr int THREADS = 320;
+  // 3 warpgroups: softmax tile 0, softmax tile 1, control (MMA warp, TMA warp, 2 idle).
+  // Launch: 384 threads x 168 registers = 64512; after re-balancing
+  // 2 x 128 x 224 + 128 x 56 = 64512 (the sum must not exceed the launch total).
+  static constexpr int THREADS = 384;
+  static constexpr uint32_t SOFTMAX_REGS = 224, CONTROL_REGS = 56;
+  static_assert(2 * 128 * SOFTMAX_REGS + 128 * CONTROL_REGS <= THREADS * 168, "register split exceeds launch");
 };
 
 struct alignas(8) AttnMisc {
@@ -383,14 +390,19 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo& t, int x,
         for (int j = 0; j < 32; ++j)
           if (32 * c + j >= lim) f[c][j] = -INFINITY;
     }
-    float m_tile = -INFINITY;
+    float mc[4];
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      float mc = f[c][0];
+    for (int c = 0; c < 4; ++c) {  // tree max: short dependency chains
+      float t[16];
 #pragma unroll
-      for (int j = 1; j < 32; ++j) mc = fmaxf(mc, f[c][j]);
-      m_tile = fmaxf(m_tile, mc * ck[c]);
+      for (int j = 0; j < 16; ++j) t[j] = fmaxf(f[c][j], f[c][j + 16]);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) t[j] = fmaxf(t[j], t[j + 8]);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) t[j] = fmaxf(t[j], t[j + 4]);
+      mc[c] = fmaxf(fmaxf(t[0], t[1]), fmaxf(t[2], t[3])) * ck[c];
     }
+    const float m_tile = fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3]));
     const float m_new = fmaxf(m, m_tile);
     float alpha = 1.f;
     bool resc = false;
@@ -422,31 +434,35 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo& t, int x,
     float rs = 0.f;
     if constexpr (C::PV == PV_BF16) {
       uint32_t pk[2][32];
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < 4; ++c)
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
           pk[c >> 1][(c & 1) * 16 + j] = pack_bf16x2(f[c][2 * j], f[c][2 * j + 1]);
-          rs += f[c][2 * j] + f[c][2 * j + 1];
+          acc[j & 7] += f[c][2 * j] + f[c][2 * j + 1];
         }
+      rs = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
       tmem_st32(tS, pk[0]);
       tmem_st32(tS + 32, pk[1]);
     } else {
       // The row sum adds the E4M3-rounded values actually stored, so the
       // normalised weights sum to one and a dominant key returns its value.
       uint32_t pk[32];
+      float racc[4];
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        uint32_t acc = 0u;  // f16x2 zero
+        uint32_t acc[2] = {0u, 0u};  // f16x2 zeros
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const uint32_t lo = pack_e4m3x2(f[c][4 * j], f[c][4 * j + 1]);
           const uint32_t hi = pack_e4m3x2(f[c][4 * j + 2], f[c][4 * j + 3]);
           pk[c * 8 + j] = lo | (hi << 16);
-          acc = hadd2(acc, hadd2(e4m3x2_to_f16x2(lo), e4m3x2_to_f16x2(hi)));
+          acc[j & 1] = hadd2(acc[j & 1], hadd2(e4m3x2_to_f16x2(lo), e4m3x2_to_f16x2(hi)));
         }
-        rs += f16x2_sum(acc);
+        racc[c] = f16x2_sum(acc[0]) + f16x2_sum(acc[1]);
       }
+      rs = (racc[0] + racc[1]) + (racc[2] + racc[3]);
       tmem_st32(tS, pk);
     }
     l += rs;
@@ -603,14 +619,18 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   const Waiter w{&misc->abort, p.err, p.wait_cycles};
 
   if (warp < 8) {
+    regs_inc<C::SOFTMAX_REGS>();
     const int x = warp >> 2;
     if (t[x].valid) attn_softmax_role<C>(p, t[x], x, b, hkv, sQ[x], misc, tmem, &tmO, w);
-  } else if (warp == 8) {
-    if (lane == 0) attn_mma_role<C>(p, t, b, hkv, sQ, sSlots, misc, tmem, w);
-    __syncwarp();
   } else {
-    if (lane == 0) attn_load_role<C>(p, t, b, hkv, sQ, sSlots, misc, &tmQ, &tmK, &tmV, w);
-    __syncwarp();
+    regs_dec<C::CONTROL_REGS>();
+    if (warp == 8) {
+      if (lane == 0) attn_mma_role<C>(p, t, b, hkv, sQ, sSlots, misc, tmem, w);
+      __syncwarp();
+    } else if (warp == 9) {
+      if (lane == 0) attn_load_role<C>(p, t, b, hkv, sQ, sSlots, misc, &tmQ, &tmK, &tmV, w);
+      __syncwarp();
+    }
   }
 
   tc_fence_before();
