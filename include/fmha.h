@@ -152,6 +152,30 @@ fmha_status fmha_quantize_blockwise(const fmha_tensor* src, const fmha_tensor* d
 /* Workspace bytes fmha_quantize_blockwise needs for this granularity and shape. */
 size_t fmha_quantize_workspace_bytes(int32_t sf_kind, int32_t B, int32_t S, int32_t H, int32_t D);
 
+/* The block quantizer for callers that cannot allocate device memory. (The
+ * pages have no counterpart: this is an addition of this library.)
+ * Some callers cannot allocate device memory for a call: a plugin inside an
+ * engine that owns all device memory and exposes no allocator, or code on a
+ * latency-critical path where cudaMalloc and the device synchronisation it
+ * can imply are not allowed. This entry point takes the same arguments as
+ * fmha_quantize_blockwise, minus the workspace, and allocates nothing: the
+ * amax accumulators live in a device array built into the library, 256 KB
+ * (65536 scale groups) that every GPU loading the library holds until the
+ * process exits. Codes and scales are identical to fmha_quantize_blockwise.
+ *  - Limit: at most 65536 scale groups (per tensor: 1; per head: B*H; per
+ *    channel: B*H*D; per token block needs none). Larger requests return
+ *    FMHA_ERR_INVALID_ARG with the sizes in fmha_last_error_message().
+ *  - The first call on a device (that device current) looks up the array's
+ *    device address with cudaGetSymbolAddress; make that first call before
+ *    any stream capture.
+ *  - All calls share the one array. It keeps the last call's contents; each
+ *    call clears the part it uses before use. Calls that overlap on the GPU
+ *    (for example on two streams at once) race and give wrong scales: order
+ *    them on one stream.                                                    */
+fmha_status fmha_quantize_blockwise_noalloc(const fmha_tensor* src, const fmha_tensor* dst, const fmha_sf* sf,
+                                            int32_t B, int32_t S, int32_t H, int32_t D,
+                                            struct CUstream_st* stream);
+
 /* Dense attention (optionally causal) over contiguous K/V ([BW-FP8] intro). */
 fmha_status fmha_fwd(const fmha_args* args, struct CUstream_st* stream);
 

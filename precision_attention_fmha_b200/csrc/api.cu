@@ -399,6 +399,25 @@ size_t fmha_quantize_workspace_bytes(int32_t sf_kind, int32_t B, int32_t S, int3
   return quant_groups(sf_kind, B < 0 ? 0 : B, H < 0 ? 0 : H, D < 0 ? 0 : D) * sizeof(uint32_t);
 }
 
+fmha_status fmha_quantize_blockwise_noalloc(const fmha_tensor* src, const fmha_tensor* dst, const fmha_sf* sf,
+                                            int32_t B, int32_t S, int32_t H, int32_t D, cudaStream_t stream) {
+  if (sf == nullptr) return fail(FMHA_ERR_INVALID_ARG, "NULL argument");
+  const size_t need = fmha_quantize_workspace_bytes(sf->kind, B, S, H, D);
+  const size_t have = kQuantNoallocScratchWords * sizeof(uint32_t);
+  if (need > have)
+    return fail(FMHA_ERR_INVALID_ARG,
+                "needs %zu bytes of scratch (%zu scale groups); the built-in scratch holds %zu bytes "
+                "(%zu groups); use fmha_quantize_blockwise with a workspace",
+                need, need / sizeof(uint32_t), have, (size_t)kQuantNoallocScratchWords);
+  void* ws = nullptr;
+  if (need > 0) {
+    cudaError_t e;
+    ws = quant_noalloc_scratch(&e);
+    if (ws == nullptr) return fail(FMHA_ERR_CUDA, "built-in scratch address: %s", cudaGetErrorString(e));
+  }
+  return fmha_quantize_blockwise(src, dst, sf, B, S, H, D, ws, need, stream);
+}
+
 fmha_status fmha_fwd(const fmha_args* args, cudaStream_t stream) {
   return run_attention(args, nullptr, 0, 0, nullptr, stream);
 }

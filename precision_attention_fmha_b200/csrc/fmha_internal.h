@@ -63,4 +63,11 @@ cudaError_t launch_attention(int qk_kind, int pv_kind, int D, bool paged, const 
                              const CUtensorMap& to, cudaStream_t stream);
 cudaError_t launch_quantize(bool to_e4m3, const QuantParams& p, cudaStream_t stream);
 
+// Size of the built-in scratch used by fmha_quantize_blockwise_noalloc, in
+// 32-bit words (one per scale group of the grid-wide granularities).
+constexpr size_t kQuantNoallocScratchWords = 65536;
+// Device address of that scratch on the current device (looked up once per
+// device); nullptr and *err set on failure.
+uint32_t* quant_noalloc_scratch(cudaError_t* err);
+
 }  // namespace fmha

@@ -18,6 +18,8 @@
 // Grid-wide granularities (per tensor / head / channel): pass 1 reduces amax
 // into the caller's workspace with atomicMax on the (non-negative) fp32 bit
 // patterns, pass 2 re-reads and quantizes: 2 + 2 + 1 B/element.
+#include <mutex>
+
 #include "fmha_internal.h"
 #include "ptx_sm100.cuh"
 
@@ -246,6 +248,36 @@ cudaError_t launch_quantize_t(const QuantParams& p, cudaStream_t stream) {
 
 cudaError_t launch_quantize(bool to_e4m3, const QuantParams& p, cudaStream_t stream) {
   return to_e4m3 ? launch_quantize_t<true>(p, stream) : launch_quantize_t<false>(p, stream);
+}
+
+// Built-in scratch for fmha_quantize_blockwise_noalloc: the amax accumulators
+// of the grid-wide granularities live in this file-scope device array instead
+// of a caller buffer, so that entry point never allocates. Every device that
+// loads the library holds it (256 KB) until the process exits. In host code the
+// name is only a stand-in for the symbol: kernels get the real device address
+// from cudaGetSymbolAddress, looked up once per device below.
+static __device__ __align__(256) uint32_t g_quant_noalloc_scratch[kQuantNoallocScratchWords];
+
+uint32_t* quant_noalloc_scratch(cudaError_t* err) {
+  constexpr int kMaxDevices = 64;
+  static uint32_t* addr[kMaxDevices] = {};
+  static std::mutex mu;
+  int dev = 0;
+  *err = cudaGetDevice(&dev);  // the caller's current device is the one the kernels run on
+  if (*err != cudaSuccess) return nullptr;
+  if (dev < 0 || dev >= kMaxDevices) {
+    *err = cudaErrorInvalidDevice;
+    return nullptr;
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    *err = cudaGetSymbolAddress(&p, g_quant_noalloc_scratch);
+    if (*err != cudaSuccess) return nullptr;
+    addr[dev] = static_cast<uint32_t*>(p);
+  }
+  *err = cudaSuccess;
+  return addr[dev];
 }
 
 }  // namespace fmha
