@@ -33,10 +33,17 @@ sys.path.insert(0, ROOT)
 METRIC = "attention TFLOPS (4·B·H·Sq·Skv·D·density) and % of dtype tensor peak"
 UNIT = "TFLOPS"
 WORKLOADS = {
-    # name: (B, H, S, D)
-    "dense_pv8_s32768": (1, 40, 32768, 128),
-    "dense_pv8_s16384": (1, 40, 16384, 128),
-    "dense_pv8_s4096": (1, 40, 4096, 128),
+    # name: (kind, B, Hq, Hkv, S, D, causal)
+    "dense_pv8_s32768": ("pv8", 1, 40, 40, 32768, 128, False),
+    "dense_pv8_s16384": ("pv8", 1, 40, 40, 16384, 128, False),
+    "dense_pv8_s4096": ("pv8", 1, 40, 40, 4096, 128, False),
+    "dense_bf16_s16384": ("bf16", 1, 40, 40, 16384, 128, False),
+    "dense_bf16_s4096": ("bf16", 1, 40, 40, 4096, 128, False),
+    "tiny_bf16": ("bf16", 1, 1, 1, 256, 64, False),
+    "all_fp8_s8192": ("fp8", 2, 32, 32, 8192, 128, False),
+    "all_fp8_s8192_causal": ("fp8", 2, 32, 32, 8192, 128, True),
+    "sage_s16384": ("sage", 1, 24, 24, 16384, 128, False),
+    "sparse_paged_s16384": ("sparse_paged", 4, 64, 8, 16384, 128, False),
 }
 DEFAULT_WORKLOAD = "dense_pv8_s32768"
 
@@ -138,6 +145,101 @@ def max_over_ranks(x, world):
     return float(t.item())
 
 
+# ------------------------------------------------------------- workloads ----
+class Work:
+    """One workload: host inputs, GPU quantization prep, the attention call."""
+
+    def __init__(self, name, dev, fmha, workloads, Scale):
+        kind, B, Hq, Hkv, S, D, causal = WORKLOADS[name]
+        self.kind, self.B, self.Hq, self.Hkv, self.S, self.D, self.causal = kind, B, Hq, Hkv, S, D, causal
+        self.dev, self.fmha, self.Scale = dev, fmha, Scale
+        bf16_peak, _, src = load_peaks()
+        self.peak_src = src
+        E4 = torch.float8_e4m3fn
+        if kind == "bf16":
+            w = workloads.normal_qkv(workloads.SEED_BASE + 1 + S, B, S, S, Hq, Hkv, D)
+            self.host = dict(zip(("q", "k", "v"), w))
+            self.peak, self.peak_note, self.dtype = bf16_peak, "bf16 burst", "bf16"
+            self.quant = []
+        elif kind == "pv8":
+            w = workloads.dense_pv8(S=S, B=B, H=Hq, D=D)
+            self.host = {n: w[n] for n in ("q", "k", "v")}
+            self.peak = 1.0 / (0.5 / bf16_peak + 0.5 / (2.0 * bf16_peak))
+            self.peak_note = f"bf16 burst {bf16_peak} for QK^T, 2x (nominal E4M3 ratio) for PV, time-weighted"
+            self.dtype = "bf16,e4m3"
+            self.quant = [("v", E4, "per_tensor", None)]
+        elif kind == "fp8":
+            w = workloads.all_fp8(S=S, B=B, H=Hq, D=D)
+            self.host = {n: w[n] for n in ("q", "k", "v")}
+            self.peak, self.peak_note, self.dtype = 2.0 * bf16_peak, f"2 x bf16 burst {bf16_peak} (nominal E4M3 ratio)", "e4m3"
+            self.quant = [("q", E4, "per_head", None), ("k", E4, "per_head", None), ("v", E4, "per_head", None)]
+        elif kind == "sage":
+            w = workloads.sage(S=S, B=B, H=Hq, D=D)
+            self.host = {n: w[n] for n in ("q", "k", "v")}
+            self.peak = 2.0 * bf16_peak
+            self.peak_note = f"2 x bf16 burst {bf16_peak} (nominal INT8 and E4M3 ratio)"
+            self.dtype = "int8,e4m3"
+            self.quant = [("q", torch.int8, "per_token_block", 128), ("k", torch.int8, "per_token_block", 64),
+                          ("v", E4, "per_channel", None)]
+        elif kind == "sparse_paged":
+            w = workloads.sparse_paged(S=S, B=B, Hq=Hq, Hkv=Hkv, D=D)
+            self.host = {"q": w["q"], "k_pool": w["k_pool"], "v_pool": w["v_pool"], "page_table": w["page_table"],
+                         "mask": w["mask"]}
+            self.peak, self.peak_note, self.dtype = bf16_peak, "bf16 burst", "bf16"
+            self.quant = []
+        self.scale = 1.0 / math.sqrt(D)
+        self.host = {n: t.contiguous().pin_memory() for n, t in self.host.items()}
+        self.dev_in = {n: t.to(dev) for n, t in self.host.items()}
+        self.o = torch.empty((B, S, Hq, D), dtype=torch.bfloat16, device=dev)
+        # density = kept score elements / (Sq * Skv)
+        if kind == "sparse_paged":
+            kept = float(self.host["mask"].to(torch.float64).sum())
+            self.density = kept * 128 * 128 / (B * Hkv * S * S)
+            self.flop = 4.0 * B * Hq * S * S * D * self.density
+        else:
+            self.density = (S + 1) / (2 * S) if causal else 1.0
+            self.flop = 4.0 * B * Hq * S * S * D * self.density
+        self.qbuf = {}
+        for name, dt, gran, rpb in self.quant:
+            x = self.dev_in[name]
+            shp = fmha.scale_shape(gran, B, S, x.shape[2], D, rpb)
+            self.qbuf[name] = (torch.empty(x.shape, dtype=dt, device=dev), torch.empty(shp, dtype=torch.float32,
+                               device=dev), torch.empty(max(4, fmha.quantize_workspace_bytes(gran, B, S, x.shape[2], D)),
+                                                        dtype=torch.uint8, device=dev), gran, rpb, dt)
+        self.sf_p = None
+        if kind == "sage":  # per-row-block P scale: P stored as 16 p
+            self.sf_p = Scale(torch.full((B, Hq, math.ceil(S / 128)), 1.0 / 16, device=dev), "per_token_block", 128)
+        # our kernels per step: token-block quantization is 1 launch, the grid-wide kinds 2, attention 1
+        self.launches = 1 + sum(1 if g == "per_token_block" else 2 for _, _, g, _ in self.quant)
+
+    def prep(self, inp):
+        for name, (out, sc, ws, gran, rpb, dt) in self.qbuf.items():
+            self.fmha.fmha_quantize_blockwise(inp[name], dt, gran, rpb, out=out, scales=sc, workspace=ws)
+
+    def attn(self, inp):
+        f, S_ = self.fmha, self.Scale
+        if self.kind == "sparse_paged":
+            f.fmha_fwd_paged(inp["q"], inp["k_pool"], inp["v_pool"], inp["page_table"], self.S, mask=inp["mask"],
+                             out=self.o, softmax_scale=self.scale)
+            return
+        ops = {n: inp[n] for n in ("q", "k", "v")}
+        sfs = {}
+        for name, (out, sc, ws, gran, rpb, dt) in self.qbuf.items():
+            ops[name] = out
+            sfs["sf_" + name] = S_(sc, gran, rpb or 0)
+        f.fmha_fwd(ops["q"], ops["k"], ops["v"], out=self.o, softmax_scale=self.scale, causal=self.causal,
+                   sf_p=self.sf_p, **sfs)
+
+    def config(self, world):
+        c = {"workload": self.kind if self.kind != "pv8" else "dense_pv8", "B": self.B, "Hq": self.Hq,
+             "Hkv": self.Hkv, "Sq": self.S, "Skv": self.S, "D": self.D, "causal": self.causal,
+             "density": round(self.density, 6),
+             "quantized_in_step": [f"{n}:{g}" for n, _, g, _ in self.quant],
+             "l2": "inputs larger than L2" if self.host["q"].numel() * 2 > 126 * 2**20 else "inputs fit in L2",
+             "parallelism": f"replicas{world}"}
+        return c
+
+
 # ------------------------------------------------------------------ ours ----
 def run_ours(args):
     from precision_attention_fmha_b200 import fmha, workloads
@@ -146,23 +248,12 @@ def run_ours(args):
     world, rank, local = dist_setup(args.gpus)
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    B, H, S, D = WORKLOADS[args.workload]
-    w = workloads.dense_pv8(S=S, B=B, H=H, D=D)
-    q_h, k_h, v_h = (w[n].pin_memory() for n in ("q", "k", "v"))
-    q, k, v = (t.to(dev) for t in (q_h, k_h, v_h))
-    scale = w["scale"]
-    v8 = torch.empty(v.shape, dtype=torch.float8_e4m3fn, device=dev)
-    sv = torch.empty(1, dtype=torch.float32, device=dev)
-    ws = torch.empty(fmha.quantize_workspace_bytes("per_tensor", B, S, H, D), dtype=torch.uint8, device=dev)
-    o = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
+    W = Work(args.workload, dev, fmha, workloads, Scale)
     stream = torch.cuda.current_stream()
 
-    def step(qd, kd, vd):
-        fmha.fmha_quantize_blockwise(vd, torch.float8_e4m3fn, "per_tensor", out=v8, scales=sv, workspace=ws)
-        fmha.fmha_fwd(qd, kd, v8, out=o, sf_v=Scale(sv, "per_tensor"), softmax_scale=scale)
-
     for _ in range(args.warmup):
-        step(q, k, v)
+        W.prep(W.dev_in)
+        W.attn(W.dev_in)
     fmha.get_device_error()
     torch.cuda.synchronize()
 
@@ -177,9 +268,9 @@ def run_ours(args):
     torch.cuda.synchronize()
     t0.record(stream)
     for i in range(K):
-        fmha.fmha_quantize_blockwise(v, torch.float8_e4m3fn, "per_tensor", out=v8, scales=sv, workspace=ws)
+        W.prep(W.dev_in)
         attn_ev[i][0].record(stream)
-        fmha.fmha_fwd(q, k, v8, out=o, sf_v=Scale(sv, "per_tensor"), softmax_scale=scale)
+        W.attn(W.dev_in)
         attn_ev[i][1].record(stream)
     t1.record(stream)
     torch.cuda.synchronize()
@@ -192,47 +283,42 @@ def run_ours(args):
     attn_ms = max_over_ranks(attn_ms, world)
 
     # ---- end-to-end: host (pinned) inputs, H2D + path + D2H of O each step ----
-    o_h = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+    o_h = torch.empty(W.o.shape, dtype=W.o.dtype, pin_memory=True)
     Ke = max(1, min(K, 10))
     barrier(world)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(Ke):
-        qd, kd, vd = (t.to(dev, non_blocking=True) for t in (q_h, k_h, v_h))
-        step(qd, kd, vd)
-        o_h.copy_(o, non_blocking=True)
+        inp = {n: t.to(dev, non_blocking=True) for n, t in W.host.items()}
+        W.prep(inp)
+        W.attn(inp)
+        o_h.copy_(W.o, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
     barrier(world)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / Ke, world)
     fmha.get_device_error()
 
-    fl = flops(B, H, S, D)
-    tflops = world * fl / (ms * 1e-3) / 1e12
-    bf16_peak, _, peak_src = load_peaks()
-    # QK^T runs at the BF16 rate, PV at the E4M3 rate (2x BF16 nominal): time-weighted peak.
-    peak = 1.0 / (0.5 / bf16_peak + 0.5 / (2.0 * bf16_peak))
-    achieved = fl / (attn_ms * 1e-3) / 1e12
-    cpu = cpu_baseline(B, H, S, D, w) if (rank == 0 and world == 1 and not args.no_cpu_baseline) else None
-    bytes_in = sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h))
+    tflops = world * W.flop / (ms * 1e-3) / 1e12
+    achieved = W.flop / (attn_ms * 1e-3) / 1e12
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(W)
+    bytes_in = sum(t.numel() * t.element_size() for t in W.host.values())
     line = {
         "metric": METRIC, "value": round(tflops, 2), "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "bf16,e4m3", "data": "synthetic (seeded N(0,1), BF16)",
-        "config": {"workload": args.workload, "B": B, "H": H, "Sq": S, "Skv": S, "D": D, "causal": False,
-                   "q_k": "bf16", "v": "e4m3 per-tensor (quantized in the step)", "p": "e4m3", "o": "bf16",
-                   "l2": "inputs larger than L2 (each of Q, K, V is %d MB)" % (q.numel() * 2 // 2**20),
-                   "parallelism": f"replicas{world}"},
-        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": round(peak, 1), "unit": "TFLOP/s",
-                     "frac": round(achieved / peak, 4), "traffic": None,
-                     "peak_note": f"{peak_src} bf16 burst {bf16_peak} x (QK at 1x, PV at 2x nominal E4M3 rate)",
-                     "kernel": "attn_fwd_kernel", "kernel_ms": round(attn_ms, 4),
-                     "frac_of_bf16_peak": round(achieved / bf16_peak, 4)},
-        "e2e": {"value": round(world * fl / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
-                "h2d_bytes_per_step": bytes_in, "d2h_bytes_per_step": o.numel() * o.element_size(),
+        "vs_baseline": None, "dtype": W.dtype, "data": "synthetic (seeded, BF16 inputs)",
+        "config": W.config(world),
+        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": round(W.peak, 1), "unit": "TFLOP/s",
+                     "frac": round(achieved / W.peak, 4), "traffic": TRAFFIC.get(args.workload),
+                     "peak_note": f"{W.peak_src}: {W.peak_note}", "kernel": "attn_fwd_kernel",
+                     "kernel_ms": round(attn_ms, 4)},
+        "e2e": {"value": round(world * W.flop / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
+                "h2d_bytes_per_step": bytes_in, "d2h_bytes_per_step": W.o.numel() * W.o.element_size(),
                 "steps": Ke},
-        "gpu_launches": K * 3,
+        "gpu_launches": K * W.launches,
         "clocks": clk,
     }
     if cpu is not None:
@@ -245,23 +331,49 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
+# DRAM bytes (read + write) of one attention launch from an ncu capture of the
+# same kernel build, per workload (None until captured for the current kernel).
+TRAFFIC = {}
+
+
 # ------------------------------------------------------------- reference ----
-def oracle_sample(w, B, H, S, D, heads=1, rows=256):
-    """The CPU oracle on a bounded sample: V quantized (per tensor over the
-    sampled heads) then float64 attention for `rows` query rows of `heads`
-    heads against the full key length. Returns (seconds, flops done)."""
+def oracle_sample(host, kind, B, Hq, Hkv, S, D, causal, rows):
+    """The CPU oracle on a bounded sample: the workload's quantization of the
+    sampled KV head (over all tokens) and float64 attention for `rows` query
+    rows of query head 0 against all keys. Returns (seconds, useful FLOPs)."""
     from oracle import attention as oa
     from oracle import quant as oq
 
-    q = w["q"][:, :rows, :heads].to(torch.float64).numpy()
-    k = w["k"][:, :, :heads].to(torch.float64).numpy()
-    v = w["v"][:, :, :heads].to(torch.float32).numpy()
     t = time.perf_counter()
-    codes, sc = oq.quantize_blockwise(v, "e4m3", "per_tensor")
-    vd = oq.dequantize(codes, sc, "e4m3", "per_tensor")
-    oa.attention(q, k, vd, w["scale"])
+    if kind == "sparse_paged":
+        pt = host["page_table"].numpy()[:1]
+        k = oa.gather_paged(host["k_pool"][:, :, :1].to(torch.float64).numpy(), pt, S)
+        v = oa.gather_paged(host["v_pool"][:, :, :1].to(torch.float64).numpy(), pt, S)
+        q = host["q"][:1, :rows, :1].to(torch.float64).numpy()
+        mask = host["mask"][:1, :1].numpy()
+        mask = mask[:, :, : -(-rows // 128)]
+    else:
+        q32 = host["q"][:1, :rows, :1].to(torch.float32).numpy()
+        k32 = host["k"][:1, :, :1].to(torch.float32).numpy()
+        v32 = host["v"][:1, :, :1].to(torch.float32).numpy()
+        spec = {"bf16": {}, "pv8": {"v": ("e4m3", "per_tensor", None)},
+                "fp8": {n: ("e4m3", "per_head", None) for n in "qkv"},
+                "sage": {"q": ("int8", "per_token_block", 128), "k": ("int8", "per_token_block", 64),
+                         "v": ("e4m3", "per_channel", None)}}[kind]
+        ops = {"q": q32, "k": k32, "v": v32}
+        for n, (dt, g, rpb) in spec.items():
+            c, sc = oq.quantize_blockwise(ops[n], dt, g, rpb)
+            ops[n] = oq.dequantize(c, sc, dt, g, rpb)
+        q, k, v = (np.asarray(ops[n], dtype=np.float64) for n in "qkv")
+        mask = None
+    Sq = q.shape[1]
+    if causal:  # the sampled rows are the first ones; keep their causal view of all keys
+        k, v = k[:, :Sq], v[:, :Sq]
+    oa.attention(q, k, v, 1.0 / math.sqrt(D), causal, mask)
     dt = time.perf_counter() - t
-    return dt, 4.0 * B * heads * rows * S * D
+    dens = ((Sq + 1) / (2 * Sq)) if causal else (float(mask.sum()) * 128 * 128 / (Sq * S) if mask is not None else 1.0)
+    keys = Sq if causal else S
+    return dt, 4.0 * Sq * keys * D * min(1.0, dens)
 
 
 def cpu_cores():
@@ -271,11 +383,11 @@ def cpu_cores():
         return os.cpu_count()
 
 
-def cpu_baseline(B, H, S, D, w, rows=1024):
-    dt, fl = oracle_sample(w, B, H, S, D, heads=1, rows=rows)
+def cpu_baseline(W, rows=1024):
+    dt, fl = oracle_sample(W.host, W.kind, W.B, W.Hq, W.Hkv, W.S, W.D, W.causal, rows)
     return {"value": round(fl / dt / 1e12, 6), "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
-            "sample": f"head 0, query rows 0..{rows - 1} against all {S} keys (plus V quantization of that head), "
-                      f"float64 NumPy, {dt:.1f} s"}
+            "sample": f"query head 0, rows 0..{rows - 1} against all keys (with the workload's quantization of "
+                      f"that head), float64 NumPy, {dt:.1f} s"}
 
 
 def run_reference(args):
@@ -285,23 +397,29 @@ def run_reference(args):
         return
     from precision_attention_fmha_b200 import workloads
 
-    B, H, S, D = WORKLOADS[args.workload]
-    w = workloads.dense_pv8(S=S, B=B, H=H, D=D)
+    kind, B, Hq, Hkv, S, D, causal = WORKLOADS[args.workload]
+    gen = {"bf16": lambda: dict(zip("qkv", workloads.normal_qkv(workloads.SEED_BASE + 1 + S, B, S, S, Hq, Hkv, D))),
+           "pv8": lambda: workloads.dense_pv8(S=S, B=B, H=Hq, D=D),
+           "fp8": lambda: workloads.all_fp8(S=S, B=B, H=Hq, D=D),
+           "sage": lambda: workloads.sage(S=S, B=B, H=Hq, D=D),
+           "sparse_paged": lambda: workloads.sparse_paged(S=S, B=B, Hq=Hq, Hkv=Hkv, D=D)}[kind]
+    host = gen()
     rows = 256
     for _ in range(args.warmup):
-        oracle_sample(w, B, H, S, D, rows=rows)
+        oracle_sample(host, kind, B, Hq, Hkv, S, D, causal, rows)
     times, fl = [], 0
     for _ in range(args.steps):
-        dt, fl = oracle_sample(w, B, H, S, D, rows=rows)
+        dt, fl = oracle_sample(host, kind, B, Hq, Hkv, S, D, causal, rows)
         times.append(dt)
     ms = 1e3 * sum(times) / len(times)
     val = fl / (ms * 1e-3) / 1e12
-    sample = f"head 0, query rows 0..{rows - 1} against all {S} keys, float64 NumPy oracle per step"
+    sample = f"query head 0, rows 0..{rows - 1} against all keys, float64 NumPy oracle per step"
     line = {
         "impl": "reference", "metric": METRIC, "value": round(val, 6), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded N(0,1), BF16)",
-        "config": {"workload": args.workload, "B": B, "H": H, "Sq": S, "Skv": S, "D": D, "causal": False},
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded, BF16 inputs)",
+        "config": {"workload": args.workload, "B": B, "Hq": Hq, "Hkv": Hkv, "Sq": S, "Skv": S, "D": D,
+                   "causal": causal},
         "cpu_baseline": {"value": round(val, 6), "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(val, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

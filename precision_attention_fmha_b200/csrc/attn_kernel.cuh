@@ -36,6 +36,23 @@
 #include "fmha_internal.h"
 #include "ptx_sm100.cuh"
 
+// Optional phase tracing for one CTA (build with -DFMHA_TRACE=<cta index>):
+// clock64 stamps of each role's phases go to a device array that the host
+// reads with fmha_trace_read(). Off in normal builds.
+#ifdef FMHA_TRACE
+#define FMHA_TRACE_SLOTS (1 << 16)
+static __device__ unsigned long long g_fmha_trace[FMHA_TRACE_SLOTS];  // one per translation unit
+#define TRACE(slot, cond)                                                                   \
+  do {                                                                                      \
+    if (blockIdx.x == (FMHA_TRACE) && (cond) && (slot) < FMHA_TRACE_SLOTS)                  \
+      g_fmha_trace[(slot)] = static_cast<unsigned long long>(clock64());                    \
+  } while (0)
+#else
+#define TRACE(slot, cond) \
+  do {                    \
+  } while (0)
+#endif
+
 namespace fmha {
 
 template <int D_, int QK_, int PV_, bool PAGED_>
@@ -132,7 +149,10 @@ struct Waiter {
   }
 };
 
-__device__ __forceinline__ bool keep_tile(const AttnParams& p, const TileInfo& t, int b, int hkv, int u) {
+// Tile info and waiters are passed by value everywhere: a runtime-indexed
+// array or a by-reference argument would live in local memory, and with the
+// shared-memory carve-out near its maximum every such load goes to L2.
+__device__ __forceinline__ bool keep_tile(const AttnParams& p, const TileInfo t, int b, int hkv, int u) {
   if (u >= t.n_kv) return false;
   if (p.mask == nullptr) return true;
   return p.mask[b * p.mask_sb + hkv * p.mask_sh + static_cast<int64_t>(t.qblk) * p.n_kv_blocks + u] != 0;
@@ -150,14 +170,18 @@ __device__ __forceinline__ float sf_lookup(const float* sf, int kind, int64_t bh
 
 // ------------------------------------------------------------ TMA producer --
 template <class C>
-__device__ void attn_load_role(const AttnParams& p, const TileInfo (&t)[2], int b, int hkv, uint8_t* const (&sQ)[2],
-                               uint8_t* sSlots, AttnMisc* misc, const CUtensorMap* tmQ, const CUtensorMap* tmK,
-                               const CUtensorMap* tmV, const Waiter& w) {
+__device__ void attn_load_role(const AttnParams& p, const TileInfo t0, const TileInfo t1, int b, int hkv,
+                               uint8_t* sQ0, uint8_t* sQ1, uint8_t* sSlots, AttnMisc* misc, const CUtensorMap* tmQ,
+                               const CUtensorMap* tmK, const CUtensorMap* tmV, const Waiter w) {
   using namespace ptx;
+  const TileInfo t[2] = {t0, t1};  // indexed only with unrolled constants below
+  uint8_t* const sQ[2] = {sQ0, sQ1};
   const uint32_t q_full = smem_addr(&misc->q_full);
   uint32_t qbytes = 0;
+#pragma unroll
   for (int x = 0; x < 2; ++x) qbytes += t[x].valid ? C::Q_TILE : 0;
   mbar_arrive_expect_tx(q_full, qbytes);
+#pragma unroll
   for (int x = 0; x < 2; ++x) {
     if (!t[x].valid) continue;
 #pragma unroll
@@ -165,14 +189,12 @@ __device__ void attn_load_role(const AttnParams& p, const TileInfo (&t)[2], int 
       tma_load_4d(smem_addr(sQ[x]) + c * C::CHUNK_BYTES, tmQ, q_full, c * C::QK_CHUNK_ELEMS, t[x].h, t[x].q0, b);
   }
   const uint64_t pol = policy_evict_last();  // K/V tiles are re-read by every CTA of this head
-  int last_phase[8];
-#pragma unroll
-  for (int s = 0; s < 8; ++s) last_phase[s] = -1;
+  uint32_t issued = 0u, issued_phase = 0u;  // per slot: a load was issued / parity of its last phase
   int slot_it = 0;
-  const int n_u = max(t[0].n_kv, t[1].n_kv);
+  const int n_u = max(t0.n_kv, t1.n_kv);
   bool ok = true;
   for (int u = 0; u < n_u && ok; ++u) {
-    if (!keep_tile(p, t[0], b, hkv, u) && !keep_tile(p, t[1], b, hkv, u)) continue;
+    if (!keep_tile(p, t0, b, hkv, u) && !keep_tile(p, t1, b, hkv, u)) continue;
     for (int kv = 0; kv < 2; ++kv) {  // K then V
       const int s = slot_it % C::STAGES;
       const uint32_t ph = (slot_it / C::STAGES) & 1;
@@ -184,7 +206,8 @@ __device__ void attn_load_role(const AttnParams& p, const TileInfo (&t)[2], int 
       const CUtensorMap* tm = kv == 0 ? tmK : tmV;
       const uint32_t dst = smem_addr(sSlots + s * C::SLOT);
       mbar_arrive_expect_tx(full, kv == 0 ? C::K_TILE : C::V_TILE);
-      last_phase[s] = static_cast<int>(ph);
+      issued |= 1u << s;
+      issued_phase = (issued_phase & ~(1u << s)) | (ph << s);
       if constexpr (!C::PAGED) {
         for (int c = 0; c < chunks; ++c)
           tma_load_4d_hint(dst + c * C::CHUNK_BYTES, tm, full, c * chunk_elems, hkv, u * C::BN, b, pol);
@@ -210,58 +233,81 @@ __device__ void attn_load_role(const AttnParams& p, const TileInfo (&t)[2], int 
   if (*w.abort_flag) {  // let every issued copy land before shared memory goes away
     w.drain(q_full, 0);
     for (int s = 0; s < C::STAGES; ++s)
-      if (last_phase[s] >= 0) w.drain(smem_addr(&misc->kv_full[s]), static_cast<uint32_t>(last_phase[s]));
+      if (issued & (1u << s)) w.drain(smem_addr(&misc->kv_full[s]), (issued_phase >> s) & 1u);
   }
 }
 
 // ------------------------------------------------------- tensor-core issue --
+// Descriptor words: lo = start address >> 4 | leading byte offset >> 4 << 16,
+// hi = stride byte offset >> 4 | version 1 (bit 46) | swizzle (bits 61-63).
+__device__ __forceinline__ uint32_t desc_lo(uint32_t addr, uint32_t lbo) {
+  return ((addr & 0x3FFFFu) >> 4) | ((lbo >> 4) << 16);
+}
+__device__ __forceinline__ uint32_t desc_hi(uint32_t sbo, uint32_t swizzle) {
+  return (sbo >> 4) | (1u << 14) | (swizzle << 29);
+}
+
+// S = Q K^T: QK_STEPS MMAs of K = 32 bytes; the K-step advances the start
+// address by 32 bytes inside a 128-byte swizzle row, then jumps to the next
+// 16 KB column block.
 template <class C>
-__device__ __forceinline__ void issue_qk(uint32_t tmem_d, uint32_t q_smem, uint32_t k_smem) {
+__device__ __forceinline__ void issue_qk(uint32_t tmem_d, uint32_t q_lo, uint32_t k_lo, uint32_t hi) {
 #pragma unroll
   for (int s = 0; s < C::QK_STEPS; ++s) {
-    const uint32_t off = (s / 4) * C::CHUNK_BYTES + (s % 4) * 32;
-    const uint64_t a = ptx::smem_desc(q_smem + off, 16, 1024, 2);
-    const uint64_t bd = ptx::smem_desc(k_smem + off, 16, 1024, 2);
-    if constexpr (C::QK == QK_BF16)
-      ptx::mma_ss_f16(tmem_d, a, bd, C::IDESC_QK, s > 0);
-    else if constexpr (C::QK == QK_E4M3)
-      ptx::mma_ss_f8(tmem_d, a, bd, C::IDESC_QK, s > 0);
-    else
-      ptx::mma_ss_i8(tmem_d, a, bd, C::IDESC_QK, s > 0);
+    const uint32_t off = ((s / 4) * C::CHUNK_BYTES + (s % 4) * 32) >> 4;
+    if constexpr (C::QK == QK_BF16) {
+      if (s == 0) ptx::mma_ss_f16_lean<false>(tmem_d, q_lo + off, hi, k_lo + off, hi, C::IDESC_QK);
+      else ptx::mma_ss_f16_lean<true>(tmem_d, q_lo + off, hi, k_lo + off, hi, C::IDESC_QK);
+    } else if constexpr (C::QK == QK_E4M3) {
+      if (s == 0) ptx::mma_ss_f8_lean<false>(tmem_d, q_lo + off, hi, k_lo + off, hi, C::IDESC_QK);
+      else ptx::mma_ss_f8_lean<true>(tmem_d, q_lo + off, hi, k_lo + off, hi, C::IDESC_QK);
+    } else {
+      if (s == 0) ptx::mma_ss_i8_lean<false>(tmem_d, q_lo + off, hi, k_lo + off, hi, C::IDESC_QK);
+      else ptx::mma_ss_i8_lean<true>(tmem_d, q_lo + off, hi, k_lo + off, hi, C::IDESC_QK);
+    }
   }
 }
 
+// O += P V: P (A operand) from TMEM, V MN-major in shared memory (d contiguous):
+// K-step s starts PV_K rows down; the 64- or 128-wide d column blocks are
+// CHUNK_BYTES apart (leading byte offset), 8-row groups 1 KB apart.
 template <class C>
-__device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint32_t v_smem, bool accumulate) {
+__device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint32_t v_lo, uint32_t hi,
+                                         uint32_t accumulate) {
 #pragma unroll
   for (int s = 0; s < C::PV_STEPS; ++s) {
-    // V is MN-major (d contiguous): K-step s starts PV_K rows down; the 64/128-wide
-    // d columns are CHUNK_BYTES apart (leading byte offset), 8-row groups 1 KB apart.
-    const uint64_t bd = ptx::smem_desc(v_smem + s * C::PV_K * 128, C::CHUNK_BYTES, 1024, 2);
-    const uint32_t a = tmem_p + s * 8;  // 8 TMEM columns = 16 bf16 / 32 e4m3 of P
+    const uint32_t off = (s * C::PV_K * 128) >> 4;
+    const uint32_t acc = s > 0 ? 1u : accumulate;
     if constexpr (C::PV == PV_BF16)
-      ptx::mma_ts_f16(tmem_o, a, bd, C::IDESC_PV, (accumulate || s > 0) ? 1u : 0u);
+      ptx::mma_ts_f16_lean(tmem_o, tmem_p + s * 8, v_lo + off, hi, C::IDESC_PV, acc);
     else
-      ptx::mma_ts_f8(tmem_o, a, bd, C::IDESC_PV, (accumulate || s > 0) ? 1u : 0u);
+      ptx::mma_ts_f8_lean(tmem_o, tmem_p + s * 8, v_lo + off, hi, C::IDESC_PV, acc);
   }
 }
 
 template <class C>
-__device__ void attn_mma_role(const AttnParams& p, const TileInfo (&t)[2], int b, int hkv, uint8_t* const (&sQ)[2],
-                              uint8_t* sSlots, AttnMisc* misc, uint32_t tmem, const Waiter& w) {
+__device__ void attn_mma_role(const AttnParams& p, const TileInfo t0, const TileInfo t1, int b, int hkv, uint8_t* sQ0,
+                              uint8_t* sQ1, uint8_t* sSlots, AttnMisc* misc, uint32_t tmem, const Waiter w) {
   using namespace ptx;
   const uint32_t s_col[2] = {0u, 128u};
+  // Descriptor words, computed once: K-major Q/K (leading offset unused, 16),
+  // MN-major V (leading offset = distance between d column blocks).
+  const uint32_t hi = desc_hi(1024, 2);
+  const uint32_t q_lo0 = desc_lo(smem_addr(sQ0), 16), q_lo1 = desc_lo(smem_addr(sQ1), 16);
+  const uint32_t k_lo0 = desc_lo(smem_addr(sSlots), 16);
+  const uint32_t v_lo0 = desc_lo(smem_addr(sSlots), C::CHUNK_BYTES);
   const uint32_t o_col[2] = {256u, 256u + C::D};
   int pend[2] = {-1, -1};
   int pv_cnt[2] = {0, 0};
   int prev_v = -1;
   int slot_it = 0;
-  const int n_u = max(t[0].n_kv, t[1].n_kv);
+  const int n_u = max(t0.n_kv, t1.n_kv);
   bool ok = w.wait(smem_addr(&misc->q_full), 0);
   tc_fence_after();
   for (int u = 0; u < n_u && ok; ++u) {
-    const bool kx[2] = {keep_tile(p, t[0], b, hkv, u), keep_tile(p, t[1], b, hkv, u)};
+    const bool kx[2] = {keep_tile(p, t0, b, hkv, u), keep_tile(p, t1, b, hkv, u)};
     if (!kx[0] && !kx[1]) continue;
+    TRACE(16384 + u * 16 + 15, true);
     const int ks = slot_it % C::STAGES;
     const uint32_t kph = (slot_it / C::STAGES) & 1;
     ++slot_it;
@@ -269,11 +315,15 @@ __device__ void attn_mma_role(const AttnParams& p, const TileInfo (&t)[2], int b
     const uint32_t vph = (slot_it / C::STAGES) & 1;
     ++slot_it;
     bool k_ready = false;
+#pragma unroll
     for (int x = 0; x < 2 && ok; ++x) {
       if (pend[x] >= 0) {  // PV of the previous tile first: S_x(u) overwrites P_x
+        TRACE(16384 + u * 16 + x * 8 + 0, true);
         if (!(ok = w.wait(smem_addr(&misc->p_full[x]), pv_cnt[x] & 1))) break;
+        TRACE(16384 + u * 16 + x * 8 + 1, true);
         tc_fence_after();
-        issue_pv<C>(tmem + o_col[x], tmem + s_col[x], smem_addr(sSlots + pend[x] * C::SLOT), pv_cnt[x] > 0);
+        issue_pv<C>(tmem + o_col[x], tmem + s_col[x], v_lo0 + pend[x] * (C::SLOT >> 4), hi, pv_cnt[x] > 0);
+        TRACE(16384 + u * 16 + x * 8 + 2, true);
         ++pv_cnt[x];
         pend[x] = -1;
       }
@@ -283,24 +333,30 @@ __device__ void attn_mma_role(const AttnParams& p, const TileInfo (&t)[2], int b
           tc_fence_after();
           k_ready = true;
         }
-        issue_qk<C>(tmem + s_col[x], smem_addr(sQ[x]), smem_addr(sSlots + ks * C::SLOT));
+        TRACE(16384 + u * 16 + x * 8 + 3, true);
+        issue_qk<C>(tmem + s_col[x], x ? q_lo1 : q_lo0, k_lo0 + ks * (C::SLOT >> 4), hi);
+        TRACE(16384 + u * 16 + x * 8 + 4, true);
         tc_commit(smem_addr(&misc->s_full[x]));
+        TRACE(16384 + u * 16 + x * 8 + 5, true);
       }
     }
     if (!ok) break;
     tc_commit(smem_addr(&misc->kv_empty[ks]));                     // K_u free once the S MMAs finish
     if (prev_v >= 0) tc_commit(smem_addr(&misc->kv_empty[prev_v]));  // previous V: its PVs are issued
     if (!(ok = w.wait(smem_addr(&misc->kv_full[vs]), vph))) break;
+    TRACE(16384 + u * 16 + 7, true);
     tc_fence_after();
+    TRACE(16384 + u * 16 + 14, true);
     pend[0] = kx[0] ? vs : -1;
     pend[1] = kx[1] ? vs : -1;
     prev_v = vs;
   }
+#pragma unroll
   for (int x = 0; x < 2 && ok; ++x) {
     if (pend[x] < 0) continue;
     if (!(ok = w.wait(smem_addr(&misc->p_full[x]), pv_cnt[x] & 1))) break;
     tc_fence_after();
-    issue_pv<C>(tmem + o_col[x], tmem + s_col[x], smem_addr(sSlots + pend[x] * C::SLOT), pv_cnt[x] > 0);
+    issue_pv<C>(tmem + o_col[x], tmem + s_col[x], v_lo0 + pend[x] * (C::SLOT >> 4), hi, pv_cnt[x] > 0);
   }
   if (ok) tc_commit(smem_addr(&misc->o_full));
   // Drain: arrives when every MMA issued above has completed.
@@ -309,9 +365,13 @@ __device__ void attn_mma_role(const AttnParams& p, const TileInfo (&t)[2], int b
 }
 
 // --------------------------------------------------------------- softmax ----
+// Per kept KV tile: load S (128 fp32 per row) from TMEM, scale and mask,
+// reduce the row max with three-input max, lazily correct O, exponentiate
+// with packed fp32x2 FMAs feeding MUFU ex2, pack P (BF16 or E4M3) over the
+// first S columns and release it to the MMA warp with one arrive per warp.
 template <class C>
-__device__ void attn_softmax_role(const AttnParams& p, const TileInfo& t, int x, int b, int hkv, uint8_t* sQx,
-                                  AttnMisc* misc, uint32_t tmem, const CUtensorMap* tmO, const Waiter& w) {
+__device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, int b, int hkv, uint8_t* sQx,
+                                  AttnMisc* misc, uint32_t tmem, const CUtensorMap* tmO, const Waiter w) {
   using namespace ptx;
   constexpr uint32_t FULL = 0xffffffffu;
   const int warp = (threadIdx.x >> 5) & 3;  // TMEM lane quadrant of this warp
@@ -349,15 +409,11 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo& t, int x,
   bool ok = true;
   for (int u = 0; u < t.n_kv; ++u) {
     if (!keep_tile(p, t, b, hkv, u)) continue;
+    TRACE(x * 8192 + it * 8 + 0, wg_tid == 0);
     ok = __all_sync(FULL, w.wait(smem_addr(&misc->s_full[x]), it & 1));
     if (!ok) break;
+    TRACE(x * 8192 + it * 8 + 1, wg_tid == 0);
     tc_fence_after();
-    uint32_t s[4][32];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, s[c]);
-    tmem_wait_ld();
-#pragma unroll
-    for (int c = 0; c < 4; ++c) reg_fence(s[c]);
 
     // Column factors: K scale per 32-key chunk (token-block K scales), times cq.
     const int kv0 = u * C::BN;
@@ -369,7 +425,15 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo& t, int x,
         f = p.sf_k[bhk * p.sf_k_nblk + min(kv0 + 32 * c, p.Skv - 1) / p.sf_k_rpb];
       ck[c] = f * cq;
     }
-    // Raw scores as fp32 (INT8 products are exact s32 < 2^22: magic-number conversion).
+    int lim = p.Skv - kv0;  // keys at or past `lim` in this tile are hidden
+    if (p.causal) lim = min(lim, row + 1 + (p.Skv - p.Sq) - kv0);
+
+    uint32_t s[4][32];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, s[c]);
+    tmem_wait_ld();
+#pragma unroll
+    for (int c = 0; c < 4; ++c) reg_fence(s[c]);
     float f[4][32];
 #pragma unroll
     for (int c = 0; c < 4; ++c)
@@ -380,9 +444,6 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo& t, int x,
         else
           f[c][j] = __uint_as_float(s[c][j]);
       }
-    // Mask keys past the sequence end and (causal) past the diagonal.
-    int lim = p.Skv - kv0;
-    if (p.causal) lim = min(lim, row + 1 + (p.Skv - p.Sq) - kv0);
     if (lim < C::BN) {
 #pragma unroll
       for (int c = 0; c < 4; ++c)
@@ -392,15 +453,14 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo& t, int x,
     }
     float mc[4];
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {  // tree max: short dependency chains
-      float t[16];
+    for (int c = 0; c < 4; ++c) {
+      float a0 = fmax3(f[c][0], f[c][1], f[c][2]), a1 = fmax3(f[c][3], f[c][4], f[c][5]);
 #pragma unroll
-      for (int j = 0; j < 16; ++j) t[j] = fmaxf(f[c][j], f[c][j + 16]);
-#pragma unroll
-      for (int j = 0; j < 8; ++j) t[j] = fmaxf(t[j], t[j + 8]);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) t[j] = fmaxf(t[j], t[j + 4]);
-      mc[c] = fmaxf(fmaxf(t[0], t[1]), fmaxf(t[2], t[3])) * ck[c];
+      for (int j = 6; j < 30; j += 4) {
+        a0 = fmax3(a0, f[c][j], f[c][j + 1]);
+        a1 = fmax3(a1, f[c][j + 2], f[c][j + 3]);
+      }
+      mc[c] = fmax3(a0, a1, fmaxf(f[c][30], f[c][31])) * ck[c];
     }
     const float m_tile = fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3]));
     const float m_new = fmaxf(m, m_tile);
@@ -412,9 +472,8 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo& t, int x,
       alpha = ex2(m - m_new);
       resc = true;
       m = m_new;
-      l *= alpha;
     }
-    if (__any_sync(FULL, resc)) {  // lazy O correction, whole warp (tcgen05.ld/st are warp-wide)
+    if (__any_sync(FULL, resc)) {
 #pragma unroll 1
       for (int c = 0; c < C::D / 32; ++c) {
         uint32_t o[32];
@@ -430,29 +489,35 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo& t, int x,
 #pragma unroll
     for (int c = 0; c < 4; ++c)
 #pragma unroll
-      for (int j = 0; j < 32; ++j) f[c][j] = ex2(fmaf(f[c][j], ck[c], -mb));
+      for (int j = 0; j < 32; j += 2) ffma2(f[c][j], f[c][j + 1], f[c][j], f[c][j + 1], ck[c], ck[c], -mb, -mb);
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+#pragma unroll
+      for (int j = 0; j < 32; ++j) f[c][j] = ex2(f[c][j]);
     float rs = 0.f;
     if constexpr (C::PV == PV_BF16) {
       uint32_t pk[2][32];
-      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+      float r0 = 0.f, r1 = 0.f, r2 = 0.f, r3 = 0.f;
 #pragma unroll
       for (int c = 0; c < 4; ++c)
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          pk[c >> 1][(c & 1) * 16 + j] = pack_bf16x2(f[c][2 * j], f[c][2 * j + 1]);
-          acc[j & 7] += f[c][2 * j] + f[c][2 * j + 1];
+        for (int j = 0; j < 16; ++j) pk[c >> 1][(c & 1) * 16 + j] = pack_bf16x2(f[c][2 * j], f[c][2 * j + 1]);
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int j = 0; j < 32; j += 4) {
+          fadd2(r0, r1, r0, r1, f[c][j], f[c][j + 1]);
+          fadd2(r2, r3, r2, r3, f[c][j + 2], f[c][j + 3]);
         }
-      rs = ((acc[0] + acc[1]) + (acc[2] + acc[3])) + ((acc[4] + acc[5]) + (acc[6] + acc[7]));
+      rs = (r0 + r1) + (r2 + r3);
       tmem_st32(tS, pk[0]);
       tmem_st32(tS + 32, pk[1]);
     } else {
-      // The row sum adds the E4M3-rounded values actually stored, so the
-      // normalised weights sum to one and a dominant key returns its value.
       uint32_t pk[32];
       float racc[4];
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        uint32_t acc[2] = {0u, 0u};  // f16x2 zeros
+        uint32_t acc[2] = {0u, 0u};
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const uint32_t lo = pack_e4m3x2(f[c][4 * j], f[c][4 * j + 1]);
@@ -465,10 +530,13 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo& t, int x,
       rs = (racc[0] + racc[1]) + (racc[2] + racc[3]);
       tmem_st32(tS, pk);
     }
-    l += rs;
+    l = l * alpha + rs;
+    TRACE(x * 8192 + it * 8 + 4, wg_tid == 0);
     tmem_wait_st();
     tc_fence_before();
-    mbar_arrive(smem_addr(&misc->p_full[x]));
+    __syncwarp();  // the warp's P stores are ordered before lane 0's arrive
+    if (lane == 0) mbar_arrive(smem_addr(&misc->p_full[x]));
+    TRACE(x * 8192 + it * 8 + 5, wg_tid == 0);
     ++it;
   }
 
@@ -589,7 +657,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     mbar_init(smem_addr(&misc->q_full), 1);
     for (int x = 0; x < 2; ++x) {
       mbar_init(smem_addr(&misc->s_full[x]), 1);
-      mbar_init(smem_addr(&misc->p_full[x]), 128);
+      mbar_init(smem_addr(&misc->p_full[x]), 4);  // one arrive per softmax warp
     }
     mbar_init(smem_addr(&misc->o_full), 1);
     mbar_init(smem_addr(&misc->drain), 1);
@@ -621,14 +689,15 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   if (warp < 8) {
     regs_inc<C::SOFTMAX_REGS>();
     const int x = warp >> 2;
-    if (t[x].valid) attn_softmax_role<C>(p, t[x], x, b, hkv, sQ[x], misc, tmem, &tmO, w);
+    const TileInfo tx = x ? t[1] : t[0];  // select by value (no runtime-indexed array)
+    if (tx.valid) attn_softmax_role<C>(p, tx, x, b, hkv, x ? sQ[1] : sQ[0], misc, tmem, &tmO, w);
   } else {
     regs_dec<C::CONTROL_REGS>();
     if (warp == 8) {
-      if (lane == 0) attn_mma_role<C>(p, t, b, hkv, sQ, sSlots, misc, tmem, w);
+      if (lane == 0) attn_mma_role<C>(p, t[0], t[1], b, hkv, sQ[0], sQ[1], sSlots, misc, tmem, w);
       __syncwarp();
     } else if (warp == 9) {
-      if (lane == 0) attn_load_role<C>(p, t, b, hkv, sQ, sSlots, misc, &tmQ, &tmK, &tmV, w);
+      if (lane == 0) attn_load_role<C>(p, t[0], t[1], b, hkv, sQ[0], sQ[1], sSlots, misc, &tmQ, &tmK, &tmV, w);
       __syncwarp();
     }
   }

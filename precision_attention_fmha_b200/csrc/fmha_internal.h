@@ -6,7 +6,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "../../include/fmha.h"
+#include "fmha.h"  // include/ is on the include path
 
 namespace fmha {
 

@@ -140,6 +140,36 @@ __device__ __forceinline__ void tc_commit(uint32_t bar) {
         "tcgen05.mma.cta_group::1.kind::" KIND " [%0], [%1], %2, %3, p;\n\t}" ::"r"(d),                \
         "r"(a), "l"(b), "r"(idesc), "r"(acc));                                                          \
   }
+// Lean variants for the issue loop: descriptors given as {lo, hi} words (only
+// the low word -- start address -- changes between K-steps) and a compile-time
+// accumulate flag, so one MMA costs two integer adds plus the instruction.
+#define FMHA_DEF_MMA_SS_LEAN(NAME, KIND)                                                                   \
+  template <bool kAcc>                                                                                     \
+  __device__ __forceinline__ void NAME(uint32_t d, uint32_t a_lo, uint32_t a_hi, uint32_t b_lo, uint32_t b_hi, \
+                                       uint32_t idesc) {                                                   \
+    asm volatile(                                                                                          \
+        "{\n\t.reg .b64 ad, bd;\n\t.reg .pred p;\n\tmov.b64 ad, {%1, %2};\n\tmov.b64 bd, {%3, %4};\n\t"    \
+        "setp.ne.b32 p, %6, 0;\n\t"                                                                        \
+        "tcgen05.mma.cta_group::1.kind::" KIND " [%0], ad, bd, %5, p;\n\t}" ::"r"(d),                       \
+        "r"(a_lo), "r"(a_hi), "r"(b_lo), "r"(b_hi), "r"(idesc), "n"(kAcc ? 1 : 0));                          \
+  }
+#define FMHA_DEF_MMA_TS_LEAN(NAME, KIND)                                                                   \
+  __device__ __forceinline__ void NAME(uint32_t d, uint32_t a_tmem, uint32_t b_lo, uint32_t b_hi, uint32_t idesc, \
+                                       uint32_t acc) {                                                     \
+    asm volatile(                                                                                          \
+        "{\n\t.reg .b64 bd;\n\t.reg .pred p;\n\tmov.b64 bd, {%2, %3};\n\t"                                \
+        "setp.ne.b32 p, %5, 0;\n\t"                                                                        \
+        "tcgen05.mma.cta_group::1.kind::" KIND " [%0], [%1], bd, %4, p;\n\t}" ::"r"(d),                    \
+        "r"(a_tmem), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(acc));                                           \
+  }
+FMHA_DEF_MMA_SS_LEAN(mma_ss_f16_lean, "f16")
+FMHA_DEF_MMA_SS_LEAN(mma_ss_f8_lean, "f8f6f4")
+FMHA_DEF_MMA_SS_LEAN(mma_ss_i8_lean, "i8")
+FMHA_DEF_MMA_TS_LEAN(mma_ts_f16_lean, "f16")
+FMHA_DEF_MMA_TS_LEAN(mma_ts_f8_lean, "f8f6f4")
+#undef FMHA_DEF_MMA_SS_LEAN
+#undef FMHA_DEF_MMA_TS_LEAN
+
 FMHA_DEF_MMA_SS(mma_ss_f16, "f16")
 FMHA_DEF_MMA_SS(mma_ss_f8, "f8f6f4")
 FMHA_DEF_MMA_SS(mma_ss_i8, "i8")
@@ -216,6 +246,42 @@ __device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi) {
   uint16_t r;
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
   return r;
+}
+
+// d = max(a, b, c) (three-input max).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+// (d0, d1) = (a0, a1) * (b0, b1) + (c0, c1), one packed instruction.
+__device__ __forceinline__ void ffma2(float& d0, float& d1, float a0, float a1, float b0, float b1, float c0,
+                                      float c1) {
+  asm("{\n\t.reg .b64 a, b, c, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\tmov.b64 c, {%6, %7};\n\t"
+      "fma.rn.f32x2 d, a, b, c;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
+// (d0, d1) = (a0, a1) + (b0, b1), one packed instruction.
+__device__ __forceinline__ void fadd2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 a, b, d;\n\tmov.b64 a, {%2, %3};\n\tmov.b64 b, {%4, %5};\n\t"
+      "add.rn.f32x2 d, a, b;\n\tmov.b64 {%0, %1}, d;\n\t}"
+      : "=f"(d0), "=f"(d1)
+      : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
+}
+// Register-fence helpers for the smaller TMEM loads / stores.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
+               "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+               : "memory");
 }
 
 // Packed e4m3x2 (lo byte first) -> packed f16x2, exact.
