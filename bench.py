@@ -207,6 +207,7 @@ class Work:
                                device=dev), torch.empty(max(4, fmha.quantize_workspace_bytes(gran, B, S, x.shape[2], D)),
                                                         dtype=torch.uint8, device=dev), gran, rpb, dt)
         self.sf_p = None
+        self.p_terms = 2 if kind == "sage" else 1  # Sage: P as two E4M3 terms (the tested configuration)
         if kind == "sage":  # per-row-block P scale: P stored as 16 p
             self.sf_p = Scale(torch.full((B, Hq, math.ceil(S / 128)), 1.0 / 16, device=dev), "per_token_block", 128)
         # our kernels per step: token-block quantization is 1 launch, the grid-wide kinds 2, attention 1
@@ -228,13 +229,13 @@ class Work:
             ops[name] = out
             sfs["sf_" + name] = S_(sc, gran, rpb or 0)
         f.fmha_fwd(ops["q"], ops["k"], ops["v"], out=self.o, softmax_scale=self.scale, causal=self.causal,
-                   sf_p=self.sf_p, **sfs)
+                   sf_p=self.sf_p, p_terms=self.p_terms, **sfs)
 
     def config(self, world):
         c = {"workload": self.kind if self.kind != "pv8" else "dense_pv8", "B": self.B, "Hq": self.Hq,
              "Hkv": self.Hkv, "Sq": self.S, "Skv": self.S, "D": self.D, "causal": self.causal,
              "density": round(self.density, 6),
-             "quantized_in_step": [f"{n}:{g}" for n, _, g, _ in self.quant],
+             "quantized_in_step": [f"{n}:{g}" for n, _, g, _ in self.quant], "p_terms": self.p_terms,
              "l2": "inputs larger than L2" if self.host["q"].numel() * 2 > 126 * 2**20 else "inputs fit in L2",
              "parallelism": f"replicas{world}"}
         return c

@@ -129,6 +129,11 @@ typedef struct {
   float softmax_scale;
   int32_t causal;
   float* lse;
+  int32_t p_terms; /* E4M3 P only: 0 or 1 = P cast to one E4M3 value (3 mantissa
+                      bits); 2 = P split into two E4M3 terms hi + lo, each fed to
+                      its own PV product (about 7 significant bits, twice the PV
+                      tensor work). Must be 0 or 1 when V is BF16. */
+  int32_t reserved; /* must be 0 */
 } fmha_args;
 
 /* Block quantizer: amax -> scale = amax / R -> codes ([DiT-Sage] section 2,

@@ -118,3 +118,35 @@ def probabilities(q, k, softmax_scale, causal=False, block_mask_bh=None, block=B
     e = np.exp(s - m)
     l = np.sum(e, axis=1, keepdims=True)
     return np.divide(e, l, out=np.zeros_like(e), where=l > 0)
+
+
+def attention_rows(q_rows, rows, k, v, softmax_scale, Sq, causal=False, block_mask_bh=None, block=BLOCK):
+    """The same attention for selected query rows of one (batch, KV head).
+
+    q_rows [n, D] are the queries at absolute positions ``rows`` (of Sq); k, v
+    [Skv, D] are that KV head's keys and values; block_mask_bh is its
+    [ceil(Sq/block), ceil(Skv/block)] block mask or None. Returns
+    (o [n, D], lse [n]) in float64 -- for spot checks of full-size outputs.
+    """
+    q = np.asarray(q_rows, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    rows = np.asarray(rows)
+    Skv = k.shape[0]
+    s = softmax_scale * (q @ k.T)
+    j = np.arange(Skv)[None, :]
+    vis = np.ones(s.shape, dtype=bool)
+    if causal:
+        vis &= j <= rows[:, None] + (Skv - Sq)
+    if block_mask_bh is not None:
+        bm = np.asarray(block_mask_bh).astype(bool)
+        vis &= bm[(rows // block)[:, None], (np.arange(Skv) // block)[None, :]]
+    s = np.where(vis, s, -np.inf)
+    m = np.max(s, axis=1, keepdims=True)
+    alive = np.isfinite(m)
+    m_safe = np.where(alive, m, 0.0)
+    e = np.exp(s - m_safe)
+    l = np.sum(e, axis=1, keepdims=True)
+    p = np.divide(e, l, out=np.zeros_like(e), where=l > 0)
+    lse = np.where(alive[:, 0], m[:, 0] + np.log(np.where(l[:, 0] > 0, l[:, 0], 1.0)), -np.inf)
+    return p @ v, lse

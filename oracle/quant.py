@@ -36,14 +36,16 @@ RANGE = {"int8": 127.0, "e4m3": 448.0}
 KINDS = ("per_tensor", "per_head", "per_token_block", "per_channel")
 
 
-def _scale_from_amax(amax_f32, out_dtype):
+def scale_from_amax(amax_f32, out_dtype):
+    """scale = fp32(amax) / fp32(R), 1.0 where amax == 0."""
     amax_f32 = np.asarray(amax_f32, dtype=np.float32)
     r = np.float32(RANGE[out_dtype])
     scale = (amax_f32 / r).astype(np.float32)  # numpy float32 division is IEEE RN-even
     return np.where(amax_f32 == 0, np.float32(1.0), scale).astype(np.float32)
 
 
-def _codes(x_f32, scale_f32, out_dtype):
+def codes_with_scale(x_f32, scale_f32, out_dtype):
+    """Codes of x for a given (broadcastable) scale: RN(fp32(x) / scale)."""
     q = (np.asarray(x_f32, dtype=np.float32) / np.asarray(scale_f32, dtype=np.float32)).astype(np.float32)
     if out_dtype == "int8":
         return np.clip(np.rint(q), -127, 127).astype(np.int8)
@@ -66,17 +68,17 @@ def quantize_blockwise(x, out_dtype, kind, rows_per_block=None):
     B, S, H, D = x.shape
     codes = np.zeros(x.shape, dtype=np.int8 if out_dtype == "int8" else np.uint8)
     if kind == "per_tensor":
-        scale = _scale_from_amax(np.max(np.abs(x)) if x.size else np.float32(0), out_dtype)
-        codes[...] = _codes(x, scale, out_dtype)
+        scale = scale_from_amax(np.max(np.abs(x)) if x.size else np.float32(0), out_dtype)
+        codes[...] = codes_with_scale(x, scale, out_dtype)
         return codes, np.array([scale], dtype=np.float32)
     if kind == "per_head":
         scales = np.zeros((B, H), dtype=np.float32)
         for b in range(B):
             for h in range(H):
                 blk = x[b, :, h, :]
-                s = _scale_from_amax(np.max(np.abs(blk)) if blk.size else np.float32(0), out_dtype)
+                s = scale_from_amax(np.max(np.abs(blk)) if blk.size else np.float32(0), out_dtype)
                 scales[b, h] = s
-                codes[b, :, h, :] = _codes(blk, s, out_dtype)
+                codes[b, :, h, :] = codes_with_scale(blk, s, out_dtype)
         return codes, scales
     if kind == "per_token_block":
         if not rows_per_block or rows_per_block <= 0:
@@ -88,9 +90,9 @@ def quantize_blockwise(x, out_dtype, kind, rows_per_block=None):
                 for i in range(nblk):
                     s0, s1 = i * rows_per_block, min(S, (i + 1) * rows_per_block)
                     blk = x[b, s0:s1, h, :]
-                    s = _scale_from_amax(np.max(np.abs(blk)), out_dtype)
+                    s = scale_from_amax(np.max(np.abs(blk)), out_dtype)
                     scales[b, h, i] = s
-                    codes[b, s0:s1, h, :] = _codes(blk, s, out_dtype)
+                    codes[b, s0:s1, h, :] = codes_with_scale(blk, s, out_dtype)
         return codes, scales
     if kind == "per_channel":
         scales = np.zeros((B, H, D), dtype=np.float32)
@@ -98,9 +100,9 @@ def quantize_blockwise(x, out_dtype, kind, rows_per_block=None):
             for h in range(H):
                 for d in range(D):
                     col = x[b, :, h, d]
-                    s = _scale_from_amax(np.max(np.abs(col)) if col.size else np.float32(0), out_dtype)
+                    s = scale_from_amax(np.max(np.abs(col)) if col.size else np.float32(0), out_dtype)
                     scales[b, h, d] = s
-                    codes[b, :, h, d] = _codes(col, s, out_dtype)
+                    codes[b, :, h, d] = codes_with_scale(col, s, out_dtype)
         return codes, scales
     raise ValueError(kind)
 

@@ -234,6 +234,9 @@ fmha_status run_attention(const fmha_args* a, const uint8_t* mask, int64_t msb, 
   if ((st = check_sf(a->sf_k, "sf_k", q8, q8, q8, 32, false)) != FMHA_OK) return st;
   if ((st = check_sf(a->sf_v, "sf_v", v8, v8, false, 1, v8)) != FMHA_OK) return st;
   if ((st = check_sf(a->sf_p, "sf_p", false, v8, v8, 128, false)) != FMHA_OK) return st;
+  if (a->reserved != 0) return fail(FMHA_ERR_INVALID_ARG, "args.reserved must be 0");
+  if (a->p_terms < 0 || a->p_terms > 2) return fail(FMHA_ERR_INVALID_ARG, "p_terms must be 0, 1 or 2");
+  if (a->p_terms == 2 && !v8) return fail(FMHA_ERR_INVALID_ARG, "p_terms = 2 needs an E4M3 V");
 
   // tensors
   const bool paged = pg != nullptr;
@@ -310,6 +313,7 @@ fmha_status run_attention(const fmha_args* a, const uint8_t* mask, int64_t msb, 
   p.sf_p = a->sf_p.ptr; p.sf_p_kind = a->sf_p.kind; p.sf_p_rpb = a->sf_p.rows_per_block > 0 ? a->sf_p.rows_per_block : 1;
   p.sf_p_nblk = ceil_div(Sq, p.sf_p_rpb);
   p.lse = a->lse;
+  p.p_terms = a->p_terms == 2 ? 2 : 1;
   p.mask = mask; p.mask_sb = msb; p.mask_sh = msh;
   if (paged) {
     p.page_table = pg->page_table; p.num_pages = pg->num_pages; p.page_size = pg->page_size;

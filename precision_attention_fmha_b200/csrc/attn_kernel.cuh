@@ -55,10 +55,12 @@ static __device__ unsigned long long g_fmha_trace[FMHA_TRACE_SLOTS];  // one per
 
 namespace fmha {
 
-template <int D_, int QK_, int PV_, bool PAGED_>
+template <int D_, int QK_, int PV_, bool PAGED_, bool P2_ = false>
 struct AttnCfg {
   static constexpr int D = D_, QK = QK_, PV = PV_;
   static constexpr bool PAGED = PAGED_;
+  static constexpr bool P2 = P2_;  // E4M3 P split into two terms (hi + lo), each with its own PV product
+  static_assert(!P2 || PV == PV_E4M3, "two-term P needs an E4M3 V");
   static constexpr int BM = 128, BN = 128;
   static constexpr int QK_ELEM = QK == QK_BF16 ? 2 : 1;
   static constexpr int V_ELEM = PV == PV_BF16 ? 2 : 1;
@@ -323,6 +325,8 @@ __device__ void attn_mma_role(const AttnParams& p, const TileInfo t0, const Tile
         TRACE(16384 + u * 16 + x * 8 + 1, true);
         tc_fence_after();
         issue_pv<C>(tmem + o_col[x], tmem + s_col[x], v_lo0 + pend[x] * (C::SLOT >> 4), hi, pv_cnt[x] > 0);
+        if constexpr (C::P2)  // the low E4M3 term of P
+          issue_pv<C>(tmem + o_col[x], tmem + s_col[x] + 32, v_lo0 + pend[x] * (C::SLOT >> 4), hi, 1u);
         TRACE(16384 + u * 16 + x * 8 + 2, true);
         ++pv_cnt[x];
         pend[x] = -1;
@@ -357,6 +361,8 @@ __device__ void attn_mma_role(const AttnParams& p, const TileInfo t0, const Tile
     if (!(ok = w.wait(smem_addr(&misc->p_full[x]), pv_cnt[x] & 1))) break;
     tc_fence_after();
     issue_pv<C>(tmem + o_col[x], tmem + s_col[x], v_lo0 + pend[x] * (C::SLOT >> 4), hi, pv_cnt[x] > 0);
+    if constexpr (C::P2)
+      issue_pv<C>(tmem + o_col[x], tmem + s_col[x] + 32, v_lo0 + pend[x] * (C::SLOT >> 4), hi, 1u);
   }
   if (ok) tc_commit(smem_addr(&misc->o_full));
   // Drain: arrives when every MMA issued above has completed.
@@ -512,6 +518,28 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, 
       rs = (r0 + r1) + (r2 + r3);
       tmem_st32(tS, pk[0]);
       tmem_st32(tS + 32, pk[1]);
+    } else if constexpr (C::P2) {
+      // Two-term E4M3 P: hi = E4M3(p g), lo = E4M3(p g - hi) (the residual taken in
+      // f16), ~7 significant bits between them; both feed their own PV product.
+      // The row sum adds the unrounded values (the pair is as precise as BF16).
+      uint32_t pk[32], pl[32];
+      float r0 = 0.f, r1 = 0.f, r2 = 0.f, r3 = 0.f;
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const float* e = &f[c][4 * j];
+          const uint32_t h01 = pack_e4m3x2(e[0], e[1]), h23 = pack_e4m3x2(e[2], e[3]);
+          pk[c * 8 + j] = h01 | (h23 << 16);
+          const uint32_t d01 = hsub2(pack_f16x2(e[0], e[1]), e4m3x2_to_f16x2(h01));
+          const uint32_t d23 = hsub2(pack_f16x2(e[2], e[3]), e4m3x2_to_f16x2(h23));
+          pl[c * 8 + j] = f16x2_to_e4m3x2(d01) | (f16x2_to_e4m3x2(d23) << 16);
+          fadd2(r0, r1, r0, r1, e[0], e[1]);
+          fadd2(r2, r3, r2, r3, e[2], e[3]);
+        }
+      rs = (r0 + r1) + (r2 + r3);
+      tmem_st32(tS, pk);
+      tmem_st32(tS + 32, pl);
     } else {
       uint32_t pk[32];
       float racc[4];

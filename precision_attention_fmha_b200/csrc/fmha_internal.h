@@ -44,6 +44,7 @@ struct AttnParams {
   const uint8_t* mask; int64_t mask_sb, mask_sh;
   // paged K/V (page_table == nullptr: contiguous)
   const int32_t* page_table; int32_t num_pages, page_size, max_pages_per_seq;
+  int32_t p_terms;      // 1 or 2 E4M3 terms for P (E4M3 V only)
   uint32_t* err;        // device error word
   uint64_t wait_cycles; // bound on one wait
 };

@@ -284,6 +284,24 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
                : "memory");
 }
 
+// Two fp32 -> packed f16x2 (lo in bits 0..15), round to nearest even.
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+__device__ __forceinline__ uint32_t hsub2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+// Packed f16x2 -> packed e4m3x2 (in the low 16 bits), round to nearest even, saturating.
+__device__ __forceinline__ uint32_t f16x2_to_e4m3x2(uint32_t v) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f16x2 %0, %1;" : "=h"(r) : "r"(v));
+  return r;
+}
+
 // Packed e4m3x2 (lo byte first) -> packed f16x2, exact.
 __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t v) {
   uint32_t r;

@@ -1,0 +1,139 @@
+"""Full-size parity: every workload at its full size, in the launch
+configuration bench.py times (GPU quantizer -> attention), checked on sampled
+outputs the oracle computes row by row.
+
+For a few sampled (batch, head) pairs the oracle quantizes that head's
+operands itself (per-tensor scales use the oracle's amax over the whole
+tensor), the GPU codes of those heads must match bit for bit, and sampled
+query rows (first, boundary, last and random rows) must match the oracle's
+float64 attention within the path's tolerance.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import attention as oa
+from oracle import quant as oq
+from precision_attention_fmha_b200 import fmha, workloads
+from precision_attention_fmha_b200.fmha import Scale
+from tests.helpers import BF16_ATOL, Q8_ATOL, Q8_COS, codes_np, cos_per_head, f32, f64
+
+pytestmark = [pytest.mark.gpu, pytest.mark.big]
+DEV = torch.device("cuda")
+TDT = {"int8": torch.int8, "e4m3": torch.float8_e4m3fn}
+
+
+def sample_rows(S, n_random=8, seed=0):
+    rng = np.random.default_rng(seed)
+    fixed = [0, 1, 2, 127, 128, S // 2, S - 2, S - 1]
+    return np.unique(np.clip(np.concatenate([fixed, rng.integers(0, S, n_random)]), 0, S - 1))
+
+
+def oracle_head(x_bf16, b, h, spec, full_x=None):
+    """Oracle dequantized operand of one (b, h) slice [S, D] (float64), plus its codes.
+    spec None = BF16 operand used as is."""
+    xs = f32(x_bf16[b:b + 1, :, h:h + 1, :])
+    if spec is None:
+        return xs[0, :, 0].astype(np.float64), None
+    out, kind, rpb = spec
+    if kind == "per_tensor":  # the scale comes from the whole tensor's amax
+        scale = oq.scale_from_amax(np.max(np.abs(f32(full_x))), out)
+        codes = oq.codes_with_scale(xs, scale, out)
+        deq = oq.dequantize(codes, np.array([scale]), out, "per_tensor")
+    else:
+        codes, sc = oq.quantize_blockwise(xs, out, kind, rpb)
+        deq = oq.dequantize(codes, sc, out, kind, rpb)
+    return deq[0, :, 0], codes[0, :, 0]
+
+
+def check_rows(mode, got_rows, ref_rows):
+    """got/ref: dict (b, h) -> [n, D] arrays."""
+    for key in ref_rows:
+        g, r = got_rows[key], ref_rows[key]
+        assert np.all(np.isfinite(g)), f"non-finite output at {key}"
+        err = np.abs(g - r).max()
+        if mode == "bf16":
+            assert err <= BF16_ATOL, f"{key}: max-abs {err:.3e}"
+        else:
+            scale = max(1.0, np.abs(r).max())
+            assert err <= Q8_ATOL * scale, f"{key}: max-abs {err:.3e} > {Q8_ATOL} x {scale:.2f}"
+            c = cos_per_head(g[None, :, None, :], r[None, :, None, :])[0]
+            assert c >= Q8_COS, f"{key}: cos {c:.6f}"
+
+
+def run_case(mode, q, k, v, specs, heads, causal=False, sf_p=None, p_terms=1):
+    """Quantize on the GPU exactly as bench.py does, run attention, compare sampled rows."""
+    B, Sq, Hq, D = q.shape
+    Skv = k.shape[1]
+    group = Hq // k.shape[2]
+    ops, sfs = {"q": q.to(DEV), "k": k.to(DEV), "v": v.to(DEV)}, {}
+    host = {"q": q, "k": k, "v": v}
+    for name, spec in specs.items():
+        out, kind, rpb = spec
+        c, sc = fmha.fmha_quantize_blockwise(ops[name], TDT[out], kind, rpb)
+        ops[name], sfs["sf_" + name] = c, Scale(sc, kind, rpb or 0)
+    o = fmha.fmha_fwd(ops["q"], ops["k"], ops["v"], softmax_scale=1 / math.sqrt(D), causal=causal, sf_p=sf_p,
+                      p_terms=p_terms, **sfs)
+    fmha.get_device_error()
+    got, ref = {}, {}
+    for (b, h) in heads:
+        hk = h // group
+        opr = {}
+        for name, hh in (("q", h), ("k", hk), ("v", hk)):
+            spec = specs.get(name)
+            deq, codes = oracle_head(host[name], b, hh, spec, host[name] if spec and spec[1] == "per_tensor" else None)
+            if codes is not None:  # GPU codes of this head must equal the oracle's
+                gc = codes_np(ops[name][b:b + 1, :, hh:hh + 1, :].contiguous())[0, :, 0]
+                assert np.array_equal(gc, codes), f"{name} codes differ for head ({b}, {hh})"
+            opr[name] = deq
+        rows = sample_rows(Sq, seed=b * 131 + h)
+        ro, _ = oa.attention_rows(opr["q"][rows], rows, opr["k"], opr["v"], 1 / math.sqrt(D), Sq, causal)
+        ref[(b, h)] = ro
+        got[(b, h)] = f64(o[b, rows, h, :])
+    check_rows(mode, got, ref)
+
+
+@pytest.mark.parametrize("S", [4096, 16384, 32768])
+def test_dense_pv8_full_size(S):
+    w = workloads.dense_pv8(S=S)
+    run_case("pv8", w["q"], w["k"], w["v"], {"v": ("e4m3", "per_tensor", None)}, heads=[(0, 0), (0, 17), (0, 39)])
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_all_fp8_full_size(causal):
+    w = workloads.all_fp8()
+    spec = {n: ("e4m3", "per_head", None) for n in "qkv"}
+    run_case("fp8", w["q"], w["k"], w["v"], spec, heads=[(0, 0), (1, 13), (1, 31)], causal=causal)
+
+
+def test_sage_full_size():
+    w = workloads.sage()
+    B, S, H, D = w["q"].shape
+    spec = {"q": ("int8", "per_token_block", 128), "k": ("int8", "per_token_block", 64),
+            "v": ("e4m3", "per_channel", None)}
+    sf_p = Scale(torch.full((B, H, math.ceil(S / 128)), 1.0 / 16, device=DEV), "per_token_block", 128)
+    run_case("sage", w["q"], w["k"], w["v"], spec, heads=[(0, 0), (0, 11), (0, 23)], sf_p=sf_p, p_terms=2)
+
+
+def test_sparse_paged_full_size():
+    w = workloads.sparse_paged()
+    B, S, Hq, D = w["q"].shape
+    Hkv = w["k"].shape[2]
+    group = Hq // Hkv
+    o = fmha.fmha_fwd_paged(w["q"].to(DEV), w["k_pool"].to(DEV), w["v_pool"].to(DEV), w["page_table"].to(DEV), S,
+                            mask=w["mask"].to(DEV), softmax_scale=w["scale"])
+    fmha.get_device_error()
+    mask = w["mask"].numpy()
+    got, ref = {}, {}
+    for (b, h) in [(0, 0), (1, 21), (3, 63)]:
+        hk = h // group
+        kk = oa.gather_paged(f64(w["k_pool"][:, :, hk:hk + 1]), w["page_table"].numpy()[b:b + 1], S)[0, :, 0]
+        vv = oa.gather_paged(f64(w["v_pool"][:, :, hk:hk + 1]), w["page_table"].numpy()[b:b + 1], S)[0, :, 0]
+        rows = sample_rows(S, seed=b * 7 + h)
+        ro, _ = oa.attention_rows(f64(w["q"][b, rows, h, :]), rows, kk, vv, w["scale"], S, False, mask[b, hk])
+        ref[(b, h)] = ro
+        got[(b, h)] = f64(o[b, rows, h, :])
+    check_rows("bf16", got, ref)

@@ -79,8 +79,9 @@ def run_dense(mode, B, Hq, Hkv, Sq, Skv, D, causal, seed, with_lse=False):
     sf_p = None
     if mode == "sage":  # per-row-block P scale: P is stored as 16 p (lazy-rescale bound 2^4 * 16 <= 448)
         sf_p = Scale(torch.full((B, Hq, math.ceil(Sq / 128)), 1 / 16, device=DEV), "per_token_block", 128)
+    p_terms = 2 if mode == "sage" else 1  # Sage: P as two E4M3 terms (its sharp softmax needs the precision)
     o = fmha.fmha_fwd(g["q"], g["k"], g["v"], sf_q=g["sf_q"], sf_k=g["sf_k"], sf_v=g["sf_v"], sf_p=sf_p,
-                      softmax_scale=scale, causal=causal, lse=lse)
+                      softmax_scale=scale, causal=causal, lse=lse, p_terms=p_terms)
     fmha.get_device_error()
     ref_o, ref_lse = oa.attention(rq, rk, rv, scale, causal)
     check(mode, o, ref_o)
@@ -88,8 +89,9 @@ def run_dense(mode, B, Hq, Hkv, Sq, Skv, D, causal, seed, with_lse=False):
         got = lse.cpu().numpy().astype(np.float64)
         fin = np.isfinite(ref_lse)
         assert np.array_equal(np.isfinite(got), fin)
-        # BF16 P: exact sum of p; E4M3 P: the sum of the stored rounded P (|err| <= ln(1 + 2^-4))
-        bound = 2e-2 if mode == "bf16" else math.log1p(2.0 ** -4) + 2e-3
+        # BF16 P and two-term E4M3 P: exact sum of p; one-term E4M3 P: the sum of the
+        # stored rounded P (|err| <= ln(1 + 2^-4))
+        bound = 2e-2 if mode in ("bf16", "sage") else math.log1p(2.0 ** -4) + 2e-3
         assert np.abs(got[fin] - ref_lse[fin]).max() < bound
     return o
 
@@ -193,4 +195,29 @@ def test_invalid_arguments_raise():
     q, k, v = workloads.normal_qkv(5, 1, 64, 64, 2, 2, 128)
     with pytest.raises(fmha.FmhaError) as e:
         fmha.fmha_fwd(q.to(DEV), k[:, :, :1].to(DEV).expand(1, 64, 2, 128), v.to(DEV), causal=True)
+    assert e.value.status == 1
+
+
+@pytest.mark.parametrize("mode", ["pv8", "fp8"])
+def test_two_term_p_is_more_accurate(mode):
+    """P split into two E4M3 terms must cut the error against the oracle well below
+    the one-term error and stay within the 8-bit tolerance."""
+    B, Hq, Hkv, S, D = 1, 2, 2, 1024, 128
+    q, k, v = workloads.normal_qkv(31, B, S, S, Hq, Hkv, D)
+    g, rq, rk, rv = prepare(mode, q, k, v)
+    ref, _ = oa.attention(rq, rk, rv, 1 / math.sqrt(D), True)
+    errs = []
+    for terms in (1, 2):
+        o = fmha.fmha_fwd(g["q"], g["k"], g["v"], sf_q=g["sf_q"], sf_k=g["sf_k"], sf_v=g["sf_v"], causal=True,
+                          p_terms=terms)
+        fmha.get_device_error()
+        check(mode, o, ref)
+        errs.append(np.abs(f64(o) - ref).max())
+    assert errs[1] < errs[0] / 3, errs
+
+
+def test_two_term_p_needs_8bit_v():
+    q, k, v = workloads.normal_qkv(32, 1, 64, 64, 1, 1, 128)
+    with pytest.raises(fmha.FmhaError) as e:
+        fmha.fmha_fwd(q.to(DEV), k.to(DEV), v.to(DEV), p_terms=2)
     assert e.value.status == 1

@@ -207,3 +207,18 @@ def test_fully_masked_rows_give_zero_and_minus_inf():
     o, lse = A.attention(q, k, v, 1.0, causal=True)  # Sq > Skv: rows 0..5 see nothing
     assert np.all(o[0, :6] == 0) and np.all(np.isneginf(lse[0, 0, :6]))
     assert np.allclose(o[0, 6, 0], v[0, 0, 0])
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_sampled_rows_equal_full_attention(causal):
+    rng = np.random.default_rng(22)
+    Sq, Skv, D, blk = 300, 420, 16, 64
+    q, k, v = _rand(rng, 1, Sq, 1, D), _rand(rng, 1, Skv, 1, D), _rand(rng, 1, Skv, 1, D)
+    bm = rng.random((1, 1, -(-Sq // blk), -(-Skv // blk))) < 0.6
+    bm[..., -1] = True
+    o, lse = A.attention(q, k, v, 0.3, causal, bm, blk)
+    rows = np.array([0, 1, 63, 64, 150, 299])
+    o2, lse2 = A.attention_rows(q[0, rows, 0], rows, k[0, :, 0], v[0, :, 0], 0.3, Sq, causal, bm[0, 0], blk)
+    assert np.allclose(o2, o[0, rows, 0], atol=1e-14)
+    fin = np.isfinite(lse[0, 0, rows])
+    assert np.array_equal(np.isfinite(lse2), fin) and np.allclose(lse2[fin], lse[0, 0, rows][fin], atol=1e-13)
