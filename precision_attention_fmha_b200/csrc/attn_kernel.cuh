@@ -75,12 +75,21 @@ struct AttnCfg {
   static constexpr int K_TILE = BN * QK_ROW_BYTES;
   static constexpr int V_TILE = BN * D * V_ELEM;
   static constexpr int SLOT = K_TILE > V_TILE ? K_TILE : V_TILE;
+  // E4M3 P is staged in shared memory (one 128 x 128 byte tile per query tile
+  // and term) so that a tile's S buffer in TMEM is free as soon as the softmax
+  // has loaded it: QK^T of the next KV tile then overlaps this tile's exp2
+  // ("FlashInfer FP8/BF16 mixed-precision attention for Blackwell", section 1).
+  // BF16 P stays in TMEM (staging it would leave too little room for K/V).
+  static constexpr bool PSMEM = PV == PV_E4M3;
+  static constexpr bool TURNS = PSMEM;  // exp-phase turn-taking between the softmax warpgroups
+  static constexpr int P_TILE = BM * BN;  // bytes per E4M3 P tile
+  static constexpr int P_BYTES = PSMEM ? 2 * P_TILE * (P2 ? 2 : 1) : 0;
   static constexpr int MISC_BYTES = 1024;
   static constexpr int SMEM_CAP = 232448;  // 227 KB opt-in maximum per CTA
-  static constexpr int STAGES_FIT = (SMEM_CAP - 1024 - MISC_BYTES - 2 * Q_TILE) / SLOT;
+  static constexpr int STAGES_FIT = (SMEM_CAP - 1024 - MISC_BYTES - 2 * Q_TILE - P_BYTES) / SLOT;
   static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
   static_assert(STAGES >= 3, "the K/V ring needs at least three slots");
-  static constexpr int SMEM_BYTES = 1024 + 2 * Q_TILE + STAGES * SLOT + MISC_BYTES;
+  static constexpr int SMEM_BYTES = 1024 + 2 * Q_TILE + P_BYTES + STAGES * SLOT + MISC_BYTES;
   static constexpr int QK_STEPS = QK_ROW_BYTES / 32;  // one MMA covers 32 bytes of K (16 bf16 / 32 8-bit)
   static constexpr int PV_K = PV == PV_BF16 ? 16 : 32;
   static constexpr int PV_STEPS = BN / PV_K;
@@ -95,6 +104,11 @@ struct AttnCfg {
   // Launch: 384 threads x 168 registers = 64512; after re-balancing
   // 2 x 128 x 224 + 128 x 56 = 64512 (the sum must not exceed the launch total).
   static constexpr int THREADS = 384;
+  // Warp roles: warpgroup 0 = control (MMA issue, TMA loads, two idle warps),
+  // warpgroups 1 and 2 = softmax of query tiles 0 and 1. The control warps
+  // come first: the issue scheduler favours older warps, and the MMA warp's
+  // short serial steps sit on the critical path of both softmax pipelines.
+  static constexpr int MMA_WARP = 0, LOAD_WARP = 1, SOFTMAX_WARP0 = 4;
   static constexpr uint32_t SOFTMAX_REGS = 224, CONTROL_REGS = 56;
   static_assert(2 * 128 * SOFTMAX_REGS + 128 * CONTROL_REGS <= THREADS * 168, "register split exceeds launch");
 };
@@ -105,6 +119,9 @@ struct alignas(8) AttnMisc {
   uint64_t p_full[2];
   uint64_t o_full;
   uint64_t drain;
+  uint64_t s_free[2];   // shared-memory P: the softmax has loaded S, its TMEM may be overwritten
+  uint64_t pv_done[2];  // shared-memory P: a PV product finished (O current, P buffer free)
+  uint64_t exp_done[2];  // softmax warpgroup x finished the exponentials of its current tile
   uint64_t kv_full[8];
   uint64_t kv_empty[8];
   uint32_t tmem_base;
@@ -139,10 +156,14 @@ struct Waiter {
     }
   }
   // Teardown wait: ignores the abort flag (used to drain in-flight async work).
+  // Its limit never drops below ~1 s, whatever the wait limit is set to: a copy
+  // or MMA already issued always completes, and shared memory / TMEM must not
+  // be released under it.
   __device__ __forceinline__ bool drain(uint32_t bar, uint32_t parity) const {
+    const uint64_t limit = budget > (1ull << 31) ? budget : (1ull << 31);
     const long long t0 = clock64();
     while (!ptx::mbar_try_wait(bar, parity)) {
-      if (static_cast<uint64_t>(clock64() - t0) > budget) {
+      if (static_cast<uint64_t>(clock64() - t0) > limit) {
         atomicOr(err, kErrTimeout);
         return false;
       }
@@ -232,11 +253,12 @@ __device__ void attn_load_role(const AttnParams& p, const TileInfo t0, const Til
       }
     }
   }
-  if (*w.abort_flag) {  // let every issued copy land before shared memory goes away
-    w.drain(q_full, 0);
-    for (int s = 0; s < C::STAGES; ++s)
-      if (issued & (1u << s)) w.drain(smem_addr(&misc->kv_full[s]), (issued_phase >> s) & 1u);
-  }
+  // Every issued copy lands before shared memory goes away. Without an abort
+  // the consumers have already seen these phases complete (no waiting); after
+  // an abort, set by any role at any time, copies may still be in flight.
+  w.drain(q_full, 0);
+  for (int s = 0; s < C::STAGES; ++s)
+    if (issued & (1u << s)) w.drain(smem_addr(&misc->kv_full[s]), (issued_phase >> s) & 1u);
 }
 
 // ------------------------------------------------------- tensor-core issue --
@@ -287,10 +309,16 @@ __device__ __forceinline__ void issue_pv(uint32_t tmem_o, uint32_t tmem_p, uint3
   }
 }
 
+// MMA issue (TMEM P). The whole warp walks the schedule -- waits, slot and
+// phase bookkeeping, descriptor words -- in warp-uniform control flow, and one
+// elected lane issues the MMAs and commits, so the address arithmetic stays
+// off the issuing lane's critical path.
 template <class C>
 __device__ void attn_mma_role(const AttnParams& p, const TileInfo t0, const TileInfo t1, int b, int hkv, uint8_t* sQ0,
                               uint8_t* sQ1, uint8_t* sSlots, AttnMisc* misc, uint32_t tmem, const Waiter w) {
   using namespace ptx;
+  constexpr uint32_t FULL = 0xffffffffu;
+  const bool leader = elect_one();
   const uint32_t s_col[2] = {0u, 128u};
   // Descriptor words, computed once: K-major Q/K (leading offset unused, 16),
   // MN-major V (leading offset = distance between d column blocks).
@@ -304,12 +332,12 @@ __device__ void attn_mma_role(const AttnParams& p, const TileInfo t0, const Tile
   int prev_v = -1;
   int slot_it = 0;
   const int n_u = max(t0.n_kv, t1.n_kv);
-  bool ok = w.wait(smem_addr(&misc->q_full), 0);
+  bool ok = __all_sync(FULL, w.wait(smem_addr(&misc->q_full), 0));
   tc_fence_after();
   for (int u = 0; u < n_u && ok; ++u) {
     const bool kx[2] = {keep_tile(p, t0, b, hkv, u), keep_tile(p, t1, b, hkv, u)};
     if (!kx[0] && !kx[1]) continue;
-    TRACE(16384 + u * 16 + 15, true);
+    TRACE(16384 + u * 16 + 15, leader);
     const int ks = slot_it % C::STAGES;
     const uint32_t kph = (slot_it / C::STAGES) & 1;
     ++slot_it;
@@ -320,37 +348,44 @@ __device__ void attn_mma_role(const AttnParams& p, const TileInfo t0, const Tile
 #pragma unroll
     for (int x = 0; x < 2 && ok; ++x) {
       if (pend[x] >= 0) {  // PV of the previous tile first: S_x(u) overwrites P_x
-        TRACE(16384 + u * 16 + x * 8 + 0, true);
-        if (!(ok = w.wait(smem_addr(&misc->p_full[x]), pv_cnt[x] & 1))) break;
-        TRACE(16384 + u * 16 + x * 8 + 1, true);
+        TRACE(16384 + u * 16 + x * 8 + 0, leader);
+        if (!(ok = __all_sync(FULL, w.wait(smem_addr(&misc->p_full[x]), pv_cnt[x] & 1)))) break;
+        TRACE(16384 + u * 16 + x * 8 + 1, leader);
         tc_fence_after();
-        issue_pv<C>(tmem + o_col[x], tmem + s_col[x], v_lo0 + pend[x] * (C::SLOT >> 4), hi, pv_cnt[x] > 0);
-        if constexpr (C::P2)  // the low E4M3 term of P
-          issue_pv<C>(tmem + o_col[x], tmem + s_col[x] + 32, v_lo0 + pend[x] * (C::SLOT >> 4), hi, 1u);
-        TRACE(16384 + u * 16 + x * 8 + 2, true);
+        if (leader) {
+          issue_pv<C>(tmem + o_col[x], tmem + s_col[x], v_lo0 + pend[x] * (C::SLOT >> 4), hi, pv_cnt[x] > 0);
+          if constexpr (C::P2)  // the low E4M3 term of P
+            issue_pv<C>(tmem + o_col[x], tmem + s_col[x] + 32, v_lo0 + pend[x] * (C::SLOT >> 4), hi, 1u);
+        }
+        __syncwarp();
+        TRACE(16384 + u * 16 + x * 8 + 2, leader);
         ++pv_cnt[x];
         pend[x] = -1;
       }
       if (kx[x]) {
         if (!k_ready) {
-          if (!(ok = w.wait(smem_addr(&misc->kv_full[ks]), kph))) break;
+          if (!(ok = __all_sync(FULL, w.wait(smem_addr(&misc->kv_full[ks]), kph)))) break;
           tc_fence_after();
           k_ready = true;
         }
-        TRACE(16384 + u * 16 + x * 8 + 3, true);
-        issue_qk<C>(tmem + s_col[x], x ? q_lo1 : q_lo0, k_lo0 + ks * (C::SLOT >> 4), hi);
-        TRACE(16384 + u * 16 + x * 8 + 4, true);
-        tc_commit(smem_addr(&misc->s_full[x]));
-        TRACE(16384 + u * 16 + x * 8 + 5, true);
+        TRACE(16384 + u * 16 + x * 8 + 3, leader);
+        if (leader) {
+          issue_qk<C>(tmem + s_col[x], x ? q_lo1 : q_lo0, k_lo0 + ks * (C::SLOT >> 4), hi);
+          tc_commit(smem_addr(&misc->s_full[x]));
+        }
+        __syncwarp();
+        TRACE(16384 + u * 16 + x * 8 + 5, leader);
       }
     }
     if (!ok) break;
-    tc_commit(smem_addr(&misc->kv_empty[ks]));                     // K_u free once the S MMAs finish
-    if (prev_v >= 0) tc_commit(smem_addr(&misc->kv_empty[prev_v]));  // previous V: its PVs are issued
-    if (!(ok = w.wait(smem_addr(&misc->kv_full[vs]), vph))) break;
-    TRACE(16384 + u * 16 + 7, true);
+    if (leader) {
+      tc_commit(smem_addr(&misc->kv_empty[ks]));                     // K_u free once the S MMAs finish
+      if (prev_v >= 0) tc_commit(smem_addr(&misc->kv_empty[prev_v]));  // previous V: its PVs are issued
+    }
+    __syncwarp();
+    if (!(ok = __all_sync(FULL, w.wait(smem_addr(&misc->kv_full[vs]), vph)))) break;
+    TRACE(16384 + u * 16 + 7, leader);
     tc_fence_after();
-    TRACE(16384 + u * 16 + 14, true);
     pend[0] = kx[0] ? vs : -1;
     pend[1] = kx[1] ? vs : -1;
     prev_v = vs;
@@ -358,15 +393,147 @@ __device__ void attn_mma_role(const AttnParams& p, const TileInfo t0, const Tile
 #pragma unroll
   for (int x = 0; x < 2 && ok; ++x) {
     if (pend[x] < 0) continue;
-    if (!(ok = w.wait(smem_addr(&misc->p_full[x]), pv_cnt[x] & 1))) break;
+    if (!(ok = __all_sync(FULL, w.wait(smem_addr(&misc->p_full[x]), pv_cnt[x] & 1)))) break;
     tc_fence_after();
-    issue_pv<C>(tmem + o_col[x], tmem + s_col[x], v_lo0 + pend[x] * (C::SLOT >> 4), hi, pv_cnt[x] > 0);
-    if constexpr (C::P2)
-      issue_pv<C>(tmem + o_col[x], tmem + s_col[x] + 32, v_lo0 + pend[x] * (C::SLOT >> 4), hi, 1u);
+    if (leader) {
+      issue_pv<C>(tmem + o_col[x], tmem + s_col[x], v_lo0 + pend[x] * (C::SLOT >> 4), hi, pv_cnt[x] > 0);
+      if constexpr (C::P2)
+        issue_pv<C>(tmem + o_col[x], tmem + s_col[x] + 32, v_lo0 + pend[x] * (C::SLOT >> 4), hi, 1u);
+    }
+    __syncwarp();
   }
-  if (ok) tc_commit(smem_addr(&misc->o_full));
   // Drain: arrives when every MMA issued above has completed.
-  tc_commit(smem_addr(&misc->drain));
+  if (leader) {
+    if (ok) tc_commit(smem_addr(&misc->o_full));
+    tc_commit(smem_addr(&misc->drain));
+  }
+  __syncwarp();
+  w.drain(smem_addr(&misc->drain), 0);
+}
+
+// Shared-memory P: O += P V with P (A operand, K-major, 128-byte swizzle)
+// read from shared memory. K-steps of 32 keys advance 32 bytes in the row.
+template <class C>
+__device__ __forceinline__ void issue_pv_ss(uint32_t tmem_o, uint32_t p_lo, uint32_t v_lo, uint32_t hi,
+                                            uint32_t accumulate) {
+#pragma unroll
+  for (int s = 0; s < C::PV_STEPS; ++s)
+    ptx::mma_ss_f8_lean_acc(tmem_o, p_lo + ((s * 32) >> 4), hi, v_lo + ((s * C::PV_K * 128) >> 4), hi,
+                            C::IDESC_PV, s > 0 ? 1u : accumulate);
+}
+
+// MMA issue for the shared-memory-P pipeline. Per kept KV tile u (in order):
+//   QK^T of the NEXT kept tile for each query tile, as soon as that tile's
+//   softmax has loaded its current S (s_free) -- this overlaps the softmax;
+//   then PV of tile u once P_x(u) is in shared memory (p_full), committed to
+//   pv_done[x], which the softmax waits on before it rewrites P or O.
+template <class C>
+__device__ void attn_mma_role_psmem(const AttnParams& p, const TileInfo t0, const TileInfo t1, int b, int hkv,
+                                    uint8_t* sQ0, uint8_t* sQ1, uint8_t* sP0, uint8_t* sP1, uint8_t* sSlots,
+                                    AttnMisc* misc, uint32_t tmem, const Waiter w) {
+  using namespace ptx;
+  constexpr uint32_t FULL = 0xffffffffu;
+  const bool leader = elect_one();
+  const uint32_t hi = desc_hi(1024, 2);
+  const uint32_t q_lo0 = desc_lo(smem_addr(sQ0), 16), q_lo1 = desc_lo(smem_addr(sQ1), 16);
+  const uint32_t p_lo0 = desc_lo(smem_addr(sP0), 16), p_lo1 = desc_lo(smem_addr(sP1), 16);
+  const uint32_t k_lo0 = desc_lo(smem_addr(sSlots), 16);
+  const uint32_t v_lo0 = desc_lo(smem_addr(sSlots), C::CHUNK_BYTES);
+  const uint32_t s_col[2] = {0u, 128u};
+  const uint32_t o_col[2] = {256u, 256u + C::D};
+  const int n_u = max(t0.n_kv, t1.n_kv);
+  int s_cnt[2] = {0, 0}, pv_cnt[2] = {0, 0};
+  int slot_it = 0;
+  bool ok = __all_sync(FULL, w.wait(smem_addr(&misc->q_full), 0));
+  tc_fence_after();
+  auto next_kept = [&](int from) {
+    int u = from;
+    while (u < n_u && !keep_tile(p, t0, b, hkv, u) && !keep_tile(p, t1, b, hkv, u)) ++u;
+    return u;
+  };
+  // Issues S_x(u) for every query tile keeping u; K_u lives in slot ks.
+  auto issue_s = [&](int u, int ks) {
+#pragma unroll
+    for (int x = 0; x < 2; ++x) {
+      if (!keep_tile(p, x ? t1 : t0, b, hkv, u)) continue;
+      if (s_cnt[x] > 0) {  // the softmax must have loaded this tile's previous S
+        if (!(ok = __all_sync(FULL, w.wait(smem_addr(&misc->s_free[x]), (s_cnt[x] - 1) & 1)))) return;
+        tc_fence_after();
+      }
+      TRACE(16384 + u * 16 + 10 + x, leader);
+      if (leader) {
+        issue_qk<C>(tmem + s_col[x], x ? q_lo1 : q_lo0, k_lo0 + ks * (C::SLOT >> 4), hi);
+        tc_commit(smem_addr(&misc->s_full[x]));
+      }
+      __syncwarp();
+      ++s_cnt[x];
+    }
+  };
+  int u = next_kept(0);
+  int vs = 0;
+  if (u < n_u && ok) {
+    const int ks = slot_it % C::STAGES;
+    const uint32_t kph = (slot_it / C::STAGES) & 1;
+    ++slot_it;
+    vs = slot_it % C::STAGES;
+    ++slot_it;
+    if ((ok = __all_sync(FULL, w.wait(smem_addr(&misc->kv_full[ks]), kph)))) {
+      tc_fence_after();
+      issue_s(u, ks);
+      if (leader) tc_commit(smem_addr(&misc->kv_empty[ks]));
+      __syncwarp();
+    }
+  }
+  while (u < n_u && ok) {
+    TRACE(16384 + u * 16 + 0, leader);
+    const int vph_it = slot_it - 1;  // ring position of V_u
+    const uint32_t vph = (vph_it / C::STAGES) & 1;
+    const int nu = next_kept(u + 1);
+    int nvs = 0;
+    if (nu < n_u) {  // QK^T of the next kept tile, overlapping this tile's softmax
+      const int nks = slot_it % C::STAGES;
+      const uint32_t nkph = (slot_it / C::STAGES) & 1;
+      ++slot_it;
+      nvs = slot_it % C::STAGES;
+      ++slot_it;
+      if (!(ok = __all_sync(FULL, w.wait(smem_addr(&misc->kv_full[nks]), nkph)))) break;
+      tc_fence_after();
+      TRACE(16384 + u * 16 + 1, leader);
+      issue_s(nu, nks);
+      if (!ok) break;
+      if (leader) tc_commit(smem_addr(&misc->kv_empty[nks]));
+      __syncwarp();
+    }
+    TRACE(16384 + u * 16 + 2, leader);
+    if (!(ok = __all_sync(FULL, w.wait(smem_addr(&misc->kv_full[vs]), vph)))) break;
+    TRACE(16384 + u * 16 + 3, leader);
+    tc_fence_after();
+#pragma unroll
+    for (int x = 0; x < 2; ++x) {
+      if (!keep_tile(p, x ? t1 : t0, b, hkv, u)) continue;
+      TRACE(16384 + u * 16 + 4 + x * 3, leader);
+      if (!(ok = __all_sync(FULL, w.wait(smem_addr(&misc->p_full[x]), pv_cnt[x] & 1)))) break;
+      TRACE(16384 + u * 16 + 5 + x * 3, leader);
+      tc_fence_after();
+      if (leader) {
+        const uint32_t plo = x ? p_lo1 : p_lo0;
+        const uint32_t vlo = v_lo0 + vs * (C::SLOT >> 4);
+        issue_pv_ss<C>(tmem + o_col[x], plo, vlo, hi, pv_cnt[x] > 0);
+        if constexpr (C::P2) issue_pv_ss<C>(tmem + o_col[x], plo + (C::P_TILE >> 4), vlo, hi, 1u);
+        tc_commit(smem_addr(&misc->pv_done[x]));
+      }
+      __syncwarp();
+      TRACE(16384 + u * 16 + 6 + x * 3, leader);
+      ++pv_cnt[x];
+    }
+    if (!ok) break;
+    if (leader) tc_commit(smem_addr(&misc->kv_empty[vs]));
+    __syncwarp();
+    u = nu;
+    vs = nvs;
+  }
+  if (leader) tc_commit(smem_addr(&misc->drain));
+  __syncwarp();
   w.drain(smem_addr(&misc->drain), 0);
 }
 
@@ -377,7 +544,8 @@ __device__ void attn_mma_role(const AttnParams& p, const TileInfo t0, const Tile
 // first S columns and release it to the MMA warp with one arrive per warp.
 template <class C>
 __device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, int b, int hkv, uint8_t* sQx,
-                                  AttnMisc* misc, uint32_t tmem, const CUtensorMap* tmO, const Waiter w) {
+                                  uint8_t* sPx, int n_turns, AttnMisc* misc, uint32_t tmem,
+                                  const CUtensorMap* tmO, const Waiter w) {
   using namespace ptx;
   constexpr uint32_t FULL = 0xffffffffu;
   const int warp = (threadIdx.x >> 5) & 3;  // TMEM lane quadrant of this warp
@@ -415,10 +583,10 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, 
   bool ok = true;
   for (int u = 0; u < t.n_kv; ++u) {
     if (!keep_tile(p, t, b, hkv, u)) continue;
-    TRACE(x * 8192 + it * 8 + 0, wg_tid == 0);
+    TRACE(x * 8192 + it * 16 + 0, wg_tid == 0);
     ok = __all_sync(FULL, w.wait(smem_addr(&misc->s_full[x]), it & 1));
     if (!ok) break;
-    TRACE(x * 8192 + it * 8 + 1, wg_tid == 0);
+    TRACE(x * 8192 + it * 16 + 1, wg_tid == 0);
     tc_fence_after();
 
     // Column factors: K scale per 32-key chunk (token-block K scales), times cq.
@@ -440,6 +608,12 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, 
     tmem_wait_ld();
 #pragma unroll
     for (int c = 0; c < 4; ++c) reg_fence(s[c]);
+    if constexpr (C::PSMEM) {  // S is in registers: the MMA warp may issue the next QK^T into this tile
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_addr(&misc->s_free[x]));
+    }
+    TRACE(x * 8192 + it * 16 + 2, wg_tid == 0);
     float f[4][32];
 #pragma unroll
     for (int c = 0; c < 4; ++c)
@@ -479,18 +653,36 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, 
       resc = true;
       m = m_new;
     }
-    if (__any_sync(FULL, resc)) {
+    // Lazy O correction (whole warp: tcgen05.ld/st are warp-wide). With P in
+    // TMEM the arrival of S proved the previous PV finished; with P in shared
+    // memory the previous PV may still run, so it is done after pv_done below.
+    auto rescale_o = [&]() {
+      if (__any_sync(FULL, resc)) {
 #pragma unroll 1
-      for (int c = 0; c < C::D / 32; ++c) {
-        uint32_t o[32];
-        tmem_ld32(tO + 32 * c, o);
-        tmem_wait_ld();
-        reg_fence(o);
+        for (int c = 0; c < C::D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(tO + 32 * c, o);
+          tmem_wait_ld();
+          reg_fence(o);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-        tmem_st32(tO + 32 * c, o);
+          for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
+          tmem_st32(tO + 32 * c, o);
+        }
       }
+    };
+    if constexpr (!C::PSMEM) rescale_o();
+    // Turn-taking on the exp2 unit: for the first n_turns tiles (both tiles
+    // walk the same KV tiles) the warpgroups alternate their exponential
+    // phases, so that one exponentiates while the other loads, reduces and
+    // packs. Tile 0 goes first.
+    TRACE(x * 8192 + it * 16 + 3, wg_tid == 0);
+    if (x == 0 ? (it >= 1 && it < n_turns) : (it < n_turns)) {
+      ok = __all_sync(FULL, w.wait(smem_addr(&misc->exp_done[x ^ 1]), (x == 0 ? it - 1 : it) & 1));
+      if (!ok) break;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) reg_fence(f[c]);
     }
+    TRACE(x * 8192 + it * 16 + 4, wg_tid == 0);
     const float mb = (m == -INFINITY ? 0.f : m) - log2g;
 #pragma unroll
     for (int c = 0; c < 4; ++c)
@@ -500,6 +692,13 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, 
     for (int c = 0; c < 4; ++c)
 #pragma unroll
       for (int j = 0; j < 32; ++j) f[c][j] = ex2(f[c][j]);
+    if (x == 0 ? (it < n_turns) : (it + 1 < n_turns)) {
+#pragma unroll
+      for (int c = 0; c < 4; ++c) reg_fence(f[c]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_addr(&misc->exp_done[x]));
+    }
+    TRACE(x * 8192 + it * 16 + 5, wg_tid == 0);
     float rs = 0.f;
     if constexpr (C::PV == PV_BF16) {
       uint32_t pk[2][32];
@@ -518,61 +717,94 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, 
       rs = (r0 + r1) + (r2 + r3);
       tmem_st32(tS, pk[0]);
       tmem_st32(tS + 32, pk[1]);
-    } else if constexpr (C::P2) {
-      // Two-term E4M3 P: hi = E4M3(p g), lo = E4M3(p g - hi) (the residual taken in
-      // f16), ~7 significant bits between them; both feed their own PV product.
-      // The row sum adds the unrounded values (the pair is as precise as BF16).
-      uint32_t pk[32], pl[32];
-      float r0 = 0.f, r1 = 0.f, r2 = 0.f, r3 = 0.f;
-#pragma unroll
-      for (int c = 0; c < 4; ++c)
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float* e = &f[c][4 * j];
-          const uint32_t h01 = pack_e4m3x2(e[0], e[1]), h23 = pack_e4m3x2(e[2], e[3]);
-          pk[c * 8 + j] = h01 | (h23 << 16);
-          const uint32_t d01 = hsub2(pack_f16x2(e[0], e[1]), e4m3x2_to_f16x2(h01));
-          const uint32_t d23 = hsub2(pack_f16x2(e[2], e[3]), e4m3x2_to_f16x2(h23));
-          pl[c * 8 + j] = f16x2_to_e4m3x2(d01) | (f16x2_to_e4m3x2(d23) << 16);
-          fadd2(r0, r1, r0, r1, e[0], e[1]);
-          fadd2(r2, r3, r2, r3, e[2], e[3]);
-        }
-      rs = (r0 + r1) + (r2 + r3);
-      tmem_st32(tS, pk);
-      tmem_st32(tS + 32, pl);
     } else {
       uint32_t pk[32];
-      float racc[4];
+      [[maybe_unused]] uint32_t pl[32];
+      if constexpr (C::P2) {
+        // Two-term E4M3 P: hi = E4M3(p g), lo = E4M3(p g - hi) (the residual taken
+        // in f16), ~7 significant bits between them; both feed their own PV
+        // product. The row sum adds the unrounded values (as precise as BF16 P).
+        float r0 = 0.f, r1 = 0.f, r2 = 0.f, r3 = 0.f;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t acc[2] = {0u, 0u};
+        for (int c = 0; c < 4; ++c)
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const uint32_t lo = pack_e4m3x2(f[c][4 * j], f[c][4 * j + 1]);
-          const uint32_t hi = pack_e4m3x2(f[c][4 * j + 2], f[c][4 * j + 3]);
-          pk[c * 8 + j] = lo | (hi << 16);
-          acc[j & 1] = hadd2(acc[j & 1], hadd2(e4m3x2_to_f16x2(lo), e4m3x2_to_f16x2(hi)));
+          for (int j = 0; j < 8; ++j) {
+            const float* e = &f[c][4 * j];
+            const uint32_t h01 = pack_e4m3x2(e[0], e[1]), h23 = pack_e4m3x2(e[2], e[3]);
+            pk[c * 8 + j] = h01 | (h23 << 16);
+            const uint32_t d01 = hsub2(pack_f16x2(e[0], e[1]), e4m3x2_to_f16x2(h01));
+            const uint32_t d23 = hsub2(pack_f16x2(e[2], e[3]), e4m3x2_to_f16x2(h23));
+            pl[c * 8 + j] = f16x2_to_e4m3x2(d01) | (f16x2_to_e4m3x2(d23) << 16);
+            fadd2(r0, r1, r0, r1, e[0], e[1]);
+            fadd2(r2, r3, r2, r3, e[2], e[3]);
+          }
+        rs = (r0 + r1) + (r2 + r3);
+      } else {
+        // The row sum adds the E4M3-rounded values actually stored, so the
+        // normalised weights sum to one and a dominant key returns its value.
+        float racc[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t acc[2] = {0u, 0u};
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const uint32_t lo = pack_e4m3x2(f[c][4 * j], f[c][4 * j + 1]);
+            const uint32_t hi = pack_e4m3x2(f[c][4 * j + 2], f[c][4 * j + 3]);
+            pk[c * 8 + j] = lo | (hi << 16);
+            acc[j & 1] = hadd2(acc[j & 1], hadd2(e4m3x2_to_f16x2(lo), e4m3x2_to_f16x2(hi)));
+          }
+          racc[c] = f16x2_sum(acc[0]) + f16x2_sum(acc[1]);
         }
-        racc[c] = f16x2_sum(acc[0]) + f16x2_sum(acc[1]);
+        rs = (racc[0] + racc[1]) + (racc[2] + racc[3]);
       }
-      rs = (racc[0] + racc[1]) + (racc[2] + racc[3]);
-      tmem_st32(tS, pk);
+      TRACE(x * 8192 + it * 16 + 6, wg_tid == 0);
+      if constexpr (C::PSMEM) {
+        // The previous PV must be done before P (single buffer) or O is rewritten.
+        if (it > 0) {
+          ok = __all_sync(FULL, w.wait(smem_addr(&misc->pv_done[x]), (it - 1) & 1));
+          if (!ok) break;
+          tc_fence_after();
+        }
+        TRACE(x * 8192 + it * 16 + 7, wg_tid == 0);
+        rescale_o();
+        // Row r of the 128 x 128-byte P tile, 16-byte chunks XOR-swizzled by r % 8
+        // (the 128-byte swizzle the PV descriptor expects).
+        const uint32_t prow = smem_addr(sPx) + r * 128;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+          const uint32_t addr = prow + ((k ^ (r & 7)) << 4);
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[4 * k]), "r"(pk[4 * k + 1]),
+                       "r"(pk[4 * k + 2]), "r"(pk[4 * k + 3])
+                       : "memory");
+          if constexpr (C::P2)
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr + C::P_TILE), "r"(pl[4 * k]),
+                         "r"(pl[4 * k + 1]), "r"(pl[4 * k + 2]), "r"(pl[4 * k + 3])
+                         : "memory");
+        }
+        fence_proxy_async_smem();  // generic-proxy P writes -> tensor-core reads
+      } else {
+        tmem_st32(tS, pk);
+        if constexpr (C::P2) tmem_st32(tS + 32, pl);
+      }
     }
     l = l * alpha + rs;
-    TRACE(x * 8192 + it * 8 + 4, wg_tid == 0);
+    TRACE(x * 8192 + it * 16 + 8, wg_tid == 0);
     tmem_wait_st();
     tc_fence_before();
     __syncwarp();  // the warp's P stores are ordered before lane 0's arrive
     if (lane == 0) mbar_arrive(smem_addr(&misc->p_full[x]));
-    TRACE(x * 8192 + it * 8 + 5, wg_tid == 0);
+    TRACE(x * 8192 + it * 16 + 9, wg_tid == 0);
     ++it;
   }
 
   // ---- epilogue ----
   bool have_o = false;
   if (ok) ok = __all_sync(FULL, w.wait(smem_addr(&misc->q_full), 0));  // Q buffer (our staging) has landed
-  if (ok && it > 0) {
-    ok = __all_sync(FULL, w.wait(smem_addr(&misc->o_full), 0));
+  if (ok && it > 0) {  // the last PV product has finished
+    if constexpr (C::PSMEM)
+      ok = __all_sync(FULL, w.wait(smem_addr(&misc->pv_done[x]), (it - 1) & 1));
+    else
+      ok = __all_sync(FULL, w.wait(smem_addr(&misc->o_full), 0));
     tc_fence_after();
     have_o = ok;
   }
@@ -638,7 +870,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* const sQ[2] = {smem, smem + C::Q_TILE};
-  uint8_t* sSlots = smem + 2 * C::Q_TILE;
+  uint8_t* const sP[2] = {smem + 2 * C::Q_TILE, smem + 2 * C::Q_TILE + C::P_BYTES / 2};  // E4M3 P (shared-memory P)
+  uint8_t* sSlots = smem + 2 * C::Q_TILE + C::P_BYTES;
   AttnMisc* misc = reinterpret_cast<AttnMisc*>(sSlots + C::STAGES * C::SLOT);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -689,6 +922,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     }
     mbar_init(smem_addr(&misc->o_full), 1);
     mbar_init(smem_addr(&misc->drain), 1);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(smem_addr(&misc->s_free[x]), 4);  // one arrive per softmax warp
+      mbar_init(smem_addr(&misc->pv_done[x]), 1);
+      mbar_init(smem_addr(&misc->exp_done[x]), 4);  // one arrive per softmax warp
+    }
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(smem_addr(&misc->kv_full[s]), 1);
       mbar_init(smem_addr(&misc->kv_empty[s]), 1);
@@ -698,11 +936,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   }
   if (C::PV == PV_E4M3 && p.sf_v_kind == FMHA_SF_PER_CHANNEL && threadIdx.x < C::D)
     misc->sf_v[threadIdx.x] = p.sf_v[(static_cast<int64_t>(b) * p.Hkv + hkv) * C::D + threadIdx.x];
-  if (warp == 8) {
+  if (warp == C::MMA_WARP) {
     tmem_alloc(smem_addr(&misc->tmem_base), C::TMEM_COLS);
     tmem_relinquish();
   }
-  if (warp == 9 && lane == 0) {
+  if (warp == C::LOAD_WARP && lane == 0) {
     prefetch_tmap(&tmQ);
     prefetch_tmap(&tmK);
     prefetch_tmap(&tmV);
@@ -714,17 +952,24 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   const uint32_t tmem = misc->tmem_base;
   const Waiter w{&misc->abort, p.err, p.wait_cycles};
 
-  if (warp < 8) {
+  if (warp >= C::SOFTMAX_WARP0 && warp < C::SOFTMAX_WARP0 + 8) {
     regs_inc<C::SOFTMAX_REGS>();
-    const int x = warp >> 2;
+    const int x = (warp - C::SOFTMAX_WARP0) >> 2;
     const TileInfo tx = x ? t[1] : t[0];  // select by value (no runtime-indexed array)
-    if (tx.valid) attn_softmax_role<C>(p, tx, x, b, hkv, x ? sQ[1] : sQ[0], misc, tmem, &tmO, w);
+    // Exp turn-taking needs both tiles to walk the same KV tiles (dense masks:
+    // prefixes [0, n_kv)); with a block mask the lists differ, so it is off.
+    int n_turns = 0;
+    if (C::TURNS && p.mask == nullptr) n_turns = min(t[0].n_kv, t[1].n_kv);
+    if (tx.valid)
+      attn_softmax_role<C>(p, tx, x, b, hkv, x ? sQ[1] : sQ[0], x ? sP[1] : sP[0], n_turns, misc, tmem, &tmO, w);
   } else {
     regs_dec<C::CONTROL_REGS>();
-    if (warp == 8) {
-      if (lane == 0) attn_mma_role<C>(p, t[0], t[1], b, hkv, sQ[0], sQ[1], sSlots, misc, tmem, w);
-      __syncwarp();
-    } else if (warp == 9) {
+    if (warp == C::MMA_WARP) {  // the whole warp; one elected lane issues
+      if constexpr (C::PSMEM)
+        attn_mma_role_psmem<C>(p, t[0], t[1], b, hkv, sQ[0], sQ[1], sP[0], sP[1], sSlots, misc, tmem, w);
+      else
+        attn_mma_role<C>(p, t[0], t[1], b, hkv, sQ[0], sQ[1], sSlots, misc, tmem, w);
+    } else if (warp == C::LOAD_WARP) {
       if (lane == 0) attn_load_role<C>(p, t[0], t[1], b, hkv, sQ[0], sQ[1], sSlots, misc, &tmQ, &tmK, &tmV, w);
       __syncwarp();
     }
@@ -732,7 +977,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 8) {
+  if (warp == C::MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }

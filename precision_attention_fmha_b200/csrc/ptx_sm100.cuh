@@ -118,6 +118,14 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
   asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
 }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+// One lane of a converged warp (the lowest active one) gets true.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\telect.sync _|p, 0xffffffff;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 // Arrive (once) on `bar` when every tcgen05 async op this thread issued so far completes.
 __device__ __forceinline__ void tc_commit(uint32_t bar) {
@@ -162,6 +170,17 @@ __device__ __forceinline__ void tc_commit(uint32_t bar) {
         "tcgen05.mma.cta_group::1.kind::" KIND " [%0], [%1], bd, %4, p;\n\t}" ::"r"(d),                    \
         "r"(a_tmem), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(acc));                                           \
   }
+#define FMHA_DEF_MMA_SS_LEAN_ACC(NAME, KIND)                                                               \
+  __device__ __forceinline__ void NAME(uint32_t d, uint32_t a_lo, uint32_t a_hi, uint32_t b_lo, uint32_t b_hi, \
+                                       uint32_t idesc, uint32_t acc) {                                     \
+    asm volatile(                                                                                          \
+        "{\n\t.reg .b64 ad, bd;\n\t.reg .pred p;\n\tmov.b64 ad, {%1, %2};\n\tmov.b64 bd, {%3, %4};\n\t"    \
+        "setp.ne.b32 p, %6, 0;\n\t"                                                                        \
+        "tcgen05.mma.cta_group::1.kind::" KIND " [%0], ad, bd, %5, p;\n\t}" ::"r"(d),                       \
+        "r"(a_lo), "r"(a_hi), "r"(b_lo), "r"(b_hi), "r"(idesc), "r"(acc));                                   \
+  }
+FMHA_DEF_MMA_SS_LEAN_ACC(mma_ss_f8_lean_acc, "f8f6f4")
+#undef FMHA_DEF_MMA_SS_LEAN_ACC
 FMHA_DEF_MMA_SS_LEAN(mma_ss_f16_lean, "f16")
 FMHA_DEF_MMA_SS_LEAN(mma_ss_f8_lean, "f8f6f4")
 FMHA_DEF_MMA_SS_LEAN(mma_ss_i8_lean, "i8")
@@ -227,6 +246,13 @@ __device__ __forceinline__ void reg_fence(uint32_t (&r)[32]) {
   for (int i = 0; i < 32; i += 8)
     asm volatile("" : "+r"(r[i]), "+r"(r[i + 1]), "+r"(r[i + 2]), "+r"(r[i + 3]), "+r"(r[i + 4]), "+r"(r[i + 5]),
                  "+r"(r[i + 6]), "+r"(r[i + 7]));
+}
+
+__device__ __forceinline__ void reg_fence(float (&r)[32]) {
+#pragma unroll
+  for (int i = 0; i < 32; i += 8)
+    asm volatile("" : "+f"(r[i]), "+f"(r[i + 1]), "+f"(r[i + 2]), "+f"(r[i + 3]), "+f"(r[i + 4]), "+f"(r[i + 5]),
+                 "+f"(r[i + 6]), "+f"(r[i + 7]));
 }
 
 // ------------------------------------------------------------ arithmetic ----

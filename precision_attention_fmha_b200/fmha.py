@@ -25,6 +25,7 @@ BF16, FP16, FP32, E4M3, INT8 = 0, 1, 2, 3, 4
 SF_KINDS = {None: 0, "none": 0, "per_tensor": 1, "per_head": 2, "per_token_block": 3, "per_channel": 4}
 STATUS = {0: "FMHA_OK", 1: "FMHA_ERR_INVALID_ARG", 2: "FMHA_ERR_UNSUPPORTED", 3: "FMHA_ERR_CUDA",
           4: "FMHA_ERR_TIMEOUT", 5: "FMHA_ERR_DEVICE_INDEX"}
+FMHA_OK, FMHA_ERR_INVALID_ARG, FMHA_ERR_UNSUPPORTED, FMHA_ERR_CUDA, FMHA_ERR_TIMEOUT, FMHA_ERR_DEVICE_INDEX = range(6)
 
 Scale = namedtuple("Scale", ["tensor", "kind", "rows_per_block"], defaults=[0])
 

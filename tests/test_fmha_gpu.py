@@ -221,3 +221,25 @@ def test_two_term_p_needs_8bit_v():
     with pytest.raises(fmha.FmhaError) as e:
         fmha.fmha_fwd(q.to(DEV), k.to(DEV), v.to(DEV), p_terms=2)
     assert e.value.status == 1
+
+
+def test_wait_limit_reports_timeout_and_context_survives():
+    """A one-cycle wait limit makes the first device wait that does not succeed
+    at once give up: the kernel records a timeout, lets its issued copies and
+    MMAs finish, frees TMEM and returns. The host sees FMHA_ERR_TIMEOUT and the
+    next launch, with the default limit, is correct."""
+    q, k, v = (t.to(DEV) for t in workloads.normal_qkv(21, 1, 4096, 4096, 8, 8, 128))
+    fmha.set_wait_timeout_cycles(1)
+    try:
+        fmha.fmha_fwd(q, k, v)
+        with pytest.raises(fmha.FmhaError) as e:
+            fmha.get_device_error()
+        assert e.value.status == fmha.FMHA_ERR_TIMEOUT
+    finally:
+        fmha.set_wait_timeout_cycles(0)
+    fmha.get_device_error()  # the error word was cleared by the read above
+    qs, ks, vs = workloads.normal_qkv(22, 1, 300, 300, 2, 2, 128)
+    o = fmha.fmha_fwd(qs.to(DEV), ks.to(DEV), vs.to(DEV))
+    fmha.get_device_error()
+    ref, _ = oa.attention(f64(qs), f64(ks), f64(vs), 1 / math.sqrt(128))
+    assert_close_bf16(f64(o), ref)
