@@ -333,8 +333,15 @@ def run_ours(args):
 
 
 # DRAM bytes (read + write) of one attention launch from an ncu capture of the
-# same kernel build, per workload (None until captured for the current kernel).
-TRAFFIC = {}
+# same kernel build, per workload (None until captured for the current kernel):
+#   ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum
+#       --clock-control none -k regex:attn_fwd -s 1 -c 1
+#       python bench.py [--workload W] --steps 1 --warmup 1 --no-cpu-baseline
+# (one pass; summary in profiles/attn_fwd_pv8_dram_traffic.md).
+TRAFFIC = {
+    "dense_pv8_s32768": 851.57e6 + 316.87e6,  # compulsory: Q,K 335.5 MB + V 167.8 MB read, O 335.5 MB written
+    "dense_pv8_s16384": 420.08e6 + 147.29e6,
+}
 
 
 # ------------------------------------------------------------- reference ----

@@ -150,9 +150,20 @@ struct Waiter {
       if (*abort_flag) return false;
       if (static_cast<uint64_t>(clock64() - t0) > budget) {
         *abort_flag = 1u;
-        atomicOr(err, kErrTimeout);
+        record_timeout(bar, parity);
         return false;
       }
+    }
+  }
+  // Sets the timeout bit and, for the first timeout only, the site bits.
+  __device__ __forceinline__ void record_timeout(uint32_t bar, uint32_t parity) const {
+    const uint32_t site = ((bar & 0xfffu) | ((parity & 1u) << 12) | (((threadIdx.x >> 5) + 1u) << 16))
+                          << kErrSiteShift;
+    uint32_t old = atomicOr(err, kErrTimeout);
+    for (int tries = 0; tries < 8 && (old >> kErrSiteShift) == 0u; ++tries) {
+      const uint32_t seen = atomicCAS(err, old | kErrTimeout, old | kErrTimeout | site);
+      if (seen == (old | kErrTimeout)) break;
+      old = seen;
     }
   }
   // Teardown wait: ignores the abort flag (used to drain in-flight async work).
@@ -164,7 +175,7 @@ struct Waiter {
     const long long t0 = clock64();
     while (!ptx::mbar_try_wait(bar, parity)) {
       if (static_cast<uint64_t>(clock64() - t0) > limit) {
-        atomicOr(err, kErrTimeout);
+        record_timeout(bar, parity);
         return false;
       }
     }

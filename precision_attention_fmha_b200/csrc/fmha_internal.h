@@ -12,6 +12,10 @@ namespace fmha {
 
 // Device error word bits (one word per device, see api.cu).
 enum : uint32_t { kErrTimeout = 1u, kErrPageIndex = 2u };
+// Bits 8..31 of the device error word: where the first wait that ran out was
+// (set once): bits 8..19 = barrier address & 0xfff (shared-memory offset of the
+// mbarrier), bit 20 = awaited parity, bits 24..28 = warp index + 1.
+constexpr uint32_t kErrSiteShift = 8u;
 
 // Default bound on one device-side wait (GPU clock cycles, ~1 s at 2 GHz).
 constexpr uint64_t kDefaultWaitCycles = 2000000000ull;
