@@ -44,6 +44,8 @@ WORKLOADS = {
     "all_fp8_s8192_causal": ("fp8", 2, 32, 32, 8192, 128, True),
     "sage_s16384": ("sage", 1, 24, 24, 16384, 128, False),
     "sparse_paged_s16384": ("sparse_paged", 4, 64, 8, 16384, 128, False),
+    # decode step: one query token per sequence against S cached tokens (S is Skv)
+    "decode_paged_s16384": ("decode_paged", 4, 64, 8, 16384, 128, False),
 }
 DEFAULT_WORKLOAD = "dense_pv8_s32768"
 
@@ -181,8 +183,9 @@ class Work:
             self.dtype = "int8,e4m3"
             self.quant = [("q", torch.int8, "per_token_block", 128), ("k", torch.int8, "per_token_block", 64),
                           ("v", E4, "per_channel", None)]
-        elif kind == "sparse_paged":
-            w = workloads.sparse_paged(S=S, B=B, Hq=Hq, Hkv=Hkv, D=D)
+        elif kind in ("sparse_paged", "decode_paged"):
+            gen = workloads.sparse_paged if kind == "sparse_paged" else workloads.decode_paged
+            w = gen(S=S, B=B, Hq=Hq, Hkv=Hkv, D=D)
             self.host = {"q": w["q"], "k_pool": w["k_pool"], "v_pool": w["v_pool"], "page_table": w["page_table"],
                          "mask": w["mask"]}
             self.peak, self.peak_note, self.dtype = bf16_peak, "bf16 burst", "bf16"
@@ -190,12 +193,25 @@ class Work:
         self.scale = 1.0 / math.sqrt(D)
         self.host = {n: t.contiguous().pin_memory() for n, t in self.host.items()}
         self.dev_in = {n: t.to(dev) for n, t in self.host.items()}
-        self.o = torch.empty((B, S, Hq, D), dtype=torch.bfloat16, device=dev)
+        self.Sq = self.host["q"].shape[1]
+        self.o = torch.empty((B, self.Sq, Hq, D), dtype=torch.bfloat16, device=dev)
         # density = kept score elements / (Sq * Skv)
+        self.ws = None
         if kind == "sparse_paged":
             kept = float(self.host["mask"].to(torch.float64).sum())
             self.density = kept * 128 * 128 / (B * Hkv * S * S)
             self.flop = 4.0 * B * Hq * S * S * D * self.density
+        elif kind == "decode_paged":  # every query row sees the kept 128-key blocks of its KV head
+            kept = float(self.host["mask"].to(torch.float64).sum())
+            self.density = kept * 128 / (B * Hkv * S)
+            self.flop = 4.0 * B * Hq * self.Sq * S * D * self.density
+            # HBM roofline: the kept K/V bytes (each read once), Q, O, page table and mask
+            self.hbm_bytes = (kept * 128 * D * 2 * 2 + 2 * B * self.Sq * Hq * D * 2
+                              + self.host["page_table"].numel() * 4 + self.host["mask"].numel())
+            self.q_dev = self.dev_in["q"]
+            nbytes = fmha.decode_workspace_bytes(self.q_dev, self.dev_in["k_pool"], S)
+            self.ws = torch.empty(max(16, nbytes), dtype=torch.uint8, device=dev)
+            self.n_parts = fmha.decode_num_parts(self.q_dev, self.dev_in["k_pool"], S)
         else:
             self.density = (S + 1) / (2 * S) if causal else 1.0
             self.flop = 4.0 * B * Hq * S * S * D * self.density
@@ -211,7 +227,10 @@ class Work:
         if kind == "sage":  # per-row-block P scale: P stored as 16 p
             self.sf_p = Scale(torch.full((B, Hq, math.ceil(S / 128)), 1.0 / 16, device=dev), "per_token_block", 128)
         # our kernels per step: token-block quantization is 1 launch, the grid-wide kinds 2, attention 1
+        # (decode: + the split merge when there are several partials)
         self.launches = 1 + sum(1 if g == "per_token_block" else 2 for _, _, g, _ in self.quant)
+        if kind == "decode_paged" and self.n_parts > 1:
+            self.launches += 1
 
     def prep(self, inp):
         for name, (out, sc, ws, gran, rpb, dt) in self.qbuf.items():
@@ -223,6 +242,10 @@ class Work:
             f.fmha_fwd_paged(inp["q"], inp["k_pool"], inp["v_pool"], inp["page_table"], self.S, mask=inp["mask"],
                              out=self.o, softmax_scale=self.scale)
             return
+        if self.kind == "decode_paged":
+            f.fmha_fwd_decode(inp["q"], inp["k_pool"], inp["v_pool"], page_table=inp["page_table"], Skv=self.S,
+                              mask=inp["mask"], workspace=self.ws, out=self.o, softmax_scale=self.scale)
+            return
         ops = {n: inp[n] for n in ("q", "k", "v")}
         sfs = {}
         for name, (out, sc, ws, gran, rpb, dt) in self.qbuf.items():
@@ -233,12 +256,25 @@ class Work:
 
     def config(self, world):
         c = {"workload": self.kind if self.kind != "pv8" else "dense_pv8", "B": self.B, "Hq": self.Hq,
-             "Hkv": self.Hkv, "Sq": self.S, "Skv": self.S, "D": self.D, "causal": self.causal,
+             "Hkv": self.Hkv, "Sq": self.Sq, "Skv": self.S, "D": self.D, "causal": self.causal,
              "density": round(self.density, 6),
              "quantized_in_step": [f"{n}:{g}" for n, _, g, _ in self.quant], "p_terms": self.p_terms,
              "l2": "inputs larger than L2" if self.host["q"].numel() * 2 > 126 * 2**20 else "inputs fit in L2",
              "parallelism": f"replicas{world}"}
         return c
+
+
+def roofline(W, args, attn_ms, achieved_tflops):
+    if W.kind == "decode_paged":  # HBM-bound: algorithmic bytes per launch over the measured copy bandwidth
+        _, hbm, src = load_peaks()
+        gbs = W.hbm_bytes / (attn_ms * 1e-3) / 1e9
+        return {"bound": "hbm", "achieved": round(gbs, 1), "peak": round(hbm, 1), "unit": "GB/s",
+                "frac": round(gbs / hbm, 4), "traffic": TRAFFIC.get(args.workload),
+                "peak_note": f"{src}: HBM copy bandwidth", "algorithmic_bytes": int(W.hbm_bytes),
+                "kernel": "attn_fwd_kernel (packed, split-KV) + split_merge_kernel", "kernel_ms": round(attn_ms, 4)}
+    return {"bound": "tensor", "achieved": round(achieved_tflops, 2), "peak": round(W.peak, 1), "unit": "TFLOP/s",
+            "frac": round(achieved_tflops / W.peak, 4), "traffic": TRAFFIC.get(args.workload),
+            "peak_note": f"{W.peak_src}: {W.peak_note}", "kernel": "attn_fwd_kernel", "kernel_ms": round(attn_ms, 4)}
 
 
 # ------------------------------------------------------------------ ours ----
@@ -312,10 +348,7 @@ def run_ours(args):
         "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": W.dtype, "data": "synthetic (seeded, BF16 inputs)",
         "config": W.config(world),
-        "roofline": {"bound": "tensor", "achieved": round(achieved, 2), "peak": round(W.peak, 1), "unit": "TFLOP/s",
-                     "frac": round(achieved / W.peak, 4), "traffic": TRAFFIC.get(args.workload),
-                     "peak_note": f"{W.peak_src}: {W.peak_note}", "kernel": "attn_fwd_kernel",
-                     "kernel_ms": round(attn_ms, 4)},
+        "roofline": roofline(W, args, attn_ms, achieved),
         "e2e": {"value": round(world * W.flop / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
                 "h2d_bytes_per_step": bytes_in, "d2h_bytes_per_step": W.o.numel() * W.o.element_size(),
                 "steps": Ke},
@@ -353,6 +386,18 @@ def oracle_sample(host, kind, B, Hq, Hkv, S, D, causal, rows):
     from oracle import quant as oq
 
     t = time.perf_counter()
+    if kind == "decode_paged":  # every batch, KV head 0 and its query heads, all (one) query rows
+        G = Hq // Hkv
+        pt = host["page_table"].numpy()
+        k = oa.gather_paged(host["k_pool"][:, :, :1].to(torch.float64).numpy(), pt, S)
+        v = oa.gather_paged(host["v_pool"][:, :, :1].to(torch.float64).numpy(), pt, S)
+        q = host["q"][:, :, :G].to(torch.float64).numpy()
+        mask = host["mask"][:, :1].numpy()
+        t = time.perf_counter() - t
+        t0 = time.perf_counter()
+        oa.attention(q, k, v, 1.0 / math.sqrt(D), False, mask)
+        dt = time.perf_counter() - t0 + t
+        return dt, 4.0 * q.shape[0] * q.shape[1] * G * float(mask.sum()) / q.shape[0] * 128 * D
     if kind == "sparse_paged":
         pt = host["page_table"].numpy()[:1]
         k = oa.gather_paged(host["k_pool"][:, :, :1].to(torch.float64).numpy(), pt, S)
@@ -410,7 +455,8 @@ def run_reference(args):
            "pv8": lambda: workloads.dense_pv8(S=S, B=B, H=Hq, D=D),
            "fp8": lambda: workloads.all_fp8(S=S, B=B, H=Hq, D=D),
            "sage": lambda: workloads.sage(S=S, B=B, H=Hq, D=D),
-           "sparse_paged": lambda: workloads.sparse_paged(S=S, B=B, Hq=Hq, Hkv=Hkv, D=D)}[kind]
+           "sparse_paged": lambda: workloads.sparse_paged(S=S, B=B, Hq=Hq, Hkv=Hkv, D=D),
+           "decode_paged": lambda: workloads.decode_paged(S=S, B=B, Hq=Hq, Hkv=Hkv, D=D)}[kind]
     host = gen()
     rows = 256
     for _ in range(args.warmup):

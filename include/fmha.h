@@ -205,6 +205,45 @@ fmha_status fmha_fwd_paged(const fmha_args* args, const int32_t* page_table, int
                            int32_t page_size, int32_t max_pages_per_seq, const uint8_t* mask,
                            int64_t mask_stride_b, int64_t mask_stride_h, struct CUstream_st* stream);
 
+/* Decode-shaped attention: few query tokens per sequence (Sq = 1 .. a few
+ * dozen), GQA-packed query tiles and split-KV ("FlashInfer block-sparse
+ * attention with PrimTS", section 1: the query tile is the query block times
+ * the query heads per KV head).
+ *   Computes exactly what fmha_fwd / fmha_fwd_paged compute (same args, same
+ *   causal alignment, same optional block mask), but puts the query heads of
+ *   one KV head into one 128-row tile (row = token * G + head in group,
+ *   G = Hq / Hkv, a power of two <= 128) so every K/V tile is read once per
+ *   KV head, and splits the KV range across CTAs.
+ *   page_table: NULL = contiguous K/V [B, Skv, Hkv, D]; otherwise the paged
+ *     pool as in fmha_fwd_paged (num_pages, page_size, max_pages_per_seq).
+ *   num_splits: KV splits per (b, KV head, query-tile pair); <= 0 chooses
+ *     about one CTA per SM. The count used is fmha_decode_num_splits().
+ *   Split j takes the kept KV tiles (after causality and the block mask) of
+ *     ranks [j*per, (j+1)*per), per = ceil(kept / splits). When all Sq * G
+ *     rows fit one 128-row tile, the CTA's two query tiles take alternate
+ *     kept tiles of the split, each as its own partial.
+ *   workspace: device memory owned by the caller, 16-byte aligned, at least
+ *     fmha_decode_workspace_bytes(args, num_splits) bytes (0 when there is a
+ *     single partial: then workspace may be NULL). With several partials each
+ *     writes O/l in fp32 and its log-sum-exp there, and a second kernel merges
+ *     them: lse = log sum_j exp(lse_j), O = sum_j exp(lse_j - lse) O_j.
+ *   Supported: D = 128, Skv <= 131072; Q/K/V BF16/BF16/BF16, BF16/BF16/E4M3
+ *   or E4M3/E4M3/E4M3 with the scale kinds of fmha_fwd; p_terms 0 or 1.
+ *   Errors: FMHA_ERR_UNSUPPORTED for other shapes/dtypes, FMHA_ERR_INVALID_ARG
+ *   for a missing or short workspace; device errors as in fmha_fwd_paged.   */
+fmha_status fmha_fwd_decode(const fmha_args* args, const int32_t* page_table, int32_t num_pages,
+                            int32_t page_size, int32_t max_pages_per_seq, const uint8_t* mask,
+                            int64_t mask_stride_b, int64_t mask_stride_h, int32_t num_splits, void* workspace,
+                            size_t workspace_bytes, struct CUstream_st* stream);
+
+/* Workspace bytes fmha_fwd_decode needs for these args and num_splits
+ * (0: a single split, or invalid sizes). Host only.                         */
+size_t fmha_decode_workspace_bytes(const fmha_args* args, int32_t num_splits);
+
+/* Number of KV splits fmha_fwd_decode uses for these args and num_splits
+ * (0 for invalid sizes). Host only; queries the current device's SM count. */
+int32_t fmha_decode_num_splits(const fmha_args* args, int32_t num_splits);
+
 /* Synchronises `stream`, then returns and clears the current device's error
  * word: FMHA_OK, FMHA_ERR_TIMEOUT or FMHA_ERR_DEVICE_INDEX (or FMHA_ERR_CUDA if
  * the synchronisation itself failed). */

@@ -13,6 +13,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstdarg>
@@ -107,33 +108,40 @@ EncodeTiledFn encode_fn(cudaError_t* err) {
   return fn;
 }
 
-// 4-D map (dims innermost first) with 128-byte swizzle. Strides in bytes for dims 1..3.
-// Size-1 dims get a packed stride so the descriptor stays valid whatever the caller's stride.
-fmha_status make_map(CUtensorMap* map, void* base, int elem_bytes, const uint64_t (&dims)[4],
-                     const int64_t (&strides_elems)[3], const uint32_t (&box)[4], const char* what) {
+// RANK-d map (dims innermost first, RANK = 4 or 5) with 128-byte swizzle.
+// Strides in elements for dims 1..RANK-1. Size-1 dims get a packed stride so
+// the descriptor stays valid whatever the caller's stride.
+template <int RANK>
+fmha_status make_map_n(CUtensorMap* map, void* base, int elem_bytes, const uint64_t (&dims)[RANK],
+                       const int64_t (&strides_elems)[RANK - 1], const uint32_t (&box)[RANK], const char* what) {
   cudaError_t e;
   EncodeTiledFn fn = encode_fn(&e);
   if (fn == nullptr) return fail(FMHA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable: %s", cudaGetErrorString(e));
-  cuuint64_t gdim[4];
-  cuuint64_t gstride[3];
-  cuuint32_t ebox[4] = {1, 1, 1, 1};
-  cuuint32_t bdim[4];
+  cuuint64_t gdim[RANK];
+  cuuint64_t gstride[RANK - 1];
+  cuuint32_t ebox[RANK];
+  cuuint32_t bdim[RANK];
   uint64_t packed = dims[0] * elem_bytes;
-  for (int i = 0; i < 4; ++i) {
+  for (int i = 0; i < RANK; ++i) {
     gdim[i] = dims[i];
     bdim[i] = box[i];
+    ebox[i] = 1;
   }
-  for (int i = 0; i < 3; ++i) {
+  for (int i = 0; i < RANK - 1; ++i) {
     uint64_t s = static_cast<uint64_t>(strides_elems[i]) * elem_bytes;
     if (dims[i + 1] == 1) s = (packed + 15) / 16 * 16;
     gstride[i] = s;
     packed = s * dims[i + 1];
   }
   const CUtensorMapDataType dt = elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
-  CUresult r = fn(map, dt, 4, base, gdim, gstride, bdim, ebox, CU_TENSOR_MAP_INTERLEAVE_NONE,
+  CUresult r = fn(map, dt, RANK, base, gdim, gstride, bdim, ebox, CU_TENSOR_MAP_INTERLEAVE_NONE,
                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(FMHA_ERR_INVALID_ARG, "TMA descriptor for %s rejected (CUresult %d)", what, (int)r);
   return FMHA_OK;
+}
+fmha_status make_map(CUtensorMap* map, void* base, int elem_bytes, const uint64_t (&dims)[4],
+                     const int64_t (&strides_elems)[3], const uint32_t (&box)[4], const char* what) {
+  return make_map_n<4>(map, base, elem_bytes, dims, strides_elems, box, what);
 }
 
 int elem_bytes(int dt) {
@@ -203,8 +211,52 @@ struct PagedArgs {
   int32_t num_pages, page_size, max_pages_per_seq;
 };
 
+struct DecodeArgs {
+  int32_t num_splits;  // <= 0: chosen here
+  void* workspace;
+  size_t workspace_bytes;
+};
+
+int sm_count() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) return 148;
+  return n;
+}
+
+// Split plan of the decode path: KV tiles per split and the split count
+// (no trailing empty split). Automatic: about one CTA per SM, at least two KV
+// tiles per split.
+struct SplitPlan {
+  int n_units, n_splits, split_tiles, interleave, n_parts;
+  size_t workspace_bytes;
+};
+SplitPlan plan_splits(int B, int Hq, int Hkv, int Sq, int Skv, int D, int requested) {
+  SplitPlan sp;
+  const int group = Hq / Hkv;
+  const int units = ceil_div(Sq * group, 128);
+  // All rows in one 128-row tile: the CTA's second query tile takes the same
+  // rows and alternate KV tiles (its own partial), so both softmax
+  // warpgroups work.
+  sp.interleave = units == 1 ? 1 : 0;
+  sp.n_units = sp.interleave ? 1 : ceil_div(units, 2);
+  const int n_kv = ceil_div(Skv, 128);
+  int splits = requested;
+  if (splits <= 0) {
+    const long long base = static_cast<long long>(B) * Hkv * sp.n_units;
+    splits = static_cast<int>(std::max<long long>(1, sm_count() / std::max<long long>(1, base)));
+    splits = std::min(splits, std::max(1, n_kv / 2));
+  }
+  splits = std::max(1, std::min(splits, std::max(1, n_kv)));
+  sp.split_tiles = std::max(1, ceil_div(n_kv, splits));
+  sp.n_splits = std::max(1, ceil_div(n_kv, sp.split_tiles));
+  sp.n_parts = sp.n_splits * (sp.interleave ? 2 : 1);
+  sp.workspace_bytes = sp.n_parts > 1 ? static_cast<size_t>(sp.n_parts) * B * Sq * Hq * (size_t(D) + 1) * 4 + 16 : 0;
+  return sp;
+}
+
 fmha_status run_attention(const fmha_args* a, const uint8_t* mask, int64_t msb, int64_t msh, const PagedArgs* pg,
-                          cudaStream_t stream) {
+                          cudaStream_t stream, const DecodeArgs* dec = nullptr) {
   if (a == nullptr) return fail(FMHA_ERR_INVALID_ARG, "args is NULL");
   const int B = a->B, Hq = a->Hq, Hkv = a->Hkv, Sq = a->Sq, Skv = a->Skv, D = a->D;
   if (B < 0 || Hq < 0 || Hkv < 0 || Sq < 0 || Skv < 0) return fail(FMHA_ERR_INVALID_ARG, "negative size");
@@ -226,6 +278,18 @@ fmha_status run_attention(const fmha_args* a, const uint8_t* mask, int64_t msb, 
   if (!tuple_ok || dout != FMHA_BF16)
     return fail(FMHA_ERR_UNSUPPORTED, "dtype tuple (q %d, k %d, v %d, o %d) unsupported", dq, dk, dv, dout);
   if (D == 64 && !(qk == QK_BF16 && pv == PV_BF16)) return fail(FMHA_ERR_UNSUPPORTED, "D=64 needs BF16 Q/K/V");
+  const bool packed = dec != nullptr;
+  const int group = Hq / Hkv;
+  int group_shift = 0;
+  if (packed) {
+    while ((1 << group_shift) < group) ++group_shift;
+    if ((1 << group_shift) != group || group > 128)
+      return fail(FMHA_ERR_UNSUPPORTED, "decode: Hq / Hkv = %d must be a power of two <= 128", group);
+    if (D != 128) return fail(FMHA_ERR_UNSUPPORTED, "decode: head dim %d (supported: 128)", D);
+    if (qk == QK_INT8) return fail(FMHA_ERR_UNSUPPORTED, "decode: INT8 Q/K not supported");
+    if (a->p_terms == 2) return fail(FMHA_ERR_UNSUPPORTED, "decode: p_terms = 2 not supported");
+    if (ceil_div(Skv, 128) > 1024) return fail(FMHA_ERR_UNSUPPORTED, "decode: Skv %d > 131072", Skv);
+  }
 
   // scale factors
   fmha_status st;
@@ -264,7 +328,15 @@ fmha_status run_attention(const fmha_args* a, const uint8_t* mask, int64_t msb, 
   // TMA descriptors
   const int eqk = qk == QK_BF16 ? 2 : 1, ev = pv == PV_BF16 ? 2 : 1;
   CUtensorMap tq, tk, tv, to;
-  {
+  if (packed) {  // (d, head in group, kv head, token, batch); box = all heads of a group x 128 / group tokens
+    const uint64_t dims[5] = {uint64_t(D), uint64_t(group), uint64_t(Hkv), uint64_t(Sq), uint64_t(B)};
+    const int64_t qstr[4] = {a->q.stride_h, a->q.stride_h * group, a->q.stride_s, a->q.stride_b};
+    const uint32_t box[5] = {uint32_t(128 / eqk), uint32_t(group), 1, uint32_t(128 / group), 1};
+    if ((st = make_map_n<5>(&tq, a->q.ptr, eqk, dims, qstr, box, "q")) != FMHA_OK) return st;
+    const int64_t ostr[4] = {a->o.stride_h, a->o.stride_h * group, a->o.stride_s, a->o.stride_b};
+    const uint32_t obox[5] = {64, uint32_t(group), 1, uint32_t(128 / group), 1};
+    if ((st = make_map_n<5>(&to, a->o.ptr, 2, dims, ostr, obox, "o")) != FMHA_OK) return st;
+  } else {
     const uint64_t dims[4] = {uint64_t(D), uint64_t(Hq), uint64_t(Sq), uint64_t(B)};
     const int64_t strides[3] = {a->q.stride_h, a->q.stride_s, a->q.stride_b};
     const uint32_t box[4] = {uint32_t(128 / eqk), 1, 128, 1};
@@ -325,6 +397,44 @@ fmha_status run_attention(const fmha_args* a, const uint8_t* mask, int64_t msb, 
   const uint64_t wc = g_wait_cycles.load();
   p.wait_cycles = wc ? wc : kDefaultWaitCycles;
 
+  if (packed) {
+    const SplitPlan sp = plan_splits(B, Hq, Hkv, Sq, Skv, D, dec->num_splits);
+    p.packed = 1;
+    p.group_shift = group_shift;
+    p.n_rows = Sq * group;
+    p.n_units = sp.n_units;
+    p.n_splits = sp.n_splits;
+    p.split_tiles = sp.split_tiles;
+    p.kv_interleave = sp.interleave;
+    p.n_parts = sp.n_parts;
+    if (sp.n_parts > 1) {
+      if (dec->workspace == nullptr || !aligned16(dec->workspace))
+        return fail(FMHA_ERR_INVALID_ARG, "decode: workspace is NULL or not 16-byte aligned (%d partials)",
+                    sp.n_parts);
+      if (dec->workspace_bytes < sp.workspace_bytes)
+        return fail(FMHA_ERR_INVALID_ARG, "decode: workspace of %zu bytes < %zu needed", dec->workspace_bytes,
+                    sp.workspace_bytes);
+      p.o_part = static_cast<float*>(dec->workspace);
+      const size_t o_elems = static_cast<size_t>(sp.n_parts) * B * Sq * Hq * D;
+      p.lse_part = p.o_part + o_elems;
+    }
+    if (static_cast<long long>(p.n_units) * p.n_splits * Hkv * B >= (1ll << 31))
+      return fail(FMHA_ERR_UNSUPPORTED, "grid too large");
+    e = launch_attention_packed(qk, pv, paged, p, tq, tk, tv, to, stream);
+    if (e != cudaSuccess) return fail(FMHA_ERR_CUDA, "decode attention launch: %s", cudaGetErrorString(e));
+    if (sp.n_parts > 1) {
+      MergeParams mp;
+      mp.o_part = p.o_part;
+      mp.lse_part = p.lse_part;
+      mp.o = static_cast<uint16_t*>(a->o.ptr);
+      mp.o_sb = a->o.stride_b; mp.o_ss = a->o.stride_s; mp.o_sh = a->o.stride_h;
+      mp.lse = a->lse;
+      mp.n_splits = sp.n_parts; mp.B = B; mp.Sq = Sq; mp.Hq = Hq; mp.D = D;
+      e = launch_split_merge(mp, stream);
+      if (e != cudaSuccess) return fail(FMHA_ERR_CUDA, "split merge launch: %s", cudaGetErrorString(e));
+    }
+    return ok_status();
+  }
   const long long head_units = p.pair_mode == PAIR_ROWS ? Hq : Hq / 2;
   if (static_cast<long long>(p.n_units) * head_units * B >= (1ll << 31))
     return fail(FMHA_ERR_UNSUPPORTED, "grid too large");
@@ -437,6 +547,30 @@ fmha_status fmha_fwd_paged(const fmha_args* args, const int32_t* page_table, int
                            int64_t mask_stride_h, cudaStream_t stream) {
   const PagedArgs pg{page_table, num_pages, page_size, max_pages_per_seq};
   return run_attention(args, mask, mask_stride_b, mask_stride_h, &pg, stream);
+}
+
+size_t fmha_decode_workspace_bytes(const fmha_args* args, int32_t num_splits) {
+  if (args == nullptr || args->B <= 0 || args->Hq <= 0 || args->Hkv <= 0 || args->Sq <= 0 || args->Skv < 0 ||
+      args->Hq % args->Hkv != 0)
+    return 0;
+  return plan_splits(args->B, args->Hq, args->Hkv, args->Sq, args->Skv, args->D, num_splits).workspace_bytes;
+}
+
+int32_t fmha_decode_num_splits(const fmha_args* args, int32_t num_splits) {
+  if (args == nullptr || args->B <= 0 || args->Hq <= 0 || args->Hkv <= 0 || args->Sq <= 0 || args->Skv < 0 ||
+      args->Hq % args->Hkv != 0)
+    return 0;
+  return plan_splits(args->B, args->Hq, args->Hkv, args->Sq, args->Skv, args->D, num_splits).n_splits;
+}
+
+fmha_status fmha_fwd_decode(const fmha_args* args, const int32_t* page_table, int32_t num_pages, int32_t page_size,
+                            int32_t max_pages_per_seq, const uint8_t* mask, int64_t mask_stride_b,
+                            int64_t mask_stride_h, int32_t num_splits, void* workspace, size_t workspace_bytes,
+                            cudaStream_t stream) {
+  const DecodeArgs dec{num_splits, workspace, workspace_bytes};
+  if (page_table == nullptr) return run_attention(args, mask, mask_stride_b, mask_stride_h, nullptr, stream, &dec);
+  const PagedArgs pg{page_table, num_pages, page_size, max_pages_per_seq};
+  return run_attention(args, mask, mask_stride_b, mask_stride_h, &pg, stream, &dec);
 }
 
 fmha_status fmha_get_device_error(cudaStream_t stream) {

@@ -55,10 +55,12 @@ static __device__ unsigned long long g_fmha_trace[FMHA_TRACE_SLOTS];  // one per
 
 namespace fmha {
 
-template <int D_, int QK_, int PV_, bool PAGED_, bool P2_ = false>
+template <int D_, int QK_, int PV_, bool PAGED_, bool P2_ = false, bool PACKED_ = false>
 struct AttnCfg {
   static constexpr int D = D_, QK = QK_, PV = PV_;
   static constexpr bool PAGED = PAGED_;
+  // GQA-packed query tiles and split-KV ranges (decode shapes).
+  static constexpr bool PACKED = PACKED_;
   static constexpr bool P2 = P2_;  // E4M3 P split into two terms (hi + lo), each with its own PV product
   static_assert(!P2 || PV == PV_E4M3, "two-term P needs an E4M3 V");
   static constexpr int BM = 128, BN = 128;
@@ -109,7 +111,7 @@ struct AttnCfg {
   // come first: the issue scheduler favours older warps, and the MMA warp's
   // short serial steps sit on the critical path of both softmax pipelines.
   static constexpr int MMA_WARP = 0, LOAD_WARP = 1, SOFTMAX_WARP0 = 4;
-  static constexpr uint32_t SOFTMAX_REGS = 224, CONTROL_REGS = 56;
+  static constexpr uint32_t SOFTMAX_REGS = 216, CONTROL_REGS = 72;
   static_assert(2 * 128 * SOFTMAX_REGS + 128 * CONTROL_REGS <= THREADS * 168, "register split exceeds launch");
 };
 
@@ -127,13 +129,24 @@ struct alignas(8) AttnMisc {
   uint32_t tmem_base;
   volatile uint32_t abort;
   float sf_v[128];
+  // Packed (decode) CTAs: the KV tiles each query tile processes, as a bit set
+  // over KV tiles (at most 1024), and its [first, last + 1) range.
+  uint32_t keep_bits[2][32];
+  int32_t range[2][2];
 };
 
+static_assert(sizeof(AttnMisc) <= 1024, "AttnMisc must fit the 1 KB misc area");
+
 struct TileInfo {
-  int h;      // query head
-  int q0;     // first query row
-  int qblk;   // 128-row query block index
-  int n_kv;   // KV tiles [0, n_kv) not excluded by causality / length
+  int h;      // query head (packed: first head of the KV head's group)
+  int q0;     // first row (packed: first packed row, = token * group + head in group)
+  int qblk;   // 128-row block index
+  int tok0;   // first query token
+  int mrow;   // block-mask row (128-token query block)
+  int u0;     // KV tiles [u0, n_kv) not excluded by causality, length or split
+  int n_kv;
+  int x;      // query tile slot in the CTA (0 or 1)
+  int part;   // packed, several partials: index of this tile's partial output
   bool valid;
 };
 
@@ -186,10 +199,14 @@ struct Waiter {
 // Tile info and waiters are passed by value everywhere: a runtime-indexed
 // array or a by-reference argument would live in local memory, and with the
 // shared-memory carve-out near its maximum every such load goes to L2.
-__device__ __forceinline__ bool keep_tile(const AttnParams& p, const TileInfo t, int b, int hkv, int u) {
+template <class C>
+__device__ __forceinline__ bool keep_tile(const AttnParams& p, const TileInfo t, int b, int hkv, int u,
+                                          const AttnMisc* misc) {
+  if constexpr (C::PACKED)  // the split's tiles were chosen up front (mask, split, query-tile share)
+    return u >= t.u0 && u < t.n_kv && ((misc->keep_bits[t.x][u >> 5] >> (u & 31)) & 1u);
   if (u >= t.n_kv) return false;
   if (p.mask == nullptr) return true;
-  return p.mask[b * p.mask_sb + hkv * p.mask_sh + static_cast<int64_t>(t.qblk) * p.n_kv_blocks + u] != 0;
+  return p.mask[b * p.mask_sb + hkv * p.mask_sh + static_cast<int64_t>(t.mrow) * p.n_kv_blocks + u] != 0;
 }
 
 __device__ __forceinline__ float sf_lookup(const float* sf, int kind, int64_t bh, int nblk, int idx_in_seq,
@@ -219,21 +236,64 @@ __device__ void attn_load_role(const AttnParams& p, const TileInfo t0, const Til
   for (int x = 0; x < 2; ++x) {
     if (!t[x].valid) continue;
 #pragma unroll
-    for (int c = 0; c < C::QK_CHUNKS; ++c)
-      tma_load_4d(smem_addr(sQ[x]) + c * C::CHUNK_BYTES, tmQ, q_full, c * C::QK_CHUNK_ELEMS, t[x].h, t[x].q0, b);
+    for (int c = 0; c < C::QK_CHUNKS; ++c) {
+      if constexpr (C::PACKED)  // box: all heads of the group x 128 / group tokens
+        tma_load_5d(smem_addr(sQ[x]) + c * C::CHUNK_BYTES, tmQ, q_full, c * C::QK_CHUNK_ELEMS, 0, hkv, t[x].tok0,
+                    b);
+      else
+        tma_load_4d(smem_addr(sQ[x]) + c * C::CHUNK_BYTES, tmQ, q_full, c * C::QK_CHUNK_ELEMS, t[x].h, t[x].q0, b);
+    }
   }
   const uint64_t pol = policy_evict_last();  // K/V tiles are re-read by every CTA of this head
   uint32_t issued = 0u, issued_phase = 0u;  // per slot: a load was issued / parity of its last phase
   int slot_it = 0;
   const int n_u = max(t0.n_kv, t1.n_kv);
   bool ok = true;
-  for (int u = 0; u < n_u && ok; ++u) {
-    if (!keep_tile(p, t0, b, hkv, u) && !keep_tile(p, t1, b, hkv, u)) continue;
+  auto next_kept = [&](int from) {
+    int v = from;
+    while (v < n_u && !keep_tile<C>(p, t0, b, hkv, v, misc) && !keep_tile<C>(p, t1, b, hkv, v, misc)) ++v;
+    return v;
+  };
+  // Paged K/V: the page-table entries of a KV tile (BN / page_size <= 8 pages)
+  // are read once for its K and V copies, and one kept tile ahead, so that
+  // their latency overlaps the wait for a free slot.
+  constexpr int kMaxPages = C::PAGED ? C::BN / 16 : 1;
+  const int per = C::PAGED ? C::BN / p.page_size : 1;
+  auto lookup = [&](int v, int (&pg)[kMaxPages]) {
+#pragma unroll
+    for (int pp = 0; pp < kMaxPages; ++pp) {
+      const int lp = v * per + pp;  // logical page of this sequence
+      pg[pp] = (pp < per && lp * p.page_size < p.Skv)
+                   ? __ldg(p.page_table + static_cast<int64_t>(b) * p.max_pages_per_seq + lp)
+                   : -1;
+    }
+  };
+  // One kept tile: K and V copies with the page entries in `cur`, while the
+  // next kept tile's entries are read into `nxt`. Two alternating buffers (the
+  // loop below runs this twice per round) keep the prefetched values out of any
+  // register copy, which would wait for the loads.
+  auto step = [&](int& u, int (&cur)[kMaxPages], int (&nxt)[kMaxPages]) {
+    const int nu = next_kept(u + 1);
+    if constexpr (C::PAGED) {
+      if (nu < n_u) lookup(nu, nxt);
+#pragma unroll
+      for (int pp = 0; pp < kMaxPages; ++pp) {  // out of range: TMA reads zeros there; reported
+        const int lp = u * per + pp;
+        if (pp < per && lp * p.page_size < p.Skv && (cur[pp] < 0 || cur[pp] >= p.num_pages)) {
+          atomicOr(p.err, kErrPageIndex);
+          cur[pp] = p.num_pages;
+        } else if (cur[pp] < 0) {
+          cur[pp] = p.num_pages;
+        }
+      }
+    }
     for (int kv = 0; kv < 2; ++kv) {  // K then V
       const int s = slot_it % C::STAGES;
       const uint32_t ph = (slot_it / C::STAGES) & 1;
       ++slot_it;
+      TRACE(32768 + u * 8 + kv * 4 + 0, true);
       if (!w.wait(smem_addr(&misc->kv_empty[s]), ph ^ 1)) { ok = false; break; }
+      TRACE(32768 + u * 8 + kv * 4 + 1, true);
       const uint32_t full = smem_addr(&misc->kv_full[s]);
       const int chunks = kv == 0 ? C::QK_CHUNKS : C::V_CHUNKS;
       const int chunk_elems = kv == 0 ? C::QK_CHUNK_ELEMS : C::V_CHUNK_ELEMS;
@@ -246,23 +306,26 @@ __device__ void attn_load_role(const AttnParams& p, const TileInfo t0, const Til
         for (int c = 0; c < chunks; ++c)
           tma_load_4d_hint(dst + c * C::CHUNK_BYTES, tm, full, c * chunk_elems, hkv, u * C::BN, b, pol);
       } else {
-        const int per = C::BN / p.page_size;
-        for (int pp = 0; pp < per; ++pp) {
-          const int lp = (u * C::BN) / p.page_size + pp;  // logical page of this sequence
-          int page = p.num_pages;                          // out of range: TMA fills zeros
-          if (lp * p.page_size < p.Skv) {
-            const int e = p.page_table[static_cast<int64_t>(b) * p.max_pages_per_seq + lp];
-            if (e >= 0 && e < p.num_pages)
-              page = e;
-            else
-              atomicOr(p.err, kErrPageIndex);
-          }
+#pragma unroll
+        for (int pp = 0; pp < kMaxPages; ++pp) {
+          if (pp >= per) break;
           for (int c = 0; c < chunks; ++c)
             tma_load_4d_hint(dst + c * C::CHUNK_BYTES + pp * p.page_size * 128, tm, full, c * chunk_elems, hkv, 0,
-                             page, pol);
+                             cur[pp], pol);
         }
       }
     }
+    u = nu;
+  };
+  int u = next_kept(min(t0.u0, t1.u0));
+  int pg_a[kMaxPages], pg_b[kMaxPages];
+  if constexpr (C::PAGED) {
+    if (u < n_u) lookup(u, pg_a);
+  }
+  while (u < n_u && ok) {
+    step(u, pg_a, pg_b);
+    if (u >= n_u || !ok) break;
+    step(u, pg_b, pg_a);
   }
   // Every issued copy lands before shared memory goes away. Without an abort
   // the consumers have already seen these phases complete (no waiting); after
@@ -345,8 +408,8 @@ __device__ void attn_mma_role(const AttnParams& p, const TileInfo t0, const Tile
   const int n_u = max(t0.n_kv, t1.n_kv);
   bool ok = __all_sync(FULL, w.wait(smem_addr(&misc->q_full), 0));
   tc_fence_after();
-  for (int u = 0; u < n_u && ok; ++u) {
-    const bool kx[2] = {keep_tile(p, t0, b, hkv, u), keep_tile(p, t1, b, hkv, u)};
+  for (int u = min(t0.u0, t1.u0); u < n_u && ok; ++u) {
+    const bool kx[2] = {keep_tile<C>(p, t0, b, hkv, u, misc), keep_tile<C>(p, t1, b, hkv, u, misc)};
     if (!kx[0] && !kx[1]) continue;
     TRACE(16384 + u * 16 + 15, leader);
     const int ks = slot_it % C::STAGES;
@@ -356,36 +419,44 @@ __device__ void attn_mma_role(const AttnParams& p, const TileInfo t0, const Tile
     const uint32_t vph = (slot_it / C::STAGES) & 1;
     ++slot_it;
     bool k_ready = false;
+    // Pass 1, query tiles that keep u: their pending PV (S_x(u) overwrites P_x
+    // in TMEM), then S_x(u). Pass 2, tiles that skip u: their pending PV, after
+    // the S MMAs above, so a tile whose softmax is still running does not hold
+    // back the other tile's S.
 #pragma unroll
-    for (int x = 0; x < 2 && ok; ++x) {
-      if (pend[x] >= 0) {  // PV of the previous tile first: S_x(u) overwrites P_x
-        TRACE(16384 + u * 16 + x * 8 + 0, leader);
-        if (!(ok = __all_sync(FULL, w.wait(smem_addr(&misc->p_full[x]), pv_cnt[x] & 1)))) break;
-        TRACE(16384 + u * 16 + x * 8 + 1, leader);
-        tc_fence_after();
-        if (leader) {
-          issue_pv<C>(tmem + o_col[x], tmem + s_col[x], v_lo0 + pend[x] * (C::SLOT >> 4), hi, pv_cnt[x] > 0);
-          if constexpr (C::P2)  // the low E4M3 term of P
-            issue_pv<C>(tmem + o_col[x], tmem + s_col[x] + 32, v_lo0 + pend[x] * (C::SLOT >> 4), hi, 1u);
-        }
-        __syncwarp();
-        TRACE(16384 + u * 16 + x * 8 + 2, leader);
-        ++pv_cnt[x];
-        pend[x] = -1;
-      }
-      if (kx[x]) {
-        if (!k_ready) {
-          if (!(ok = __all_sync(FULL, w.wait(smem_addr(&misc->kv_full[ks]), kph)))) break;
+    for (int pass = 0; pass < 2; ++pass) {
+#pragma unroll
+      for (int x = 0; x < 2 && ok; ++x) {
+        if (kx[x] != (pass == 0)) continue;
+        if (pend[x] >= 0) {
+          TRACE(16384 + u * 16 + x * 8 + 0, leader);
+          if (!(ok = __all_sync(FULL, w.wait(smem_addr(&misc->p_full[x]), pv_cnt[x] & 1)))) break;
+          TRACE(16384 + u * 16 + x * 8 + 1, leader);
           tc_fence_after();
-          k_ready = true;
+          if (leader) {
+            issue_pv<C>(tmem + o_col[x], tmem + s_col[x], v_lo0 + pend[x] * (C::SLOT >> 4), hi, pv_cnt[x] > 0);
+            if constexpr (C::P2)  // the low E4M3 term of P
+              issue_pv<C>(tmem + o_col[x], tmem + s_col[x] + 32, v_lo0 + pend[x] * (C::SLOT >> 4), hi, 1u);
+          }
+          __syncwarp();
+          TRACE(16384 + u * 16 + x * 8 + 2, leader);
+          ++pv_cnt[x];
+          pend[x] = -1;
         }
-        TRACE(16384 + u * 16 + x * 8 + 3, leader);
-        if (leader) {
-          issue_qk<C>(tmem + s_col[x], x ? q_lo1 : q_lo0, k_lo0 + ks * (C::SLOT >> 4), hi);
-          tc_commit(smem_addr(&misc->s_full[x]));
+        if (kx[x]) {
+          if (!k_ready) {
+            if (!(ok = __all_sync(FULL, w.wait(smem_addr(&misc->kv_full[ks]), kph)))) break;
+            tc_fence_after();
+            k_ready = true;
+          }
+          TRACE(16384 + u * 16 + x * 8 + 3, leader);
+          if (leader) {
+            issue_qk<C>(tmem + s_col[x], x ? q_lo1 : q_lo0, k_lo0 + ks * (C::SLOT >> 4), hi);
+            tc_commit(smem_addr(&misc->s_full[x]));
+          }
+          __syncwarp();
+          TRACE(16384 + u * 16 + x * 8 + 5, leader);
         }
-        __syncwarp();
-        TRACE(16384 + u * 16 + x * 8 + 5, leader);
       }
     }
     if (!ok) break;
@@ -459,14 +530,14 @@ __device__ void attn_mma_role_psmem(const AttnParams& p, const TileInfo t0, cons
   tc_fence_after();
   auto next_kept = [&](int from) {
     int u = from;
-    while (u < n_u && !keep_tile(p, t0, b, hkv, u) && !keep_tile(p, t1, b, hkv, u)) ++u;
+    while (u < n_u && !keep_tile<C>(p, t0, b, hkv, u, misc) && !keep_tile<C>(p, t1, b, hkv, u, misc)) ++u;
     return u;
   };
   // Issues S_x(u) for every query tile keeping u; K_u lives in slot ks.
   auto issue_s = [&](int u, int ks) {
 #pragma unroll
     for (int x = 0; x < 2; ++x) {
-      if (!keep_tile(p, x ? t1 : t0, b, hkv, u)) continue;
+      if (!keep_tile<C>(p, x ? t1 : t0, b, hkv, u, misc)) continue;
       if (s_cnt[x] > 0) {  // the softmax must have loaded this tile's previous S
         if (!(ok = __all_sync(FULL, w.wait(smem_addr(&misc->s_free[x]), (s_cnt[x] - 1) & 1)))) return;
         tc_fence_after();
@@ -480,7 +551,7 @@ __device__ void attn_mma_role_psmem(const AttnParams& p, const TileInfo t0, cons
       ++s_cnt[x];
     }
   };
-  int u = next_kept(0);
+  int u = next_kept(min(t0.u0, t1.u0));
   int vs = 0;
   if (u < n_u && ok) {
     const int ks = slot_it % C::STAGES;
@@ -521,7 +592,7 @@ __device__ void attn_mma_role_psmem(const AttnParams& p, const TileInfo t0, cons
     tc_fence_after();
 #pragma unroll
     for (int x = 0; x < 2; ++x) {
-      if (!keep_tile(p, x ? t1 : t0, b, hkv, u)) continue;
+      if (!keep_tile<C>(p, x ? t1 : t0, b, hkv, u, misc)) continue;
       TRACE(16384 + u * 16 + 4 + x * 3, leader);
       if (!(ok = __all_sync(FULL, w.wait(smem_addr(&misc->p_full[x]), pv_cnt[x] & 1)))) break;
       TRACE(16384 + u * 16 + 5 + x * 3, leader);
@@ -562,12 +633,14 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, 
   const int warp = (threadIdx.x >> 5) & 3;  // TMEM lane quadrant of this warp
   const int lane = threadIdx.x & 31;
   const int r = warp * 32 + lane;  // row within the tile
-  const int row = t.q0 + r;        // query row
+  // Query token and head of this row (packed: row r = token r >> shift, head r & (group - 1)).
+  const int row = C::PACKED ? t.tok0 + (r >> p.group_shift) : t.q0 + r;
+  const int head = C::PACKED ? t.h + (r & ((1 << p.group_shift) - 1)) : t.h;
   const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
   const uint32_t tS = tmem + lane_off + (x ? 128u : 0u);
   const uint32_t tO = tmem + lane_off + (x ? 256u + C::D : 256u);
   const int wg_tid = threadIdx.x & 127;
-  const int64_t bhq = static_cast<int64_t>(b) * p.Hq + t.h;
+  const int64_t bhq = static_cast<int64_t>(b) * p.Hq + head;
   const int64_t bhk = static_cast<int64_t>(b) * p.Hkv + hkv;
 
   // Row factor: softmax scale * log2(e) * Q scale of this row.
@@ -583,7 +656,7 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, 
   if constexpr (C::PV == PV_E4M3) {
     float sfp = 1.f / 16.f;
     if (p.sf_p_kind == FMHA_SF_PER_TENSOR) sfp = p.sf_p[0];
-    if (p.sf_p_kind == FMHA_SF_PER_TOKEN_BLOCK) sfp = p.sf_p[bhq * p.sf_p_nblk + t.q0 / p.sf_p_rpb];
+    if (p.sf_p_kind == FMHA_SF_PER_TOKEN_BLOCK) sfp = p.sf_p[bhq * p.sf_p_nblk + t.tok0 / p.sf_p_rpb];
     log2g = -__log2f(sfp);
     tau = fminf(8.f, fmaxf(0.f, floorf(__log2f(448.f * sfp))));
   }
@@ -592,8 +665,8 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, 
   float l = 0.f;        // running row sum of the stored P (times g)
   int it = 0;
   bool ok = true;
-  for (int u = 0; u < t.n_kv; ++u) {
-    if (!keep_tile(p, t, b, hkv, u)) continue;
+  for (int u = t.u0; u < t.n_kv; ++u) {
+    if (!keep_tile<C>(p, t, b, hkv, u, misc)) continue;
     TRACE(x * 8192 + it * 16 + 0, wg_tid == 0);
     ok = __all_sync(FULL, w.wait(smem_addr(&misc->s_full[x]), it & 1));
     if (!ok) break;
@@ -833,6 +906,26 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, 
       reg_fence(o[0]);
       reg_fence(o[1]);
     }
+    if constexpr (C::PACKED) {
+      if (p.n_parts > 1) {  // one partial: O / l in fp32 for the merge kernel (no staging)
+        if (row < p.Sq && ok) {
+          float* dst = p.o_part + ((((int64_t)t.part * p.B + b) * p.Sq + row) * p.Hq + head) * C::D + 64 * c64;
+#pragma unroll
+          for (int j = 0; j < 64; j += 4) {
+            float v4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              v4[e] = have_o ? __uint_as_float(o[(j + e) >> 5][(j + e) & 31]) * inv_l : 0.f;
+              if (C::PV == PV_E4M3 && p.sf_v_kind == FMHA_SF_PER_CHANNEL) v4[e] *= misc->sf_v[64 * c64 + j + e];
+            }
+            asm volatile("st.global.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst + j), "f"(v4[0]), "f"(v4[1]),
+                         "f"(v4[2]), "f"(v4[3])
+                         : "memory");
+          }
+        }
+        continue;
+      }
+    }
     uint32_t pk[32];
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
@@ -860,12 +953,17 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, 
     fence_proxy_async_smem();
     named_bar_sync(1 + x, 128);
     if (wg_tid == 0 && ok) {
-      tma_store_4d(tmO, stage0 + buf * C::CHUNK_BYTES, 64 * c64, t.h, t.q0, b);
+      if constexpr (C::PACKED)
+        tma_store_5d(tmO, stage0 + buf * C::CHUNK_BYTES, 64 * c64, 0, hkv, t.tok0, b);
+      else
+        tma_store_4d(tmO, stage0 + buf * C::CHUNK_BYTES, 64 * c64, t.h, t.q0, b);
       bulk_commit();
     }
   }
-  if (p.lse != nullptr && row < p.Sq && ok) {
-    const float lse = l > 0.f ? (m + __log2f(l) - log2g) * 0.69314718055994531f : -INFINITY;
+  const float lse = l > 0.f ? (m + __log2f(l) - log2g) * 0.69314718055994531f : -INFINITY;
+  if (C::PACKED && p.n_parts > 1) {
+    if (row < p.Sq && ok) p.lse_part[(((int64_t)t.part * p.B + b) * p.Hq + head) * p.Sq + row] = lse;
+  } else if (p.lse != nullptr && row < p.Sq && ok) {
     p.lse[bhq * p.Sq + row] = lse;
   }
   if (wg_tid == 0) bulk_wait0();
@@ -889,7 +987,83 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   // ---- work item -> (b, heads, query rows) ----
   int b, hkv;
   TileInfo t[2];
-  {
+  if constexpr (C::PACKED) {
+    // (unit pair, split, kv head, batch); rows are Sq * group packed rows.
+    int item = blockIdx.x;
+    const int pr = item % p.n_units;
+    item /= p.n_units;
+    const int split = item % p.n_splits;
+    item /= p.n_splits;
+    hkv = item % p.Hkv;
+    b = item / p.Hkv;
+    const int toks = C::BM >> p.group_shift;  // query tokens per 128-row unit
+    for (int x = 0; x < 2; ++x) {
+      t[x].h = hkv * p.group;
+      t[x].qblk = p.kv_interleave ? 0 : 2 * pr + x;  // interleaved: both tiles hold all rows
+      t[x].q0 = t[x].qblk * C::BM;
+      t[x].tok0 = t[x].qblk * toks;
+      t[x].mrow = t[x].tok0 / C::BM;
+      t[x].valid = t[x].q0 < p.n_rows;
+      int n = p.n_kv_blocks;  // causal / length limit; the split's tiles are chosen below
+      if (p.causal) {
+        const int last = min(t[x].tok0 + toks - 1, p.Sq - 1) + (p.Skv - p.Sq);
+        n = last < 0 ? 0 : min(p.n_kv_blocks, last / C::BN + 1);
+      }
+      t[x].n_kv = t[x].valid ? n : 0;
+      t[x].u0 = 0;
+      t[x].x = x;
+      t[x].part = p.kv_interleave ? 2 * split + x : split;
+    }
+    // Warp 2 (idle) picks the split's kept KV tiles: rank r of the kept tiles
+    // in [0, n) goes to split r / per; interleaved tiles take alternate ranks.
+    if (warp == 2) {
+      for (int x = 0; x < 2; ++x) {
+        if (p.kv_interleave && x == 1) break;  // tile 1 shares tile 0's scan
+        const int n = t[x].n_kv;
+        const uint8_t* mrow = p.mask == nullptr ? nullptr
+                              : p.mask + b * p.mask_sb + hkv * p.mask_sh + static_cast<int64_t>(t[x].mrow) * p.n_kv_blocks;
+        int total = 0;
+        for (int base = 0; base < n; base += 32) {
+          const int u = base + lane;
+          const bool k = u < n && (mrow == nullptr || mrow[u] != 0);
+          total += __popc(__ballot_sync(0xffffffffu, k));
+        }
+        const int per = (total + p.n_splits - 1) / p.n_splits;
+        const int r0 = split * per, r1 = min(total, r0 + per);
+        int lo[2] = {1 << 30, 1 << 30}, hi[2] = {0, 0};
+        int cnt = 0;
+        for (int base = 0; base < 1024; base += 32) {
+          const int u = base + lane;
+          const bool k = u < n && (mrow == nullptr || mrow[u] != 0);
+          const uint32_t bal = __ballot_sync(0xffffffffu, k);
+          const int rank = cnt + __popc(bal & ((1u << lane) - 1u));
+          const bool mine = k && rank >= r0 && rank < r1;
+          const int dest = p.kv_interleave ? ((rank - r0) & 1) : x;
+          const uint32_t b0 = __ballot_sync(0xffffffffu, mine && dest == 0);
+          const uint32_t b1 = __ballot_sync(0xffffffffu, mine && dest == 1);
+          if (lane == 0) {
+            if (p.kv_interleave) {
+              misc->keep_bits[0][base >> 5] = b0;
+              misc->keep_bits[1][base >> 5] = b1;
+            } else {
+              misc->keep_bits[x][base >> 5] = x ? b1 : b0;
+            }
+          }
+          if (b0) { lo[0] = min(lo[0], base + __ffs(b0) - 1); hi[0] = base + 32 - __clz(b0); }
+          if (b1) { lo[1] = min(lo[1], base + __ffs(b1) - 1); hi[1] = base + 32 - __clz(b1); }
+          cnt += __popc(bal);
+        }
+        if (lane == 0) {
+          if (p.kv_interleave) {
+            for (int y = 0; y < 2; ++y) { misc->range[y][0] = lo[y]; misc->range[y][1] = hi[y]; }
+          } else {
+            misc->range[x][0] = lo[x];
+            misc->range[x][1] = hi[x];
+          }
+        }
+      }
+    }
+  } else {
     int item = blockIdx.x;
     if (p.pair_mode == PAIR_ROWS) {
       int pr = item % p.n_units;
@@ -915,6 +1089,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     hkv = t[0].h / p.group;
     for (int x = 0; x < 2; ++x) {
       t[x].q0 = t[x].qblk * C::BM;
+      t[x].tok0 = t[x].q0;
+      t[x].mrow = t[x].qblk;
+      t[x].u0 = 0;
+      t[x].x = x;
+      t[x].part = 0;
       t[x].valid = t[x].q0 < p.Sq;
       int n = p.n_kv_blocks;
       if (p.causal) {
@@ -962,6 +1141,17 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = misc->tmem_base;
   const Waiter w{&misc->abort, p.err, p.wait_cycles};
+  if constexpr (C::PACKED) {
+    for (int x = 0; x < 2; ++x) {
+      if (t[x].valid) {
+        t[x].u0 = misc->range[x][0];
+        t[x].n_kv = misc->range[x][1];
+      } else {
+        t[x].u0 = 1 << 30;
+        t[x].n_kv = 0;
+      }
+    }
+  }
 
   if (warp >= C::SOFTMAX_WARP0 && warp < C::SOFTMAX_WARP0 + 8) {
     regs_inc<C::SOFTMAX_REGS>();
@@ -970,7 +1160,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     // Exp turn-taking needs both tiles to walk the same KV tiles (dense masks:
     // prefixes [0, n_kv)); with a block mask the lists differ, so it is off.
     int n_turns = 0;
-    if (C::TURNS && p.mask == nullptr) n_turns = min(t[0].n_kv, t[1].n_kv);
+    if (C::TURNS && !C::PACKED && p.mask == nullptr) n_turns = min(t[0].n_kv, t[1].n_kv);
     if (tx.valid)
       attn_softmax_role<C>(p, tx, x, b, hkv, x ? sQ[1] : sQ[0], x ? sP[1] : sP[0], n_turns, misc, tmem, &tmO, w);
   } else {
@@ -1000,7 +1190,7 @@ cudaError_t launch_attention_t(const AttnParams& p, const CUtensorMap& tq, const
   auto kern = attn_fwd_kernel<C>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  const int head_units = p.pair_mode == PAIR_ROWS ? p.Hq : p.Hq / 2;
+  const int head_units = C::PACKED ? p.Hkv * p.n_splits : (p.pair_mode == PAIR_ROWS ? p.Hq : p.Hq / 2);
   const long long blocks = static_cast<long long>(p.n_units) * head_units * p.B;
   kern<<<static_cast<unsigned>(blocks), C::THREADS, C::SMEM_BYTES, stream>>>(p, tq, tk, tv, to);
   return cudaGetLastError();

@@ -49,6 +49,19 @@ struct AttnParams {
   // paged K/V (page_table == nullptr: contiguous)
   const int32_t* page_table; int32_t num_pages, page_size, max_pages_per_seq;
   int32_t p_terms;      // 1 or 2 E4M3 terms for P (E4M3 V only)
+  // GQA-packed query tiles (decode shapes): row r of a 128-row unit is query
+  // token r >> group_shift of head (hkv * group + (r & (group - 1))); n_units
+  // then counts pairs of 128-row units of the Sq * group packed rows.
+  int32_t packed, group_shift, n_rows;
+  // Split-KV (packed only): split j of a (b, kv head) takes the kept KV tiles
+  // of ranks [j * per, (j + 1) * per), per = ceil(kept / n_splits). With several
+  // partials each query tile writes O / l (fp32) and its lse to o_part / lse_part.
+  // kv_interleave: all packed rows fit one 128-row tile, so the CTA's two query
+  // tiles hold the same rows and take alternate kept KV tiles of the split;
+  // each is then its own partial (n_parts = 2 * n_splits), else n_parts = n_splits.
+  int32_t n_splits, split_tiles, kv_interleave, n_parts;
+  float* o_part;   // [n_parts, B, Sq, Hq, D] when n_parts > 1
+  float* lse_part; // [n_parts, B, Hq, Sq]
   uint32_t* err;        // device error word
   uint64_t wait_cycles; // bound on one wait
 };
@@ -67,6 +80,18 @@ cudaError_t launch_attention(int qk_kind, int pv_kind, int D, bool paged, const 
                              const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                              const CUtensorMap& to, cudaStream_t stream);
 cudaError_t launch_quantize(bool to_e4m3, const QuantParams& p, cudaStream_t stream);
+// Decode path: attention over GQA-packed tiles (p.packed = 1), then, for
+// n_splits > 1, the split merge into o (bf16, element strides) and lse.
+cudaError_t launch_attention_packed(int qk_kind, int pv_kind, bool paged, const AttnParams& p,
+                                    const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                                    const CUtensorMap& to, cudaStream_t stream);
+struct MergeParams {
+  const float* o_part; const float* lse_part;
+  uint16_t* o; int64_t o_sb, o_ss, o_sh;  // bf16 bits
+  float* lse;                             // nullable [B, Hq, Sq]
+  int32_t n_splits, B, Sq, Hq, D;
+};
+cudaError_t launch_split_merge(const MergeParams& m, cudaStream_t stream);
 
 // Size of the built-in scratch used by fmha_quantize_blockwise_noalloc, in
 // 32-bit words (one per scale group of the grid-wide granularities).

@@ -75,6 +75,11 @@ def load_library(path=None):
     lib.fmha_fwd_block_sparse.argtypes = [ctypes.POINTER(_Args), vp, i64, i64, vp]
     lib.fmha_fwd_paged.argtypes = [ctypes.POINTER(_Args), vp, i32, i32, i32, vp, i64, i64, vp]
     lib.fmha_get_device_error.argtypes = [vp]
+    lib.fmha_fwd_decode.argtypes = [ctypes.POINTER(_Args), vp, i32, i32, i32, vp, i64, i64, i32, vp, sz, vp]
+    lib.fmha_decode_workspace_bytes.argtypes = [ctypes.POINTER(_Args), i32]
+    lib.fmha_decode_workspace_bytes.restype = sz
+    lib.fmha_decode_num_splits.argtypes = [ctypes.POINTER(_Args), i32]
+    lib.fmha_decode_num_splits.restype = i32
     lib.fmha_status_string.argtypes = [ctypes.c_int]
     lib.fmha_status_string.restype = ctypes.c_char_p
     lib.fmha_last_error_message.restype = ctypes.c_char_p
@@ -229,6 +234,65 @@ def fmha_fwd_paged(q, k_pool, v_pool, page_table, Skv, mask=None, out=None, sf_q
     _check(lib.fmha_fwd_paged(ctypes.byref(a), page_table.data_ptr(), k_pool.shape[0], k_pool.shape[1],
                               page_table.shape[1], mptr, msb, msh, _stream(stream)))
     return out
+
+
+def fmha_fwd_decode(q, k, v, page_table=None, Skv=None, mask=None, num_splits=0, workspace=None, out=None,
+                    sf_q=None, sf_k=None, sf_v=None, sf_p=None, softmax_scale=None, causal=False, lse=None,
+                    stream=None):
+    """Decode-shaped attention (few query tokens, GQA-packed tiles, split-KV).
+
+    k / v: contiguous [B, Skv, Hkv, D], or page pools [num_pages, page_size, Hkv, D]
+    with page_table int32 [B, max_pages] and Skv. The workspace (uint8 CUDA tensor)
+    is allocated here when not given. Returns O (BF16 [B, Sq, Hq, D])."""
+    lib = load_library()
+    out = _out_like(q, out)
+    if page_table is not None:
+        if page_table.dtype != torch.int32 or page_table.dim() != 2 or not page_table.is_contiguous():
+            raise ValueError("page_table must be contiguous int32 [B, max_pages_per_seq]")
+        if Skv is None:
+            raise ValueError("Skv is required with a page table")
+    a = _args(q, k, v, out, sf_q, sf_k, sf_v, sf_p, softmax_scale, causal, lse, Skv=Skv)
+    mptr, msb, msh = None, 0, 0
+    if mask is not None:
+        msb, msh = _mask_strides(mask, q.shape[1], a.Skv)
+        mptr = mask.data_ptr()
+    need = lib.fmha_decode_workspace_bytes(ctypes.byref(a), int(num_splits))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    wptr, wbytes = (workspace.data_ptr(), workspace.numel() * workspace.element_size()) if workspace is not None \
+        else (None, 0)
+    if page_table is not None:
+        pt, npages, psize, maxp = page_table.data_ptr(), k.shape[0], k.shape[1], page_table.shape[1]
+    else:
+        pt, npages, psize, maxp = None, 0, 0, 0
+    _check(lib.fmha_fwd_decode(ctypes.byref(a), pt, npages, psize, maxp, mptr, msb, msh, int(num_splits), wptr,
+                               wbytes, _stream(stream)))
+    return out
+
+
+def decode_num_splits(q, k, Skv=None, num_splits=0):
+    """KV splits fmha_fwd_decode uses for these shapes (host only)."""
+    B, Sq, Hq, D = q.shape
+    a = _Args()
+    a.B, a.Hq, a.Hkv, a.Sq, a.Skv, a.D = B, Hq, k.shape[2], Sq, k.shape[1] if Skv is None else Skv, D
+    return load_library().fmha_decode_num_splits(ctypes.byref(a), int(num_splits))
+
+
+def decode_workspace_bytes(q, k, Skv=None, num_splits=0):
+    """Workspace bytes fmha_fwd_decode needs for these shapes (host only)."""
+    B, Sq, Hq, D = q.shape
+    a = _Args()
+    a.B, a.Hq, a.Hkv, a.Sq, a.Skv, a.D = B, Hq, k.shape[2], Sq, k.shape[1] if Skv is None else Skv, D
+    return load_library().fmha_decode_workspace_bytes(ctypes.byref(a), int(num_splits))
+
+
+def decode_num_parts(q, k, Skv=None, num_splits=0):
+    """Partial outputs fmha_fwd_decode merges (1: no merge launch)."""
+    need = decode_workspace_bytes(q, k, Skv, num_splits)
+    if need == 0:
+        return 1
+    B, Sq, Hq, D = q.shape
+    return (need - 16) // (B * Sq * Hq * (D + 1) * 4)
 
 
 def get_device_error(stream=None):

@@ -129,3 +129,25 @@ def sparse_paged(S=16384, B=4, Hq=64, Hkv=8, D=128, page_size=64, density=0.25):
     mask = block_mask(seed + 2, B, Hkv, S, S, density)
     return dict(q=q, k=k, v=v, k_pool=kp, v_pool=vp, page_table=pt, mask=mask,
                 page_size=page_size, scale=1.0 / math.sqrt(D))
+
+
+def decode_mask(seed, B, Hkv, Sq, Skv, density=0.25, block=128):
+    """Block mask for decode shapes: Bernoulli(density) over KV blocks, the last
+    KV block (the newest tokens) always kept."""
+    rng = np.random.default_rng(seed)
+    nq, nk = -(-Sq // block), -(-Skv // block)
+    m = (rng.random(size=(B, Hkv, nq, nk)) < density).astype(np.uint8)
+    m[:, :, :, nk - 1] = 1
+    return torch.from_numpy(m)
+
+
+def decode_paged(S=16384, B=4, Hq=64, Hkv=8, D=128, Sq=1, page_size=64, density=0.25):
+    """Decode step over a block-sparse paged cache: Sq query tokens per sequence
+    against S cached tokens (GQA Hq/Hkv), pages in a seeded permutation."""
+    seed = SEED_BASE + 6 + S
+    q, _, _ = normal_qkv(seed, B, Sq, 1, Hq, Hkv, D)
+    _, k, v = normal_qkv(seed + 1, B, 1, S, Hq, Hkv, D)
+    kp, vp, pt = paged_pool(seed + 2, k, v, page_size)
+    mask = decode_mask(seed + 3, B, Hkv, Sq, S, density)
+    return dict(q=q, k=k, v=v, k_pool=kp, v_pool=vp, page_table=pt, mask=mask,
+                page_size=page_size, scale=1.0 / math.sqrt(D))
