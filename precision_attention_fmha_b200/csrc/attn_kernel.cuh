@@ -150,6 +150,9 @@ struct TileInfo {
   bool valid;
 };
 
+// Suspend-time hint of one barrier probe, in ns.
+constexpr uint32_t kWaitSleepNs = 1000;
+
 // Bounded mbarrier wait. Returns false on timeout (recorded) or CTA abort.
 struct Waiter {
   volatile uint32_t* abort_flag;
@@ -159,13 +162,17 @@ struct Waiter {
     if (ptx::mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (true) {
-      if (ptx::mbar_try_wait(bar, parity)) return true;
-      if (*abort_flag) return false;
+      // The limit is checked before every sleeping probe, so a limit shorter
+      // than one probe still gives up after the first unsatisfied probe.
       if (static_cast<uint64_t>(clock64() - t0) > budget) {
         *abort_flag = 1u;
         record_timeout(bar, parity);
         return false;
       }
+      // Sleep in the barrier (woken when the phase completes) rather than spin:
+      // a spinning warp takes issue slots from the warps sharing its scheduler.
+      if (ptx::mbar_try_wait_sleep(bar, parity, kWaitSleepNs)) return true;
+      if (*abort_flag) return false;
     }
   }
   // Sets the timeout bit and, for the first timeout only, the site bits.
@@ -221,22 +228,32 @@ __device__ __forceinline__ float sf_lookup(const float* sf, int kind, int64_t bh
 
 // ------------------------------------------------------------ TMA producer --
 template <class C>
+// TMA producer, run by the whole warp: the schedule (kept tiles, slots,
+// phases) is warp-uniform; lane 0 posts each slot's expected bytes, then the
+// copies of one tile (chunks x pages) are issued from different lanes at once,
+// and for paged K/V each lane reads the page-table entry of its page.
 __device__ void attn_load_role(const AttnParams& p, const TileInfo t0, const TileInfo t1, int b, int hkv,
                                uint8_t* sQ0, uint8_t* sQ1, uint8_t* sSlots, AttnMisc* misc, const CUtensorMap* tmQ,
                                const CUtensorMap* tmK, const CUtensorMap* tmV, const Waiter w) {
   using namespace ptx;
+  constexpr uint32_t FULL = 0xffffffffu;
+  const int lane = threadIdx.x & 31;
   const TileInfo t[2] = {t0, t1};  // indexed only with unrolled constants below
   uint8_t* const sQ[2] = {sQ0, sQ1};
   const uint32_t q_full = smem_addr(&misc->q_full);
-  uint32_t qbytes = 0;
+  if (lane == 0) {
+    uint32_t qbytes = 0;
 #pragma unroll
-  for (int x = 0; x < 2; ++x) qbytes += t[x].valid ? C::Q_TILE : 0;
-  mbar_arrive_expect_tx(q_full, qbytes);
+    for (int x = 0; x < 2; ++x) qbytes += t[x].valid ? C::Q_TILE : 0;
+    mbar_arrive_expect_tx(q_full, qbytes);
+  }
+  __syncwarp();
 #pragma unroll
   for (int x = 0; x < 2; ++x) {
     if (!t[x].valid) continue;
 #pragma unroll
     for (int c = 0; c < C::QK_CHUNKS; ++c) {
+      if (lane != x * C::QK_CHUNKS + c) continue;
       if constexpr (C::PACKED)  // box: all heads of the group x 128 / group tokens
         tma_load_5d(smem_addr(sQ[x]) + c * C::CHUNK_BYTES, tmQ, q_full, c * C::QK_CHUNK_ELEMS, 0, hkv, t[x].tok0,
                     b);
@@ -249,80 +266,78 @@ __device__ void attn_load_role(const AttnParams& p, const TileInfo t0, const Til
   int slot_it = 0;
   const int n_u = max(t0.n_kv, t1.n_kv);
   bool ok = true;
+  // Next KV tile at or after `from` that either query tile keeps.
   auto next_kept = [&](int from) {
-    int v = from;
-    while (v < n_u && !keep_tile<C>(p, t0, b, hkv, v, misc) && !keep_tile<C>(p, t1, b, hkv, v, misc)) ++v;
-    return v;
-  };
-  // Paged K/V: the page-table entries of a KV tile (BN / page_size <= 8 pages)
-  // are read once for its K and V copies, and one kept tile ahead, so that
-  // their latency overlaps the wait for a free slot.
-  constexpr int kMaxPages = C::PAGED ? C::BN / 16 : 1;
-  const int per = C::PAGED ? C::BN / p.page_size : 1;
-  auto lookup = [&](int v, int (&pg)[kMaxPages]) {
-#pragma unroll
-    for (int pp = 0; pp < kMaxPages; ++pp) {
-      const int lp = v * per + pp;  // logical page of this sequence
-      pg[pp] = (pp < per && lp * p.page_size < p.Skv)
-                   ? __ldg(p.page_table + static_cast<int64_t>(b) * p.max_pages_per_seq + lp)
-                   : -1;
+    if constexpr (C::PACKED) {  // scan the keep-bit words (at most 32)
+      for (int wd = from >> 5; wd < 32 && (wd << 5) < n_u; ++wd) {
+        uint32_t bits = misc->keep_bits[0][wd] | misc->keep_bits[1][wd];
+        if (wd == (from >> 5)) bits &= ~0u << (from & 31);
+        if (bits) return min(n_u, (wd << 5) + __ffs(bits) - 1);
+      }
+      return n_u;
+    } else {
+      int v = from;
+      while (v < n_u && !keep_tile<C>(p, t0, b, hkv, v, misc) && !keep_tile<C>(p, t1, b, hkv, v, misc)) ++v;
+      return v;
     }
   };
-  // One kept tile: K and V copies with the page entries in `cur`, while the
-  // next kept tile's entries are read into `nxt`. Two alternating buffers (the
-  // loop below runs this twice per round) keep the prefetched values out of any
-  // register copy, which would wait for the loads.
-  auto step = [&](int& u, int (&cur)[kMaxPages], int (&nxt)[kMaxPages]) {
+  // Paged K/V: lane l reads the page-table entry of page l of a tile (BN /
+  // page_size <= 8 pages) once for its K and V copies, one kept tile ahead.
+  const int per = C::PAGED ? C::BN / p.page_size : 1;
+  auto lookup = [&](int v) {
+    int e = -1;
+    const int lp = v * per + lane;  // logical page of this sequence
+    if (C::PAGED && lane < per && lp * p.page_size < p.Skv)
+      e = __ldg(p.page_table + static_cast<int64_t>(b) * p.max_pages_per_seq + lp);
+    return e;
+  };
+  // One kept tile u: lane l issues copy l (page l / chunks, chunk l % chunks)
+  // of K, then of V, using the page entry read one tile earlier (`cur`).
+  auto step = [&](int& u, int& cur, int& nxt) {
     const int nu = next_kept(u + 1);
+    int page = 0;
     if constexpr (C::PAGED) {
-      if (nu < n_u) lookup(nu, nxt);
-#pragma unroll
-      for (int pp = 0; pp < kMaxPages; ++pp) {  // out of range: TMA reads zeros there; reported
-        const int lp = u * per + pp;
-        if (pp < per && lp * p.page_size < p.Skv && (cur[pp] < 0 || cur[pp] >= p.num_pages)) {
-          atomicOr(p.err, kErrPageIndex);
-          cur[pp] = p.num_pages;
-        } else if (cur[pp] < 0) {
-          cur[pp] = p.num_pages;
-        }
-      }
+      if (nu < n_u) nxt = lookup(nu);
+      const int lp = u * per + lane;
+      const bool in_seq = lane < per && lp * p.page_size < p.Skv;
+      if (in_seq && (cur < 0 || cur >= p.num_pages)) atomicOr(p.err, kErrPageIndex);
+      page = (in_seq && cur >= 0 && cur < p.num_pages) ? cur : p.num_pages;  // out of range: TMA reads zeros
     }
     for (int kv = 0; kv < 2; ++kv) {  // K then V
       const int s = slot_it % C::STAGES;
       const uint32_t ph = (slot_it / C::STAGES) & 1;
       ++slot_it;
-      TRACE(32768 + u * 8 + kv * 4 + 0, true);
-      if (!w.wait(smem_addr(&misc->kv_empty[s]), ph ^ 1)) { ok = false; break; }
-      TRACE(32768 + u * 8 + kv * 4 + 1, true);
+      TRACE(32768 + u * 8 + kv * 4 + 0, lane == 0);
+      if (!(ok = __all_sync(FULL, w.wait(smem_addr(&misc->kv_empty[s]), ph ^ 1)))) break;
+      TRACE(32768 + u * 8 + kv * 4 + 1, lane == 0);
       const uint32_t full = smem_addr(&misc->kv_full[s]);
       const int chunks = kv == 0 ? C::QK_CHUNKS : C::V_CHUNKS;
       const int chunk_elems = kv == 0 ? C::QK_CHUNK_ELEMS : C::V_CHUNK_ELEMS;
       const CUtensorMap* tm = kv == 0 ? tmK : tmV;
       const uint32_t dst = smem_addr(sSlots + s * C::SLOT);
-      mbar_arrive_expect_tx(full, kv == 0 ? C::K_TILE : C::V_TILE);
+      if (lane == 0) mbar_arrive_expect_tx(full, kv == 0 ? C::K_TILE : C::V_TILE);
+      __syncwarp();
       issued |= 1u << s;
       issued_phase = (issued_phase & ~(1u << s)) | (ph << s);
       if constexpr (!C::PAGED) {
-        for (int c = 0; c < chunks; ++c)
-          tma_load_4d_hint(dst + c * C::CHUNK_BYTES, tm, full, c * chunk_elems, hkv, u * C::BN, b, pol);
+        if (lane < chunks)
+          tma_load_4d_hint(dst + lane * C::CHUNK_BYTES, tm, full, lane * chunk_elems, hkv, u * C::BN, b, pol);
       } else {
-#pragma unroll
-        for (int pp = 0; pp < kMaxPages; ++pp) {
-          if (pp >= per) break;
-          for (int c = 0; c < chunks; ++c)
-            tma_load_4d_hint(dst + c * C::CHUNK_BYTES + pp * p.page_size * 128, tm, full, c * chunk_elems, hkv, 0,
-                             cur[pp], pol);
-        }
+        const int pp = lane / chunks, c = lane - pp * chunks;
+        const int pg = __shfl_sync(FULL, page, pp & 31);
+        if (pp < per)
+          tma_load_4d_hint(dst + c * C::CHUNK_BYTES + pp * p.page_size * 128, tm, full, c * chunk_elems, hkv, 0, pg,
+                           pol);
       }
     }
     u = nu;
   };
   int u = next_kept(min(t0.u0, t1.u0));
-  int pg_a[kMaxPages], pg_b[kMaxPages];
+  int pg_a = -1, pg_b = -1;
   if constexpr (C::PAGED) {
-    if (u < n_u) lookup(u, pg_a);
+    if (u < n_u) pg_a = lookup(u);
   }
-  while (u < n_u && ok) {
+  while (u < n_u && ok) {  // two alternating page registers: no copy waits for a pending lookup
     step(u, pg_a, pg_b);
     if (u >= n_u || !ok) break;
     step(u, pg_b, pg_a);
@@ -330,9 +345,12 @@ __device__ void attn_load_role(const AttnParams& p, const TileInfo t0, const Til
   // Every issued copy lands before shared memory goes away. Without an abort
   // the consumers have already seen these phases complete (no waiting); after
   // an abort, set by any role at any time, copies may still be in flight.
-  w.drain(q_full, 0);
-  for (int s = 0; s < C::STAGES; ++s)
-    if (issued & (1u << s)) w.drain(smem_addr(&misc->kv_full[s]), (issued_phase >> s) & 1u);
+  if (lane == 0) {
+    w.drain(q_full, 0);
+    for (int s = 0; s < C::STAGES; ++s)
+      if (issued & (1u << s)) w.drain(smem_addr(&misc->kv_full[s]), (issued_phase >> s) & 1u);
+  }
+  __syncwarp();
 }
 
 // ------------------------------------------------------- tensor-core issue --
@@ -1170,9 +1188,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         attn_mma_role_psmem<C>(p, t[0], t[1], b, hkv, sQ[0], sQ[1], sP[0], sP[1], sSlots, misc, tmem, w);
       else
         attn_mma_role<C>(p, t[0], t[1], b, hkv, sQ[0], sQ[1], sSlots, misc, tmem, w);
-    } else if (warp == C::LOAD_WARP) {
-      if (lane == 0) attn_load_role<C>(p, t[0], t[1], b, hkv, sQ[0], sQ[1], sSlots, misc, &tmQ, &tmK, &tmV, w);
-      __syncwarp();
+    } else if (warp == C::LOAD_WARP) {  // the whole warp
+      attn_load_role<C>(p, t[0], t[1], b, hkv, sQ[0], sQ[1], sSlots, misc, &tmQ, &tmK, &tmV, w);
     }
   }
 
