@@ -1035,6 +1035,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     // Warp 2 (idle) picks the split's kept KV tiles: rank r of the kept tiles
     // in [0, n) goes to split r / per; interleaved tiles take alternate ranks.
     if (warp == 2) {
+      // Words past the larger tile's limit are never read; those below it are
+      // all written (shared memory starts with stale contents).
+      const int n_words = (max(t[0].n_kv, t[1].n_kv) + 31) >> 5;
       for (int x = 0; x < 2; ++x) {
         if (p.kv_interleave && x == 1) break;  // tile 1 shares tile 0's scan
         const int n = t[x].n_kv;
@@ -1050,7 +1053,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         const int r0 = split * per, r1 = min(total, r0 + per);
         int lo[2] = {1 << 30, 1 << 30}, hi[2] = {0, 0};
         int cnt = 0;
-        for (int base = 0; base < 1024; base += 32) {
+        for (int base = 0; base < (n_words << 5); base += 32) {
           const int u = base + lane;
           const bool k = u < n && (mrow == nullptr || mrow[u] != 0);
           const uint32_t bal = __ballot_sync(0xffffffffu, k);
