@@ -12,6 +12,9 @@ What it computes (plain, slow, obviously correct):
 * ``quant``     -- block quantization: amax -> scale = amax/R -> INT8 or E4M3
                    codes, in IEEE float32 exactly as stated (one division for
                    the scale, one per element for the code).
+* ``nvfp4``     -- per-token NVFP4 quantization: E2M1 codec from the format
+                   definition and the two-level (E4M3 per 16 elements, fp32
+                   per token) scaling in IEEE float32.
 * ``attention`` -- scaled-dot-product attention in float64 on dequantized
                    operands, with causal / 128x128 block masks, GQA and a
                    paged-KV gather.
@@ -25,6 +28,9 @@ Sources (page titles; sections):
   PR #5900), introduction (dense context FMHA, QK-BF16/PV-FP8 and all-FP8).
 * "FlashInfer block-sparse attention with PrimTS" (flashinfer PR #4474),
   section 2 (block-sparse API over contiguous and paged K/V).
+* "FlashInfer per-token NVFP4 quantization kernel" (flashinfer PR #3237),
+  introduction and sections 1-2 (per-token NVFP4 codes, on-chip input
+  staging, a switchable fast-math path).
 
 The pages never write the attention formula down; the oracle uses the
 textbook definition O = softmax(scale * Q K^T) V. Every reading taken where
