@@ -46,6 +46,8 @@ WORKLOADS = {
     "sparse_paged_s16384": ("sparse_paged", 4, 64, 8, 16384, 128, False),
     # decode step: one query token per sequence against S cached tokens (S is Skv)
     "decode_paged_s16384": ("decode_paged", 4, 64, 8, 16384, 128, False),
+    # per-token NVFP4 quantization of S tokens x D channels (B, H unused)
+    "nvfp4_t16384_k4096": ("nvfp4", 1, 1, 1, 16384, 4096, False),
 }
 DEFAULT_WORKLOAD = "dense_pv8_s32768"
 
@@ -277,6 +279,86 @@ def roofline(W, args, attn_ms, achieved_tflops):
             "peak_note": f"{W.peak_src}: {W.peak_note}", "kernel": "attn_fwd_kernel", "kernel_ms": round(attn_ms, 4)}
 
 
+def run_nvfp4(args):
+    """Per-token NVFP4 quantization of a BF16 [S, D] activation matrix: HBM-bound."""
+    from precision_attention_fmha_b200 import fmha
+
+    world, rank, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    _, _, _, _, T, K, _ = WORKLOADS[args.workload]
+    rng = np.random.default_rng(1000 + 7 + T)
+    xh = torch.from_numpy(rng.standard_normal((T, K), dtype=np.float32)).to(torch.bfloat16).pin_memory()
+    x = xh.to(dev)
+    codes = torch.empty((T, K // 2), dtype=torch.uint8, device=dev)
+    sb = torch.empty((T, K // 16), dtype=torch.uint8, device=dev)
+    st = torch.empty((T,), dtype=torch.float32, device=dev)
+    step = lambda inp: fmha.quantize_nvfp4(inp, codes=codes, block_scales=sb, token_scales=st)
+    for _ in range(args.warmup):
+        step(x)
+    fmha.get_device_error()
+    K_ = args.steps
+    stream = torch.cuda.current_stream()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    t0.record(stream)
+    for _ in range(K_):
+        step(x)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    ms = max_over_ranks(t0.elapsed_time(t1) / K_, world)
+    out_bytes = codes.numel() + sb.numel() + st.numel() * 4
+    algo = x.numel() * 2 + out_bytes
+    _, hbm, src = load_peaks()
+    gbs = algo / (ms * 1e-3) / 1e9
+    # end to end: pinned host input in, codes and scales out, every step
+    oh = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (codes, sb, st)]
+    Ke = max(1, min(K_, 10))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(Ke):
+        step(xh.to(dev, non_blocking=True))
+        for h, d in zip(oh, (codes, sb, st)):
+            h.copy_(d, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / Ke, world)
+    fmha.get_device_error()
+    line = {
+        "metric": "per-token NVFP4 quantization GB/s (2 B read + 0.5625 B written per element + 4 B per token)",
+        "value": round(world * gbs, 1), "unit": "GB/s", "n_gpus": world, "steps": K_, "warmup": args.warmup,
+        "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16->e2m1", "data": "synthetic (seeded N(0,1), BF16)",
+        "config": {"workload": "nvfp4_per_token", "tokens": T, "K": K, "l2": "inputs fit in L2" if x.numel() * 2 <= 126 * 2**20
+                   else "inputs larger than L2", "parallelism": f"replicas{world}"},
+        "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": round(hbm, 1), "unit": "GB/s",
+                     "frac": round(gbs / hbm, 4), "traffic": None, "peak_note": f"{src}: HBM copy bandwidth",
+                     "algorithmic_bytes": int(algo), "kernel": "nvfp4_quant_kernel", "kernel_ms": round(ms, 5)},
+        "e2e": {"value": round(world * algo / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+                "h2d_bytes_per_step": x.numel() * 2, "d2h_bytes_per_step": out_bytes, "steps": Ke},
+        "gpu_launches": K_,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        from oracle import nvfp4 as on
+        n = 64
+        tt = time.perf_counter()
+        on.quantize_per_token(xh[:n].to(torch.float32).numpy())
+        dt = time.perf_counter() - tt
+        line["cpu_baseline"] = {"value": round(n * K * 2.5625 / dt / 1e9, 6), "unit": "GB/s", "cores": cpu_cores(),
+                                "kind": "oracle", "sample": f"rows 0..{n - 1} of {T}, NumPy oracle, {dt:.2f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 # ------------------------------------------------------------------ ours ----
 def run_ours(args):
     from precision_attention_fmha_b200 import fmha, workloads
@@ -481,6 +563,34 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def run_reference_nvfp4(args):
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    from oracle import nvfp4 as on
+    _, _, _, _, T, K, _ = WORKLOADS[args.workload]
+    rng = np.random.default_rng(1000 + 7 + T)
+    n = 64  # rows per step: a bounded sample of the T tokens
+    x = torch.from_numpy(rng.standard_normal((n, K), dtype=np.float32)).to(torch.bfloat16).to(torch.float32).numpy()
+    for _ in range(args.warmup):
+        on.quantize_per_token(x)
+    times = []
+    for _ in range(args.steps):
+        t = time.perf_counter()
+        on.quantize_per_token(x)
+        times.append(time.perf_counter() - t)
+    ms = 1e3 * sum(times) / len(times)
+    val = n * K * 2.5625 / (ms * 1e-3) / 1e9
+    print(json.dumps({
+        "impl": "reference", "metric": "per-token NVFP4 quantization GB/s (2 B read + 0.5625 B written per element + 4 B per token)",
+        "value": round(val, 6), "unit": "GB/s", "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded N(0,1), BF16)",
+        "config": {"workload": args.workload, "tokens": T, "K": K},
+        "cpu_baseline": {"value": round(val, 6), "unit": "GB/s", "cores": cpu_cores(), "kind": "oracle",
+                         "sample": f"{n} of {T} rows per step, NumPy oracle"},
+        "e2e": {"value": round(val, 6), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -492,10 +602,11 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
+    nvfp4 = WORKLOADS[args.workload][0] == "nvfp4"
     if args.impl == "reference":
-        run_reference(args)
+        run_reference_nvfp4(args) if nvfp4 else run_reference(args)
     else:
-        run_ours(args)
+        run_nvfp4(args) if nvfp4 else run_ours(args)
 
 
 if __name__ == "__main__":

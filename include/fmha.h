@@ -236,6 +236,27 @@ fmha_status fmha_fwd_decode(const fmha_args* args, const int32_t* page_table, in
                             int64_t mask_stride_b, int64_t mask_stride_h, int32_t num_splits, void* workspace,
                             size_t workspace_bytes, struct CUstream_st* stream);
 
+/* Per-token NVFP4 quantization of a BF16 matrix [rows, K] ("FlashInfer
+ * per-token NVFP4 quantization kernel"): E2M1 element codes, one E4M3 scale
+ * per 16 consecutive elements and one fp32 scale per row (token):
+ *   s_t  = amax_row / 2688  (448 * 6; 1 when the row is zero)
+ *   sb   = E4M3((amax_block / s_t) / 6)      IEEE fp32 divisions, RN, satfinite
+ *   e    = decode(sb) * s_t
+ *   code = E2M1(x / e)  (fast_math != 0: E2M1(x * (1 / e))), 0 when e == 0;
+ *   E2M1 rounds to nearest even and saturates to +-6.
+ *   Dequantization: x ~= e2m1(code) * decode(sb) * s_t.
+ * src: device BF16, 16-byte aligned, row stride in elements (multiple of 8).
+ * codes: device uint8 [rows, K/2], element 2i in the low nibble of byte i,
+ *   8-byte aligned, row stride in bytes (multiple of 8).
+ * block_scales: device uint8 E4M3 [rows, K/16], row stride in bytes.
+ * token_scales: device float [rows].
+ * K: multiple of 16, at most 16384. The caller owns every buffer; nothing is
+ * allocated. FMHA_ERR_UNSUPPORTED for other K, FMHA_ERR_INVALID_ARG for bad
+ * pointers, alignment or strides.                                           */
+fmha_status fmha_quantize_nvfp4(const void* src, int64_t src_row_stride, int32_t rows, int32_t K, uint8_t* codes,
+                                int64_t codes_row_stride, uint8_t* block_scales, int64_t block_scales_row_stride,
+                                float* token_scales, int32_t fast_math, struct CUstream_st* stream);
+
 /* Workspace bytes fmha_fwd_decode needs for these args and num_splits
  * (0: a single split, or invalid sizes). Host only.                         */
 size_t fmha_decode_workspace_bytes(const fmha_args* args, int32_t num_splits);

@@ -549,6 +549,33 @@ fmha_status fmha_fwd_paged(const fmha_args* args, const int32_t* page_table, int
   return run_attention(args, mask, mask_stride_b, mask_stride_h, &pg, stream);
 }
 
+fmha_status fmha_quantize_nvfp4(const void* src, int64_t src_row_stride, int32_t rows, int32_t K, uint8_t* codes,
+                                int64_t codes_row_stride, uint8_t* block_scales, int64_t block_scales_row_stride,
+                                float* token_scales, int32_t fast_math, cudaStream_t stream) {
+  if (rows < 0 || K < 0) return fail(FMHA_ERR_INVALID_ARG, "negative size");
+  if (rows == 0 || K == 0) return ok_status();
+  if (K % 16 != 0 || K > 16384) return fail(FMHA_ERR_UNSUPPORTED, "K = %d (supported: multiples of 16 up to 16384)", K);
+  if (src == nullptr || codes == nullptr || block_scales == nullptr || token_scales == nullptr)
+    return fail(FMHA_ERR_INVALID_ARG, "a pointer is NULL");
+  if (!aligned16(src) || (rows > 1 && ((src_row_stride * 2) % 16 != 0 || src_row_stride < K)))
+    return fail(FMHA_ERR_INVALID_ARG, "src must be 16-byte aligned with a row stride >= K, a multiple of 8 elements");
+  if ((reinterpret_cast<uintptr_t>(codes) & 7u) != 0 || (rows > 1 && (codes_row_stride % 8 != 0 || codes_row_stride < K / 2)))
+    return fail(FMHA_ERR_INVALID_ARG, "codes must be 8-byte aligned with a row stride >= K/2, a multiple of 8 bytes");
+  if (rows > 1 && block_scales_row_stride < K / 16)
+    return fail(FMHA_ERR_INVALID_ARG, "block_scales row stride < K/16");
+  if ((reinterpret_cast<uintptr_t>(token_scales) & 3u) != 0) return fail(FMHA_ERR_INVALID_ARG, "token_scales misaligned");
+  Nvfp4Params p;
+  p.src = static_cast<const uint16_t*>(src); p.src_rs = src_row_stride;
+  p.rows = rows; p.K = K;
+  p.codes = codes; p.codes_rs = codes_row_stride;
+  p.sb = block_scales; p.sb_rs = block_scales_row_stride;
+  p.st = token_scales;
+  p.fast = fast_math ? 1 : 0;
+  cudaError_t e = launch_nvfp4(p, stream);
+  if (e != cudaSuccess) return fail(FMHA_ERR_CUDA, "nvfp4 launch: %s", cudaGetErrorString(e));
+  return ok_status();
+}
+
 size_t fmha_decode_workspace_bytes(const fmha_args* args, int32_t num_splits) {
   if (args == nullptr || args->B <= 0 || args->Hq <= 0 || args->Hkv <= 0 || args->Sq <= 0 || args->Skv < 0 ||
       args->Hq % args->Hkv != 0)

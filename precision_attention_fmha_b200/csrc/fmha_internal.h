@@ -93,6 +93,17 @@ struct MergeParams {
 };
 cudaError_t launch_split_merge(const MergeParams& m, cudaStream_t stream);
 
+// Per-token NVFP4 quantization of a BF16 [rows, K] matrix (K % 16 == 0, K <= 16384).
+struct Nvfp4Params {
+  const uint16_t* src; int64_t src_rs;  // bf16 bits, row stride in elements
+  int32_t rows, K;
+  uint8_t* codes; int64_t codes_rs;     // [rows, K/2] packed E2M1, row stride in bytes
+  uint8_t* sb; int64_t sb_rs;           // [rows, K/16] E4M3 block scales, row stride in bytes
+  float* st;                            // [rows] token scales
+  int32_t fast;                         // 1: x * (1 / e) instead of x / e
+};
+cudaError_t launch_nvfp4(const Nvfp4Params& p, cudaStream_t stream);
+
 // Size of the built-in scratch used by fmha_quantize_blockwise_noalloc, in
 // 32-bit words (one per scale group of the grid-wide granularities).
 constexpr size_t kQuantNoallocScratchWords = 65536;

@@ -76,6 +76,7 @@ def load_library(path=None):
     lib.fmha_fwd_paged.argtypes = [ctypes.POINTER(_Args), vp, i32, i32, i32, vp, i64, i64, vp]
     lib.fmha_get_device_error.argtypes = [vp]
     lib.fmha_fwd_decode.argtypes = [ctypes.POINTER(_Args), vp, i32, i32, i32, vp, i64, i64, i32, vp, sz, vp]
+    lib.fmha_quantize_nvfp4.argtypes = [vp, i64, i32, i32, vp, i64, vp, i64, vp, i32, vp]
     lib.fmha_decode_workspace_bytes.argtypes = [ctypes.POINTER(_Args), i32]
     lib.fmha_decode_workspace_bytes.restype = sz
     lib.fmha_decode_num_splits.argtypes = [ctypes.POINTER(_Args), i32]
@@ -276,6 +277,25 @@ def decode_num_splits(q, k, Skv=None, num_splits=0):
     a = _Args()
     a.B, a.Hq, a.Hkv, a.Sq, a.Skv, a.D = B, Hq, k.shape[2], Sq, k.shape[1] if Skv is None else Skv, D
     return load_library().fmha_decode_num_splits(ctypes.byref(a), int(num_splits))
+
+
+def quantize_nvfp4(x, fast_math=False, codes=None, block_scales=None, token_scales=None, stream=None):
+    """Per-token NVFP4 of a BF16 CUDA matrix [rows, K] (row stride x.stride(0)).
+
+    Returns (codes uint8 [rows, K/2], block_scales float8_e4m3fn [rows, K/16],
+    token_scales float32 [rows])."""
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or x.stride(1) != 1:
+        raise ValueError("x must be a BF16 [rows, K] matrix with unit column stride")
+    rows, K = x.shape
+    dev = x.device
+    codes = torch.empty((rows, K // 2), dtype=torch.uint8, device=dev) if codes is None else codes
+    block_scales = torch.empty((rows, K // 16), dtype=torch.uint8, device=dev) if block_scales is None \
+        else block_scales.view(torch.uint8)
+    token_scales = torch.empty((rows,), dtype=torch.float32, device=dev) if token_scales is None else token_scales
+    _check(load_library().fmha_quantize_nvfp4(x.data_ptr(), x.stride(0), rows, K, codes.data_ptr(), codes.stride(0),
+                                              block_scales.data_ptr(), block_scales.stride(0),
+                                              token_scales.data_ptr(), 1 if fast_math else 0, _stream(stream)))
+    return codes, block_scales.view(torch.float8_e4m3fn), token_scales
 
 
 def decode_workspace_bytes(q, k, Skv=None, num_splits=0):

@@ -97,3 +97,35 @@ def test_paged_argument_checks(lib):
     assert lib.fmha_fwd_paged(ctypes.byref(a), 0x30000, 8, 48, 4, None, 0, 0, None) == 2  # page size
     assert lib.fmha_fwd_paged(ctypes.byref(a), None, 8, 64, 4, None, 0, 0, None) == 1      # no table
     assert lib.fmha_fwd_paged(ctypes.byref(a), 0x30000, 8, 64, 3, None, 0, 0, None) == 1   # too few pages
+
+
+def test_header_declares_decode_and_nvfp4(lib):
+    names = declared_functions()
+    for n in ("fmha_fwd_decode", "fmha_decode_workspace_bytes", "fmha_decode_num_splits", "fmha_quantize_nvfp4"):
+        assert n in names and hasattr(lib, n)
+
+
+def test_nvfp4_argument_checks(lib):
+    f = lib.fmha_quantize_nvfp4
+    src, codes, sb, st = 0x10000, 0x20000, 0x30000, 0x40000
+    assert f(src, 64, 4, 40, codes, 32, sb, 4, st, 0, None) == 2       # K not a multiple of 16
+    assert f(src, 32768, 4, 32768, codes, 16384, sb, 2048, st, 0, None) == 2  # K above 16384
+    assert f(src + 2, 64, 4, 64, codes, 32, sb, 4, st, 0, None) == 1   # src misaligned
+    assert f(src, 60, 4, 64, codes, 32, sb, 4, st, 0, None) == 1       # src row stride < K
+    assert f(src, 64, 4, 64, codes + 4, 32, sb, 4, st, 0, None) == 1   # codes misaligned
+    assert f(src, 64, 4, 64, codes, 28, sb, 4, st, 0, None) == 1       # codes row stride
+    assert f(src, 64, 4, 64, codes, 32, sb, 3, st, 0, None) == 1       # block-scale row stride
+    assert f(None, 64, 4, 64, codes, 32, sb, 4, st, 0, None) == 1      # NULL
+    assert f(src, 64, 0, 64, codes, 32, sb, 4, st, 0, None) == 0       # nothing to do
+
+
+def test_decode_plan_on_host(lib):
+    a = _args()
+    a.B, a.Hq, a.Hkv, a.Sq, a.Skv, a.D = 4, 64, 8, 1, 16384, 128
+    splits = lib.fmha_decode_num_splits(ctypes.byref(a), 4)
+    assert splits == 4
+    # 8 partials (4 splits x the 2 interleaved query tiles), each O [B, Sq, Hq, D] fp32 + lse
+    assert lib.fmha_decode_workspace_bytes(ctypes.byref(a), 4) == 8 * 4 * 1 * 64 * 129 * 4 + 16
+    assert lib.fmha_decode_num_splits(ctypes.byref(a), 1000) == 128
+    a.Sq = 40  # 320 packed rows: no interleave; one split = one partial, no workspace
+    assert lib.fmha_decode_workspace_bytes(ctypes.byref(a), 1) == 0
