@@ -70,3 +70,28 @@ def test_full_size_sampled_rows():
     x = make_rows(19, 16384, 4096)
     rows = np.unique(np.concatenate([[0, 1, 8191, 16383], np.random.default_rng(3).integers(0, 16384, 28)]))
     check(x, False, rows_sample=rows)
+
+
+@pytest.mark.parametrize("fast", [False, True])
+def test_elements_at_rounding_midpoints(fast):
+    """Values whose scaled value x / e falls on or next to an E2M1 rounding
+    midpoint (0.25, 0.75, ..., 5): the exact path must still round RN(x / e)."""
+    rng = np.random.default_rng(23)
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+    rows = []
+    for A in (6.0, 3.0, 0.1875, 448.0, 1.0 / 3.0, 1234.5):
+        a = np.float32(ml_dtypes.bfloat16(A))
+        s_t = np.float32(a / np.float32(2688.0))
+        q = np.float32(np.float32(a / s_t) / np.float32(6.0))
+        from oracle import e4m3
+        sb = e4m3.decode(e4m3.encode(np.array([q])))[0]
+        e = np.float32(np.float32(sb) * s_t)
+        for _ in range(4):
+            row = np.zeros(256, dtype=np.float32)
+            row[0] = a
+            m = rng.choice(mids, 255) * rng.choice([-1.0, 1.0], 255)
+            jitter = 1 + rng.choice([-2.0 ** -8, 0.0, 2.0 ** -8], 255)  # one BF16 step either side, or none
+            row[1:] = (m * e * jitter).astype(np.float32)
+            rows.append(row)
+    x = torch.from_numpy(np.stack(rows)).to(torch.bfloat16)
+    check(x, fast)
