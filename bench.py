@@ -117,36 +117,13 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
 
 
+from precision_attention_fmha_b200.replicas import barrier, job_throughput, max_over_ranks, teardown  # noqa: E402
+from precision_attention_fmha_b200.replicas import setup as replicas_setup  # noqa: E402
+
+
 def dist_setup(n_gpus):
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        import datetime
-
-        import torch.distributed as dist
-
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
-    return world, rank, local
-
-
-def barrier(world):
-    if world > 1:
-        import torch.distributed as dist
-
-        dist.barrier()
-
-
-def max_over_ranks(x, world):
-    if world == 1:
-        return x
-    import torch.distributed as dist
-
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
+    """Replicas only: one process per GPU over NCCL, no collective on the data path."""
+    return replicas_setup("nccl")
 
 
 # ------------------------------------------------------------- workloads ----
@@ -357,6 +334,7 @@ def run_nvfp4(args):
                                 "kind": "oracle", "sample": f"rows 0..{n - 1} of {T}, NumPy oracle, {dt:.2f} s"}
     if rank == 0:
         print(json.dumps(line), flush=True)
+    teardown(world)
 
 
 # ------------------------------------------------------------------ ours ----
@@ -437,7 +415,7 @@ def run_ours(args):
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / Ke, world)
     fmha.get_device_error()
 
-    tflops = world * W.flop / (ms * 1e-3) / 1e12
+    tflops = job_throughput(W.flop, world, ms) / 1e12
     achieved = W.flop / (attn_ms * 1e-3) / 1e12
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -459,10 +437,7 @@ def run_ours(args):
         line["cpu_baseline"] = cpu
     if rank == 0:
         print(json.dumps(line), flush=True)
-    if world > 1:
-        import torch.distributed as dist
-
-        dist.destroy_process_group()
+    teardown(world)
 
 
 # DRAM bytes (read + write) of one attention launch from an ncu capture of the
