@@ -585,6 +585,42 @@ def run_reference_nvfp4(args):
         "e2e": {"value": round(val, 6), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}), flush=True)
 
 
+def probe_peaks():
+    """Library GEMM peaks on this GPU (8192^3, best of 10, CUDA events): bf16
+    torch.matmul, E4M3 torch._scaled_mm (fp32 scales, bf16 out), INT8
+    torch._int_mm. Context for the 8-bit rooflines; the reported peaks stay
+    MEASURED_PEAKS.json's bf16 burst with the nominal 2x ratio for 8-bit."""
+    dev = torch.device("cuda")
+    n = 8192
+    a = torch.randn(n, n, device=dev, dtype=torch.bfloat16)
+    b = torch.randn(n, n, device=dev, dtype=torch.bfloat16)
+    a8, b8 = a.to(torch.float8_e4m3fn), b.to(torch.float8_e4m3fn).t().contiguous().t()
+    one = torch.ones((), device=dev, dtype=torch.float32)
+    ai = torch.randint(-100, 100, (n, n), device=dev, dtype=torch.int8)
+    bi = torch.randint(-100, 100, (n, n), device=dev, dtype=torch.int8).t().contiguous().t()
+    runs = {"bf16_matmul": lambda: a @ b,
+            "e4m3_scaled_mm": lambda: torch._scaled_mm(a8, b8, scale_a=one, scale_b=one, out_dtype=torch.bfloat16),
+            "int8_int_mm": lambda: torch._int_mm(ai, bi)}
+    out = {}
+    for name, f in runs.items():
+        try:
+            for _ in range(3):
+                f()
+            torch.cuda.synchronize()
+            best = 1e30
+            for _ in range(10):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                f()
+                e1.record()
+                torch.cuda.synchronize()
+                best = min(best, e0.elapsed_time(e1))
+            out[name] = round(2.0 * n ** 3 / (best * 1e-3) / 1e12, 1)
+        except Exception as e:  # a dtype path this torch build lacks
+            out[name] = f"unavailable: {type(e).__name__}: {e}"[:160]
+    print(json.dumps({"probe": "library GEMM peaks, 8192^3, TFLOP/s (TOP/s for int8)", **out}), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -593,7 +629,11 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--probe-peaks", action="store_true", help="print library GEMM peaks (bf16, E4M3, INT8) and exit")
     args = ap.parse_args()
+    if args.probe_peaks:
+        probe_peaks()
+        return
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
     nvfp4 = WORKLOADS[args.workload][0] == "nvfp4"
