@@ -86,7 +86,7 @@ struct AttnCfg {
   static constexpr bool TURNS = PSMEM;  // exp-phase turn-taking between the softmax warpgroups
   static constexpr int P_TILE = BM * BN;  // bytes per E4M3 P tile
   static constexpr int P_BYTES = PSMEM ? 2 * P_TILE * (P2 ? 2 : 1) : 0;
-  static constexpr int MISC_BYTES = 1024;
+  static constexpr int MISC_BYTES = 2048;
   static constexpr int SMEM_CAP = 232448;  // 227 KB opt-in maximum per CTA
   static constexpr int STAGES_FIT = (SMEM_CAP - 1024 - MISC_BYTES - 2 * Q_TILE - P_BYTES) / SLOT;
   static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
@@ -105,13 +105,20 @@ struct AttnCfg {
   // 3 warpgroups: softmax tile 0, softmax tile 1, control (MMA warp, TMA warp, 2 idle).
   // Launch: 384 threads x 168 registers = 64512; after re-balancing
   // 2 x 128 x 224 + 128 x 56 = 64512 (the sum must not exceed the launch total).
-  static constexpr int THREADS = 384;
+  // Threads per query row in the softmax. 2 splits every row's 128 scores
+  // between two warps of the same TMEM lane quadrant (64 columns each, 640
+  // threads, a row-max exchange per tile); it is correct but measured 10-15 %
+  // slower than one thread per row (more warps per scheduler, 104 registers).
+  static constexpr int NH = 1;
+  static constexpr int THREADS = 128 + 256 * NH;
   // Warp roles: warpgroup 0 = control (MMA issue, TMA loads, two idle warps),
   // warpgroups 1 and 2 = softmax of query tiles 0 and 1. The control warps
   // come first: the issue scheduler favours older warps, and the MMA warp's
   // short serial steps sit on the critical path of both softmax pipelines.
   static constexpr int MMA_WARP = 0, LOAD_WARP = 1, SOFTMAX_WARP0 = 4;
-  static constexpr uint32_t SOFTMAX_REGS = 216, CONTROL_REGS = 72;
+  // setmaxnreg split of the launch's registers (THREADS x 168 or x 96):
+  // 384 threads: 2*128*216 + 128*72; 640 threads: 4*128*104 + 128*64.
+  static constexpr uint32_t SOFTMAX_REGS = NH == 2 ? 104 : 216, CONTROL_REGS = NH == 2 ? 64 : 72;
   static_assert(2 * 128 * SOFTMAX_REGS + 128 * CONTROL_REGS <= THREADS * 168, "register split exceeds launch");
 };
 
@@ -133,9 +140,11 @@ struct alignas(8) AttnMisc {
   // over KV tiles (at most 1024), and its [first, last + 1) range.
   uint32_t keep_bits[2][32];
   int32_t range[2][2];
+  // Two threads per row: one exchange slot per row of each query tile.
+  float xchg[2][128];
 };
 
-static_assert(sizeof(AttnMisc) <= 1024, "AttnMisc must fit the 1 KB misc area");
+static_assert(sizeof(AttnMisc) <= 2048, "AttnMisc must fit the 2 KB misc area");
 
 struct TileInfo {
   int h;      // query head (packed: first head of the KV head's group)
@@ -159,7 +168,9 @@ struct Waiter {
   uint32_t* err;
   uint64_t budget;
   __device__ __forceinline__ bool wait(uint32_t bar, uint32_t parity) const {
-    if (ptx::mbar_try_wait(bar, parity)) return true;
+    // First a non-blocking test: try_wait may itself suspend the thread for a
+    // hardware-chosen time, which would let a short limit never run out.
+    if (ptx::mbar_test_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (true) {
       // The limit is checked before every sleeping probe, so a limit shorter
@@ -643,11 +654,14 @@ __device__ void attn_mma_role_psmem(const AttnParams& p, const TileInfo t0, cons
 // with packed fp32x2 FMAs feeding MUFU ex2, pack P (BF16 or E4M3) over the
 // first S columns and release it to the MMA warp with one arrive per warp.
 template <class C>
-__device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, int b, int hkv, uint8_t* sQx,
-                                  uint8_t* sPx, int n_turns, AttnMisc* misc, uint32_t tmem,
+__device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, int h, int b, int hkv,
+                                  uint8_t* sQx, uint8_t* sPx, int n_turns, AttnMisc* misc, uint32_t tmem,
                                   const CUtensorMap* tmO, const Waiter w) {
   using namespace ptx;
   constexpr uint32_t FULL = 0xffffffffu;
+  // h: which part of each row this thread owns when NH threads share a row:
+  // S columns [32 * NC * h, 32 * NC * (h + 1)), O columns likewise over D.
+  constexpr int NH = C::NH, NC = 4 / NH, OB = C::D / 32 / NH;
   const int warp = (threadIdx.x >> 5) & 3;  // TMEM lane quadrant of this warp
   const int lane = threadIdx.x & 31;
   const int r = warp * 32 + lane;  // row within the tile
@@ -658,6 +672,30 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, 
   const uint32_t tS = tmem + lane_off + (x ? 128u : 0u);
   const uint32_t tO = tmem + lane_off + (x ? 256u + C::D : 256u);
   const int wg_tid = threadIdx.x & 127;
+  const bool lead = wg_tid == 0 && h == 0;  // one thread of the query tile
+  // The two threads of a row meet through one shared-memory slot and the
+  // named barrier of their lane quadrant's two warps (ids 3..10).
+  const uint32_t pair_bar = 3u + 4u * x + warp;
+  // ok_io: in, this thread's wait results; out, the AND over both threads, so
+  // that the two warps of a pair always leave the tile loop together (named
+  // barriers have no time limit: a warp must not wait for a partner that left).
+  auto pair_combine = [&](float v, bool is_max, bool& ok_io) {
+    if constexpr (NH == 1) {
+      return v;
+    } else {
+      float* slot = &misc->xchg[x][r];
+      if (h == 1) *slot = v;
+      ok_io = named_bar_and(pair_bar, 64, ok_io);
+      float res = v;
+      if (h == 0) {
+        res = is_max ? fmaxf(v, *slot) : v + *slot;
+        *slot = res;
+      }
+      named_bar_sync(pair_bar, 64);
+      if (h == 1) res = *slot;
+      return res;
+    }
+  };
   const int64_t bhq = static_cast<int64_t>(b) * p.Hq + head;
   const int64_t bhk = static_cast<int64_t>(b) * p.Hkv + hkv;
 
@@ -685,40 +723,41 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, 
   bool ok = true;
   for (int u = t.u0; u < t.n_kv; ++u) {
     if (!keep_tile<C>(p, t, b, hkv, u, misc)) continue;
-    TRACE(x * 8192 + it * 16 + 0, wg_tid == 0);
-    ok = __all_sync(FULL, w.wait(smem_addr(&misc->s_full[x]), it & 1));
-    if (!ok) break;
-    TRACE(x * 8192 + it * 16 + 1, wg_tid == 0);
+    TRACE(x * 8192 + it * 16 + 0, lead);
+    // A failed wait does not leave the loop here: the exchange below does, for
+    // both threads of the row at once (the work in between is harmless).
+    ok = __all_sync(FULL, w.wait(smem_addr(&misc->s_full[x]), it & 1)) && ok;
+    TRACE(x * 8192 + it * 16 + 1, lead);
     tc_fence_after();
 
     // Column factors: K scale per 32-key chunk (token-block K scales), times cq.
     const int kv0 = u * C::BN;
-    float ck[4];
+    float ck[NC];
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
+    for (int c = 0; c < NC; ++c) {
       float f = ck_uniform;
       if (C::QK != QK_BF16 && p.sf_k_kind == FMHA_SF_PER_TOKEN_BLOCK)
-        f = p.sf_k[bhk * p.sf_k_nblk + min(kv0 + 32 * c, p.Skv - 1) / p.sf_k_rpb];
+        f = p.sf_k[bhk * p.sf_k_nblk + min(kv0 + 32 * (NC * h + c), p.Skv - 1) / p.sf_k_rpb];
       ck[c] = f * cq;
     }
     int lim = p.Skv - kv0;  // keys at or past `lim` in this tile are hidden
     if (p.causal) lim = min(lim, row + 1 + (p.Skv - p.Sq) - kv0);
 
-    uint32_t s[4][32];
+    uint32_t s[NC][32];
 #pragma unroll
-    for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, s[c]);
+    for (int c = 0; c < NC; ++c) tmem_ld32(tS + 32 * (NC * h + c), s[c]);
     tmem_wait_ld();
 #pragma unroll
-    for (int c = 0; c < 4; ++c) reg_fence(s[c]);
+    for (int c = 0; c < NC; ++c) reg_fence(s[c]);
     if constexpr (C::PSMEM) {  // S is in registers: the MMA warp may issue the next QK^T into this tile
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_addr(&misc->s_free[x]));
     }
-    TRACE(x * 8192 + it * 16 + 2, wg_tid == 0);
-    float f[4][32];
+    TRACE(x * 8192 + it * 16 + 2, lead);
+    float f[NC][32];
 #pragma unroll
-    for (int c = 0; c < 4; ++c)
+    for (int c = 0; c < NC; ++c)
 #pragma unroll
       for (int j = 0; j < 32; ++j) {
         if constexpr (C::QK == QK_INT8)
@@ -728,14 +767,14 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, 
       }
     if (lim < C::BN) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+      for (int c = 0; c < NC; ++c)
 #pragma unroll
         for (int j = 0; j < 32; ++j)
-          if (32 * c + j >= lim) f[c][j] = -INFINITY;
+          if (32 * (NC * h + c) + j >= lim) f[c][j] = -INFINITY;
     }
-    float mc[4];
+    float mc[NC];
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
+    for (int c = 0; c < NC; ++c) {
       float a0 = fmax3(f[c][0], f[c][1], f[c][2]), a1 = fmax3(f[c][3], f[c][4], f[c][5]);
 #pragma unroll
       for (int j = 6; j < 30; j += 4) {
@@ -744,7 +783,13 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, 
       }
       mc[c] = fmax3(a0, a1, fmaxf(f[c][30], f[c][31])) * ck[c];
     }
-    const float m_tile = fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3]));
+    float m_part = mc[0];
+#pragma unroll
+    for (int c = 1; c < NC; ++c) m_part = fmaxf(m_part, mc[c]);
+    // Both threads of the row have loaded their S columns once they meet here,
+    // so P may overwrite S columns of either part from now on.
+    const float m_tile = pair_combine(m_part, true, ok);
+    if (!ok) break;
     const float m_new = fmaxf(m, m_tile);
     float alpha = 1.f;
     bool resc = false;
@@ -761,14 +806,14 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, 
     auto rescale_o = [&]() {
       if (__any_sync(FULL, resc)) {
 #pragma unroll 1
-        for (int c = 0; c < C::D / 32; ++c) {
+        for (int c = 0; c < OB; ++c) {  // this thread's O columns
           uint32_t o[32];
-          tmem_ld32(tO + 32 * c, o);
+          tmem_ld32(tO + 32 * (OB * h + c), o);
           tmem_wait_ld();
           reg_fence(o);
 #pragma unroll
           for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-          tmem_st32(tO + 32 * c, o);
+          tmem_st32(tO + 32 * (OB * h + c), o);
         }
       }
     };
@@ -777,58 +822,60 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, 
     // walk the same KV tiles) the warpgroups alternate their exponential
     // phases, so that one exponentiates while the other loads, reduces and
     // packs. Tile 0 goes first.
-    TRACE(x * 8192 + it * 16 + 3, wg_tid == 0);
+    TRACE(x * 8192 + it * 16 + 3, lead);
     if (x == 0 ? (it >= 1 && it < n_turns) : (it < n_turns)) {
-      ok = __all_sync(FULL, w.wait(smem_addr(&misc->exp_done[x ^ 1]), (x == 0 ? it - 1 : it) & 1));
-      if (!ok) break;
+      ok = __all_sync(FULL, w.wait(smem_addr(&misc->exp_done[x ^ 1]), (x == 0 ? it - 1 : it) & 1)) && ok;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) reg_fence(f[c]);
+      for (int c = 0; c < NC; ++c) reg_fence(f[c]);
     }
-    TRACE(x * 8192 + it * 16 + 4, wg_tid == 0);
+    TRACE(x * 8192 + it * 16 + 4, lead);
     const float mb = (m == -INFINITY ? 0.f : m) - log2g;
 #pragma unroll
-    for (int c = 0; c < 4; ++c)
+    for (int c = 0; c < NC; ++c)
 #pragma unroll
       for (int j = 0; j < 32; j += 2) ffma2(f[c][j], f[c][j + 1], f[c][j], f[c][j + 1], ck[c], ck[c], -mb, -mb);
 #pragma unroll
-    for (int c = 0; c < 4; ++c)
+    for (int c = 0; c < NC; ++c)
 #pragma unroll
       for (int j = 0; j < 32; ++j) f[c][j] = ex2(f[c][j]);
     if (x == 0 ? (it < n_turns) : (it + 1 < n_turns)) {
 #pragma unroll
-      for (int c = 0; c < 4; ++c) reg_fence(f[c]);
+      for (int c = 0; c < NC; ++c) reg_fence(f[c]);
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_addr(&misc->exp_done[x]));
     }
-    TRACE(x * 8192 + it * 16 + 5, wg_tid == 0);
+    TRACE(x * 8192 + it * 16 + 5, lead);
     float rs = 0.f;
     if constexpr (C::PV == PV_BF16) {
-      uint32_t pk[2][32];
+      // BF16 P of this thread's columns goes over TMEM columns [32 * NC/2 * h, ...)
+      // of S (two values per column); the pair exchange above ordered it after
+      // both threads' S loads.
+      uint32_t pk[NC / 2][32];
       float r0 = 0.f, r1 = 0.f, r2 = 0.f, r3 = 0.f;
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+      for (int c = 0; c < NC; ++c)
 #pragma unroll
         for (int j = 0; j < 16; ++j) pk[c >> 1][(c & 1) * 16 + j] = pack_bf16x2(f[c][2 * j], f[c][2 * j + 1]);
 #pragma unroll
-      for (int c = 0; c < 4; ++c)
+      for (int c = 0; c < NC; ++c)
 #pragma unroll
         for (int j = 0; j < 32; j += 4) {
           fadd2(r0, r1, r0, r1, f[c][j], f[c][j + 1]);
           fadd2(r2, r3, r2, r3, f[c][j + 2], f[c][j + 3]);
         }
       rs = (r0 + r1) + (r2 + r3);
-      tmem_st32(tS, pk[0]);
-      tmem_st32(tS + 32, pk[1]);
+#pragma unroll
+      for (int q = 0; q < NC / 2; ++q) tmem_st32(tS + 32 * (NC / 2 * h + q), pk[q]);
     } else {
-      uint32_t pk[32];
-      [[maybe_unused]] uint32_t pl[32];
+      uint32_t pk[8 * NC];
+      [[maybe_unused]] uint32_t pl[8 * NC];
       if constexpr (C::P2) {
         // Two-term E4M3 P: hi = E4M3(p g), lo = E4M3(p g - hi) (the residual taken
         // in f16), ~7 significant bits between them; both feed their own PV
         // product. The row sum adds the unrounded values (as precise as BF16 P).
         float r0 = 0.f, r1 = 0.f, r2 = 0.f, r3 = 0.f;
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
+        for (int c = 0; c < NC; ++c)
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
             const float* e = &f[c][4 * j];
@@ -844,9 +891,9 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, 
       } else {
         // The row sum adds the E4M3-rounded values actually stored, so the
         // normalised weights sum to one and a dominant key returns its value.
-        float racc[4];
+        float racc[NC];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < NC; ++c) {
           uint32_t acc[2] = {0u, 0u};
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
@@ -857,45 +904,48 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, 
           }
           racc[c] = f16x2_sum(acc[0]) + f16x2_sum(acc[1]);
         }
-        rs = (racc[0] + racc[1]) + (racc[2] + racc[3]);
+        rs = racc[0];
+#pragma unroll
+        for (int c = 1; c < NC; ++c) rs += racc[c];
       }
-      TRACE(x * 8192 + it * 16 + 6, wg_tid == 0);
+      TRACE(x * 8192 + it * 16 + 6, lead);
       if constexpr (C::PSMEM) {
         // The previous PV must be done before P (single buffer) or O is rewritten.
         if (it > 0) {
-          ok = __all_sync(FULL, w.wait(smem_addr(&misc->pv_done[x]), (it - 1) & 1));
-          if (!ok) break;
+          ok = __all_sync(FULL, w.wait(smem_addr(&misc->pv_done[x]), (it - 1) & 1)) && ok;
           tc_fence_after();
         }
-        TRACE(x * 8192 + it * 16 + 7, wg_tid == 0);
+        TRACE(x * 8192 + it * 16 + 7, lead);
         rescale_o();
         // Row r of the 128 x 128-byte P tile, 16-byte chunks XOR-swizzled by r % 8
-        // (the 128-byte swizzle the PV descriptor expects).
+        // (the 128-byte swizzle the PV descriptor expects); this thread writes
+        // the chunks of its columns.
         const uint32_t prow = smem_addr(sPx) + r * 128;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) {
+        for (int kk = 0; kk < 2 * NC; ++kk) {
+          const int k = 2 * NC * h + kk;
           const uint32_t addr = prow + ((k ^ (r & 7)) << 4);
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[4 * k]), "r"(pk[4 * k + 1]),
-                       "r"(pk[4 * k + 2]), "r"(pk[4 * k + 3])
+          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[4 * kk]), "r"(pk[4 * kk + 1]),
+                       "r"(pk[4 * kk + 2]), "r"(pk[4 * kk + 3])
                        : "memory");
           if constexpr (C::P2)
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr + C::P_TILE), "r"(pl[4 * k]),
-                         "r"(pl[4 * k + 1]), "r"(pl[4 * k + 2]), "r"(pl[4 * k + 3])
+            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr + C::P_TILE), "r"(pl[4 * kk]),
+                         "r"(pl[4 * kk + 1]), "r"(pl[4 * kk + 2]), "r"(pl[4 * kk + 3])
                          : "memory");
         }
         fence_proxy_async_smem();  // generic-proxy P writes -> tensor-core reads
-      } else {
+      } else if constexpr (NH == 1) {  // E4M3 P in TMEM (unused while E4M3 P goes through shared memory)
         tmem_st32(tS, pk);
         if constexpr (C::P2) tmem_st32(tS + 32, pl);
       }
     }
     l = l * alpha + rs;
-    TRACE(x * 8192 + it * 16 + 8, wg_tid == 0);
+    TRACE(x * 8192 + it * 16 + 8, lead);
     tmem_wait_st();
     tc_fence_before();
     __syncwarp();  // the warp's P stores are ordered before lane 0's arrive
     if (lane == 0) mbar_arrive(smem_addr(&misc->p_full[x]));
-    TRACE(x * 8192 + it * 16 + 9, wg_tid == 0);
+    TRACE(x * 8192 + it * 16 + 9, lead);
     ++it;
   }
 
@@ -910,67 +960,73 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, 
     tc_fence_after();
     have_o = ok;
   }
+  // The row sum of the stored P: the threads of a row add their parts.
+  {
+    bool ok_pair = ok;
+    l = pair_combine(l, false, ok_pair);
+  }
   float sfv = 1.f;
   if (C::PV == PV_E4M3 && p.sf_v_kind != FMHA_SF_PER_CHANNEL) sfv = sf_lookup(p.sf_v, p.sf_v_kind, bhk, 1, 0, 1);
   const float inv_l = l > 0.f ? sfv / l : 0.f;
   const uint32_t stage0 = smem_addr(sQx);
+  constexpr uint32_t TILE_THREADS = 128 * NH;
 #pragma unroll 1
   for (int c64 = 0; c64 < C::D / 64; ++c64) {
+    // 32-column blocks of this 64-column chunk held by this thread (its O
+    // columns are [32 * OB * h, 32 * OB * (h + 1))); warp-uniform.
+    const bool mine[2] = {(2 * c64) / OB == h, (2 * c64 + 1) / OB == h};
     uint32_t o[2][32];
     if (have_o) {
-      tmem_ld32(tO + 64 * c64, o[0]);
-      tmem_ld32(tO + 64 * c64 + 32, o[1]);
+      if (mine[0]) tmem_ld32(tO + 64 * c64, o[0]);
+      if (mine[1]) tmem_ld32(tO + 64 * c64 + 32, o[1]);
       tmem_wait_ld();
       reg_fence(o[0]);
       reg_fence(o[1]);
     }
+    auto out_val = [&](int col) {  // column col (0..63) of this chunk, scaled
+      float v = have_o ? __uint_as_float(o[col >> 5][col & 31]) * inv_l : 0.f;
+      if (C::PV == PV_E4M3 && p.sf_v_kind == FMHA_SF_PER_CHANNEL) v *= misc->sf_v[64 * c64 + col];
+      return v;
+    };
     if constexpr (C::PACKED) {
       if (p.n_parts > 1) {  // one partial: O / l in fp32 for the merge kernel (no staging)
         if (row < p.Sq && ok) {
           float* dst = p.o_part + ((((int64_t)t.part * p.B + b) * p.Sq + row) * p.Hq + head) * C::D + 64 * c64;
 #pragma unroll
           for (int j = 0; j < 64; j += 4) {
-            float v4[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              v4[e] = have_o ? __uint_as_float(o[(j + e) >> 5][(j + e) & 31]) * inv_l : 0.f;
-              if (C::PV == PV_E4M3 && p.sf_v_kind == FMHA_SF_PER_CHANNEL) v4[e] *= misc->sf_v[64 * c64 + j + e];
-            }
-            asm volatile("st.global.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst + j), "f"(v4[0]), "f"(v4[1]),
-                         "f"(v4[2]), "f"(v4[3])
+            if (!mine[j >> 5]) continue;
+            asm volatile("st.global.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst + j), "f"(out_val(j)),
+                         "f"(out_val(j + 1)), "f"(out_val(j + 2)), "f"(out_val(j + 3))
                          : "memory");
           }
         }
         continue;
       }
     }
-    uint32_t pk[32];
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      float a = have_o ? __uint_as_float(o[j >> 4][(2 * j) & 31]) * inv_l : 0.f;
-      float bb = have_o ? __uint_as_float(o[j >> 4][(2 * j + 1) & 31]) * inv_l : 0.f;
-      if (C::PV == PV_E4M3 && p.sf_v_kind == FMHA_SF_PER_CHANNEL) {
-        a *= misc->sf_v[64 * c64 + 2 * j];
-        bb *= misc->sf_v[64 * c64 + 2 * j + 1];
-      }
-      pk[j] = pack_bf16x2(a, bb);
-    }
     const int buf = c64 % C::O_STAGE_BUFS;
     if (c64 >= C::O_STAGE_BUFS) {  // buffer reuse: the previous store must have read it
-      if (wg_tid == 0) bulk_wait_read0();
-      named_bar_sync(1 + x, 128);
+      if (lead) bulk_wait_read0();
+      named_bar_sync(1 + x, TILE_THREADS);
     }
     const uint32_t base = stage0 + buf * C::CHUNK_BYTES + r * 128;
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const uint32_t addr = base + ((k ^ (r & 7)) << 4);
-      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[4 * k]), "r"(pk[4 * k + 1]),
-                   "r"(pk[4 * k + 2]), "r"(pk[4 * k + 3])
-                   : "memory");
+    for (int sc = 0; sc < 2; ++sc) {
+      if (!mine[sc]) continue;
+      uint32_t pk[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) pk[j] = pack_bf16x2(out_val(32 * sc + 2 * j), out_val(32 * sc + 2 * j + 1));
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const int k = 4 * sc + kk;
+        const uint32_t addr = base + ((k ^ (r & 7)) << 4);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[4 * kk]), "r"(pk[4 * kk + 1]),
+                     "r"(pk[4 * kk + 2]), "r"(pk[4 * kk + 3])
+                     : "memory");
+      }
     }
     fence_proxy_async_smem();
-    named_bar_sync(1 + x, 128);
-    if (wg_tid == 0 && ok) {
+    named_bar_sync(1 + x, TILE_THREADS);
+    if (lead && ok) {
       if constexpr (C::PACKED)
         tma_store_5d(tmO, stage0 + buf * C::CHUNK_BYTES, 64 * c64, 0, hkv, t.tok0, b);
       else
@@ -979,12 +1035,14 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, 
     }
   }
   const float lse = l > 0.f ? (m + __log2f(l) - log2g) * 0.69314718055994531f : -INFINITY;
-  if (C::PACKED && p.n_parts > 1) {
-    if (row < p.Sq && ok) p.lse_part[(((int64_t)t.part * p.B + b) * p.Hq + head) * p.Sq + row] = lse;
-  } else if (p.lse != nullptr && row < p.Sq && ok) {
-    p.lse[bhq * p.Sq + row] = lse;
+  if (h == 0) {
+    if (C::PACKED && p.n_parts > 1) {
+      if (row < p.Sq && ok) p.lse_part[(((int64_t)t.part * p.B + b) * p.Hq + head) * p.Sq + row] = lse;
+    } else if (p.lse != nullptr && row < p.Sq && ok) {
+      p.lse[bhq * p.Sq + row] = lse;
+    }
   }
-  if (wg_tid == 0) bulk_wait0();
+  if (lead) bulk_wait0();
 }
 
 // ------------------------------------------------------------------ kernel --
@@ -1129,14 +1187,14 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     mbar_init(smem_addr(&misc->q_full), 1);
     for (int x = 0; x < 2; ++x) {
       mbar_init(smem_addr(&misc->s_full[x]), 1);
-      mbar_init(smem_addr(&misc->p_full[x]), 4);  // one arrive per softmax warp
+      mbar_init(smem_addr(&misc->p_full[x]), 4 * C::NH);  // one arrive per softmax warp
     }
     mbar_init(smem_addr(&misc->o_full), 1);
     mbar_init(smem_addr(&misc->drain), 1);
     for (int x = 0; x < 2; ++x) {
-      mbar_init(smem_addr(&misc->s_free[x]), 4);  // one arrive per softmax warp
+      mbar_init(smem_addr(&misc->s_free[x]), 4 * C::NH);  // one arrive per softmax warp
       mbar_init(smem_addr(&misc->pv_done[x]), 1);
-      mbar_init(smem_addr(&misc->exp_done[x]), 4);  // one arrive per softmax warp
+      mbar_init(smem_addr(&misc->exp_done[x]), 4 * C::NH);  // one arrive per softmax warp
     }
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(smem_addr(&misc->kv_full[s]), 1);
@@ -1174,16 +1232,18 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     }
   }
 
-  if (warp >= C::SOFTMAX_WARP0 && warp < C::SOFTMAX_WARP0 + 8) {
+  if (warp >= C::SOFTMAX_WARP0 && warp < C::SOFTMAX_WARP0 + 8 * C::NH) {
     regs_inc<C::SOFTMAX_REGS>();
-    const int x = (warp - C::SOFTMAX_WARP0) >> 2;
+    const int x = (warp - C::SOFTMAX_WARP0) / (4 * C::NH);     // query tile
+    const int h = ((warp - C::SOFTMAX_WARP0) >> 2) % C::NH;   // part of each row
     const TileInfo tx = x ? t[1] : t[0];  // select by value (no runtime-indexed array)
     // Exp turn-taking needs both tiles to walk the same KV tiles (dense masks:
     // prefixes [0, n_kv)); with a block mask the lists differ, so it is off.
     int n_turns = 0;
     if (C::TURNS && !C::PACKED && p.mask == nullptr) n_turns = min(t[0].n_kv, t[1].n_kv);
     if (tx.valid)
-      attn_softmax_role<C>(p, tx, x, b, hkv, x ? sQ[1] : sQ[0], x ? sP[1] : sP[0], n_turns, misc, tmem, &tmO, w);
+      attn_softmax_role<C>(p, tx, x, h, b, hkv, x ? sQ[1] : sQ[0], x ? sP[1] : sP[0], n_turns, misc, tmem, &tmO,
+                           w);
   } else {
     regs_dec<C::CONTROL_REGS>();
     if (warp == C::MMA_WARP) {  // the whole warp; one elected lane issues
