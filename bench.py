@@ -447,9 +447,9 @@ def run_ours(args):
 #       python bench.py [--workload W] --steps 1 --warmup 1 --no-cpu-baseline
 # (one pass; summary in profiles/attn_fwd_pv8_dram_traffic.md).
 TRAFFIC = {
-    "dense_pv8_s32768": 844.54e6 + 315.89e6,  # compulsory: Q,K 335.5 MB + V 167.8 MB read, O 335.5 MB written
-    "dense_pv8_s16384": 421.07e6 + 145.54e6,
-    "decode_paged_s16384": 69.24e6 + 1.24e6 + 1.08e6,  # attention (kept K/V read once) + split merge
+    "dense_pv8_s32768": 847.74e6 + 315.64e6,  # compulsory: Q,K 335.5 MB + V 167.8 MB read, O 335.5 MB written
+    "dense_pv8_s16384": 420.76e6 + 145.64e6,
+    "decode_paged_s16384": 69.25e6 + 1.01e6 + 1.08e6,  # attention (kept K/V read once) + split merge
 }
 
 
