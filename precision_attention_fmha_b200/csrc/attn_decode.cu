@@ -52,17 +52,28 @@ __global__ void __launch_bounds__(128) split_merge_kernel(const MergeParams m) {
   if (mx != -INFINITY) {
     const long long split_stride_o = static_cast<long long>(m.B) * m.Sq * m.Hq * m.D;
     const long long o_off = ((static_cast<long long>(b) * m.Sq + tok) * m.Hq + h) * m.D + 4 * lane;
-    for (int j = 0; j < m.n_splits; ++j) {
-      const float lj = m.lse_part[j * split_stride_lse + lse_off];
-      if (lj == -INFINITY) continue;
-      const float wj = expf(lj - mx);
-      wsum += wj;
-      if (4 * lane < m.D) {
-        const float4 v = *reinterpret_cast<const float4*>(m.o_part + j * split_stride_o + o_off);
-        acc[0] += wj * v.x;
-        acc[1] += wj * v.y;
-        acc[2] += wj * v.z;
-        acc[3] += wj * v.w;
+    // Partials in groups of 8: all loads of a group are issued before any is
+    // used, so the row pays about one memory latency per group, not per partial.
+    for (int j0 = 0; j0 < m.n_splits; j0 += 8) {
+      float lj[8];
+      float4 v[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const int j = j0 + k;
+        lj[k] = j < m.n_splits ? m.lse_part[j * split_stride_lse + lse_off] : -INFINITY;
+        v[k] = (j < m.n_splits && 4 * lane < m.D)
+                   ? *reinterpret_cast<const float4*>(m.o_part + j * split_stride_o + o_off)
+                   : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        if (lj[k] == -INFINITY) continue;  // a split that saw no key
+        const float wj = expf(lj[k] - mx);
+        wsum += wj;
+        acc[0] += wj * v[k].x;
+        acc[1] += wj * v[k].y;
+        acc[2] += wj * v[k].z;
+        acc[3] += wj * v[k].w;
       }
     }
   }
