@@ -9,20 +9,24 @@
 //
 // One CTA owns two 128-row query tiles X = 0, 1 that share every K/V tile
 // (either two consecutive query blocks of one head, or the same query block
-// of two query heads that read the same KV head). 384 threads, one CTA/SM:
-//   warps 0-3  softmax for tile 0 (TMEM lanes 0-127: one query row per thread)
-//   warps 4-7  softmax for tile 1
-//   warp  8    tensor-core issue (one thread): S = Q K^T and O += P V
-//   warp  9    TMA producer (one thread): Q once, then K_j, V_j into a ring
-//   warps 10-11 idle (they complete the third warpgroup, whose registers are
-//              handed to the softmax warpgroups with setmaxnreg)
+// of two query heads that read the same KV head; for decode, GQA-packed tiles
+// of one KV head's query heads). 384 threads, one CTA/SM:
+//   warp  0     tensor-core issue (warp-uniform, one elected lane issues)
+//   warp  1     TMA producer (warp-uniform; one tile's copies from several lanes)
+//   warps 2-3   idle (warp 2 picks decode splits' KV tiles in the prologue);
+//               warpgroup 0 hands its registers to the softmax with setmaxnreg
+//   warps 4-7   softmax for tile 0 (TMEM lanes 0-127: one query row per thread)
+//   warps 8-11  softmax for tile 1
 // TMEM (512 columns): S0 [0,128) S1 [128,256) O0 [256,256+D) O1 [256+D,256+2D).
-// The softmax writes P (BF16 or E4M3) over the first columns of its S tile and
-// the PV product reads P straight from TMEM, so P never touches shared memory.
-// Because the issue thread orders S_X(j+1) after PV_X(j), the arrival of
-// S_X(j+1) also proves PV_X(j) finished; the softmax warps therefore rescale O
-// themselves (only when the running row max grows by more than 2^tau, the
-// "lazy correction" of the Blackwell page, section 3) before releasing P_X(j+1).
+// BF16 P is written over the first columns of its S tile and the PV product
+// reads it from TMEM; the issue order puts S_X(j+1) after PV_X(j), so the
+// arrival of S_X(j+1) proves PV_X(j) finished and the softmax rescales O itself
+// (only when the running row max grows by more than 2^tau, the "lazy
+// correction" of the Blackwell page, section 3) before releasing P_X(j+1).
+// E4M3 P goes to shared memory instead (the Blackwell page, section 1), so a
+// tile's S columns are free once the softmax has loaded them: QK^T of the next
+// KV tile overlaps the softmax, and the two softmax warpgroups take turns in
+// their exp2 phases.
 // The epilogue scales O by 1/l (and the V / P scale factors), converts to BF16,
 // stages 64-column halves in the dead Q buffer and writes them with TMA stores
 // ("FlashInfer DeepSeek-V4 sparse-MLA: Cake backend", section 1: output through
@@ -102,9 +106,6 @@ struct AttnCfg {
                                                        : ptx::make_idesc(2, 1, 1, 0, 0, BN, BM);
   static constexpr uint32_t IDESC_PV =
       PV == PV_BF16 ? ptx::make_idesc(1, 1, 1, 0, 1, D, BM) : ptx::make_idesc(1, 0, 0, 0, 1, D, BM);
-  // 3 warpgroups: softmax tile 0, softmax tile 1, control (MMA warp, TMA warp, 2 idle).
-  // Launch: 384 threads x 168 registers = 64512; after re-balancing
-  // 2 x 128 x 224 + 128 x 56 = 64512 (the sum must not exceed the launch total).
   // Threads per query row in the softmax. 2 splits every row's 128 scores
   // between two warps of the same TMEM lane quadrant (64 columns each, 640
   // threads, a row-max exchange per tile); it is correct but measured 10-15 %
