@@ -449,7 +449,7 @@ def run_ours(args):
 TRAFFIC = {
     "dense_pv8_s32768": 847.74e6 + 315.64e6,  # compulsory: Q,K 335.5 MB + V 167.8 MB read, O 335.5 MB written
     "dense_pv8_s16384": 420.76e6 + 145.64e6,
-    "decode_paged_s16384": 69.25e6 + 1.01e6 + 1.08e6,  # attention (kept K/V read once) + split merge
+    "decode_paged_s16384": 69.25e6 + 0.89e6 + 1.08e6,  # attention (kept K/V read once) + split merge
 }
 
 
