@@ -11,7 +11,9 @@ What it computes (plain, slow, obviously correct):
                    format definition (bias 7, no infinities, max 448).
 * ``quant``     -- block quantization: amax -> scale = amax/R -> INT8 or E4M3
                    codes, in IEEE float32 exactly as stated (one division for
-                   the scale, one per element for the code).
+                   the scale, one per element for the code); the token mean
+                   per channel and quantization of x minus a shift, for
+                   SageAttention's K smoothing.
 * ``nvfp4``     -- per-token NVFP4 quantization: E2M1 codec from the format
                    definition and the two-level (E4M3 per 16 elements, fp32
                    per token) scaling in IEEE float32.

@@ -58,14 +58,48 @@ def num_blocks(S, rows_per_block):
     return (S + rows_per_block - 1) // rows_per_block
 
 
-def quantize_blockwise(x, out_dtype, kind, rows_per_block=None):
+def channel_mean(x):
+    """Token mean of x [B, S, H, D] for every (b, h, d) -> float32 [B, H, D].
+
+    K smoothing. SageAttention quantizes K after subtracting K's mean over the
+    tokens (Zhang et al., "SageAttention: Accurate 8-Bit Attention for
+    Plug-and-play Inference Acceleration", 2024, smoothing of K). The pages
+    name SageAttention and its block-wise scale factors, but not this step.
+    The readings taken are:
+    * the mean runs over all S tokens of one (b, h), separately per channel d;
+    * the S values (exact in float32) are summed in float64, the sum is
+      divided by S in float64, and the quotient is rounded once to float32;
+    * S = 0 gives a zero mean.
+    A shift that is constant over the tokens of one (b, h) moves every score of
+    a query row by the same amount, q . mean. Softmax ignores that, so O is
+    unchanged, and the log-sum-exp moves by softmax_scale * q . mean.
+    """
+    x = np.asarray(x, dtype=np.float32)
+    B, S, H, D = x.shape
+    if S == 0:
+        return np.zeros((B, H, D), dtype=np.float32)
+    total = x.astype(np.float64).sum(axis=1)  # [B, H, D]
+    return (total / np.float64(S)).astype(np.float32)
+
+
+def quantize_blockwise(x, out_dtype, kind, rows_per_block=None, shift=None):
     """x: float32 array [B, S, H, D] (exact BF16 values). Returns (codes, scales).
 
     codes has x's shape (int8, or uint8 E4M3 bit patterns); scales is float32
     with the layout of ``kind`` given in the module docstring.
+
+    shift (optional, float32 [B, H, D], e.g. ``channel_mean(x)``): the values
+    quantized are x - shift, one float32 round-to-nearest-even subtraction per
+    element, and every block's amax is taken over those differences. The codes
+    then dequantize to x - shift.
     """
     x = np.asarray(x, dtype=np.float32)
     B, S, H, D = x.shape
+    if shift is not None:
+        sh = np.asarray(shift, dtype=np.float32)
+        if sh.shape != (B, H, D):
+            raise ValueError(f"shift must have shape {(B, H, D)}, got {sh.shape}")
+        x = (x - sh[:, None, :, :]).astype(np.float32)
     codes = np.zeros(x.shape, dtype=np.int8 if out_dtype == "int8" else np.uint8)
     if kind == "per_tensor":
         scale = scale_from_amax(np.max(np.abs(x)) if x.size else np.float32(0), out_dtype)
