@@ -181,6 +181,42 @@ fmha_status fmha_quantize_blockwise_noalloc(const fmha_tensor* src, const fmha_t
                                             int32_t B, int32_t S, int32_t H, int32_t D,
                                             struct CUstream_st* stream);
 
+/* K smoothing for the SageAttention path. (The pages name SageAttention and
+ * its block scales, not this step; it follows the SageAttention paper, Zhang
+ * et al. 2024: quantize K minus its mean over the tokens.) A shift that is
+ * constant over the keys of one (b, h_kv) moves every score of a query row by
+ * softmax_scale * q . shift. Softmax ignores that, so attention on the
+ * smoothed keys gives the same O. The log-sum-exp (fmha_args.lse) is that of
+ * the smoothed scores, lower by softmax_scale * q . shift. Smoothing removes
+ * a per-channel bias from K before its blocks are scaled, which makes the
+ * INT8 steps smaller.
+ *
+ * fmha_channel_mean: mean[b, h, d] = fp32(sum_s x[b, s, h, d] / S), for
+ *   src BF16 [B, S, H, D] (element strides, D contiguous, 16-byte aligned
+ *   rows) and mean fp32 [B, H, D] contiguous (device, caller-owned). The sum
+ *   is taken in fp64 in a fixed order (per CTA, then over CTAs), divided by S
+ *   in fp64 and rounded once to fp32. Results do not depend on timing. They
+ *   equal any other summation order wherever the fp64 sum of the S values is
+ *   exact, which holds for BF16 inputs whose magnitudes span at most about
+ *   2^(45 - log2 S). S = 0 gives zeros. D must be a power of two in [8, 2048].
+ *   workspace: device, 8-byte aligned, at least
+ *   fmha_channel_mean_workspace_bytes(B, S, H, D) bytes (0 when S == 0). It
+ *   must not be shared with a concurrent call.
+ * fmha_quantize_blockwise_shifted: fmha_quantize_blockwise applied to
+ *   x - shift, with shift fp32 [B, H, D] contiguous (device, 16-byte aligned,
+ *   not NULL), normally the output of fmha_channel_mean. Each element is first
+ *   reduced by one fp32 round-to-nearest subtraction, and the amax, scale and
+ *   code rules apply to that difference. The codes dequantize to
+ *   x - shift. Other arguments, the workspace rule and the errors are those
+ *   of fmha_quantize_blockwise.                                              */
+size_t fmha_channel_mean_workspace_bytes(int32_t B, int32_t S, int32_t H, int32_t D);
+fmha_status fmha_channel_mean(const fmha_tensor* src, float* mean, int32_t B, int32_t S, int32_t H, int32_t D,
+                              void* workspace, size_t workspace_bytes, struct CUstream_st* stream);
+fmha_status fmha_quantize_blockwise_shifted(const fmha_tensor* src, const float* shift, const fmha_tensor* dst,
+                                            const fmha_sf* sf, int32_t B, int32_t S, int32_t H, int32_t D,
+                                            void* workspace, size_t workspace_bytes,
+                                            struct CUstream_st* stream);
+
 /* Dense attention (optionally causal) over contiguous K/V ([BW-FP8] intro). */
 fmha_status fmha_fwd(const fmha_args* args, struct CUstream_st* stream);
 

@@ -443,6 +443,13 @@ fmha_status run_attention(const fmha_args* a, const uint8_t* mask, int64_t msb, 
   return ok_status();
 }
 
+// Token rows one CTA of the channel-mean kernel sums: 16 KB of BF16 input.
+int mean_rows_per_cta(int D) { return D >= 8 ? (2048 / (D / 8) > 0 ? 2048 / (D / 8) : 1) : 1; }
+
+fmha_status quantize_impl(const fmha_tensor* src, const float* shift, const fmha_tensor* dst, const fmha_sf* sf,
+                          int32_t B, int32_t S, int32_t H, int32_t D, void* workspace, size_t workspace_bytes,
+                          cudaStream_t stream);
+
 size_t quant_groups(int kind, int B, int H, int D) {
   switch (kind) {
     case FMHA_SF_PER_TENSOR: return 1;
@@ -459,6 +466,63 @@ extern "C" {
 fmha_status fmha_quantize_blockwise(const fmha_tensor* src, const fmha_tensor* dst, const fmha_sf* sf, int32_t B,
                                     int32_t S, int32_t H, int32_t D, void* workspace, size_t workspace_bytes,
                                     cudaStream_t stream) {
+  return quantize_impl(src, nullptr, dst, sf, B, S, H, D, workspace, workspace_bytes, stream);
+}
+
+fmha_status fmha_quantize_blockwise_shifted(const fmha_tensor* src, const float* shift, const fmha_tensor* dst,
+                                            const fmha_sf* sf, int32_t B, int32_t S, int32_t H, int32_t D,
+                                            void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  if (shift == nullptr) return fail(FMHA_ERR_INVALID_ARG, "shift is NULL");
+  if (reinterpret_cast<uintptr_t>(shift) & 15u) return fail(FMHA_ERR_INVALID_ARG, "shift must be 16-byte aligned");
+  return quantize_impl(src, shift, dst, sf, B, S, H, D, workspace, workspace_bytes, stream);
+}
+
+size_t fmha_channel_mean_workspace_bytes(int32_t B, int32_t S, int32_t H, int32_t D) {
+  if (B <= 0 || S <= 0 || H <= 0 || D < 8) return 0;
+  return size_t(B) * H * ceil_div(S, mean_rows_per_cta(D)) * D * sizeof(double);
+}
+
+fmha_status fmha_channel_mean(const fmha_tensor* src, float* mean, int32_t B, int32_t S, int32_t H, int32_t D,
+                              void* workspace, size_t workspace_bytes, cudaStream_t stream) {
+  if (src == nullptr) return fail(FMHA_ERR_INVALID_ARG, "NULL argument");
+  if (B < 0 || S < 0 || H < 0 || D < 0) return fail(FMHA_ERR_INVALID_ARG, "negative size");
+  if (src->dtype != FMHA_BF16) return fail(FMHA_ERR_UNSUPPORTED, "channel mean input must be BF16");
+  if (D < 8 || D > 2048 || (D & (D - 1)) != 0)
+    return fail(FMHA_ERR_UNSUPPORTED, "channel mean needs D a power of two in [8, 2048]");
+  if (B == 0 || H == 0) return ok_status();
+  if (mean == nullptr || (reinterpret_cast<uintptr_t>(mean) & 3u))
+    return fail(FMHA_ERR_INVALID_ARG, "mean is NULL or misaligned");
+  if (S > 0) {
+    fmha_status st;
+    if ((st = check_tensor(*src, "src", B, S, H, D)) != FMHA_OK) return st;
+    const size_t need = fmha_channel_mean_workspace_bytes(B, S, H, D);
+    if (workspace == nullptr || workspace_bytes < need)
+      return fail(FMHA_ERR_INVALID_ARG, "workspace needs %zu bytes", need);
+    if (reinterpret_cast<uintptr_t>(workspace) & 7u) return fail(FMHA_ERR_INVALID_ARG, "workspace misaligned");
+  }
+  QuantParams p;
+  memset(&p, 0, sizeof(p));
+  p.src = static_cast<const uint16_t*>(src->ptr);
+  p.s_sb = src->stride_b; p.s_ss = src->stride_s; p.s_sh = src->stride_h;
+  p.B = B; p.S = S; p.H = H; p.D = D;
+  p.rows_per_cta = mean_rows_per_cta(D);
+  p.n_chunks = S > 0 ? ceil_div(S, p.rows_per_cta) : 0;
+  p.partial = static_cast<double*>(workspace);
+  p.mean = mean;
+  if (static_cast<int64_t>(p.n_chunks) > 65535 || H > 65535 || B > 65535)
+    return fail(FMHA_ERR_UNSUPPORTED, "grid too large");
+  cudaError_t e = launch_channel_mean(p, stream);
+  if (e != cudaSuccess) return fail(FMHA_ERR_CUDA, "channel mean launch: %s", cudaGetErrorString(e));
+  return ok_status();
+}
+
+}  // extern "C"
+
+namespace {
+
+fmha_status quantize_impl(const fmha_tensor* src, const float* shift, const fmha_tensor* dst, const fmha_sf* sf,
+                          int32_t B, int32_t S, int32_t H, int32_t D, void* workspace, size_t workspace_bytes,
+                          cudaStream_t stream) {
   if (src == nullptr || dst == nullptr || sf == nullptr) return fail(FMHA_ERR_INVALID_ARG, "NULL argument");
   if (B < 0 || S < 0 || H < 0 || D < 0) return fail(FMHA_ERR_INVALID_ARG, "negative size");
   if (src->dtype != FMHA_BF16) return fail(FMHA_ERR_UNSUPPORTED, "quantizer input must be BF16");
@@ -503,10 +567,15 @@ fmha_status fmha_quantize_blockwise(const fmha_tensor* src, const fmha_tensor* d
   p.B = B; p.S = S; p.H = H; p.D = D;
   p.ws = static_cast<uint32_t*>(workspace);
   p.rows_per_cta = 2048 / (D / 8) > 0 ? 2048 / (D / 8) : 1;
+  p.shift = shift;
   cudaError_t e = launch_quantize(dst->dtype == FMHA_E4M3, p, stream);
   if (e != cudaSuccess) return fail(FMHA_ERR_CUDA, "quantizer launch: %s", cudaGetErrorString(e));
   return ok_status();
 }
+
+}  // namespace
+
+extern "C" {
 
 size_t fmha_quantize_workspace_bytes(int32_t sf_kind, int32_t B, int32_t S, int32_t H, int32_t D) {
   (void)S;

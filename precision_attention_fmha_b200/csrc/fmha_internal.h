@@ -72,7 +72,12 @@ struct QuantParams {
   float* sf; int32_t kind; int32_t rpb; int32_t nblk;
   int32_t B, S, H, D;
   uint32_t* ws;          // amax accumulators (float bits) for the grid-wide kinds
-  int32_t rows_per_cta;  // grid-wide kinds: token rows per CTA
+  int32_t rows_per_cta;  // grid-wide kinds and the token mean: token rows per CTA
+  const float* shift;    // nullable fp32 [B, H, D]: values quantized are x - shift
+  // Token mean per channel (K smoothing): per-CTA fp64 partial sums, then the mean.
+  double* partial;       // [B, H, n_chunks, D]
+  float* mean;           // [B, H, D]
+  int32_t n_chunks;
 };
 
 // Launchers (defined in the .cu files). They return cudaSuccess or the launch error.
@@ -80,6 +85,7 @@ cudaError_t launch_attention(int qk_kind, int pv_kind, int D, bool paged, const 
                              const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                              const CUtensorMap& to, cudaStream_t stream);
 cudaError_t launch_quantize(bool to_e4m3, const QuantParams& p, cudaStream_t stream);
+cudaError_t launch_channel_mean(const QuantParams& p, cudaStream_t stream);
 // Decode path: attention over GQA-packed tiles (p.packed = 1), then, for
 // n_splits > 1, the split merge into o (bf16, element strides) and lse.
 cudaError_t launch_attention_packed(int qk_kind, int pv_kind, bool paged, const AttnParams& p,

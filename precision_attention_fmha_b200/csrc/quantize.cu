@@ -18,6 +18,12 @@
 // Grid-wide granularities (per tensor / head / channel): pass 1 reduces amax
 // into the caller's workspace with atomicMax on the (non-negative) fp32 bit
 // patterns, pass 2 re-reads and quantizes: 2 + 2 + 1 B/element.
+//
+// K smoothing (SageAttention, Zhang et al. 2024): every kernel can quantize
+// x - shift[b, h, d] instead of x (one fp32 round-to-nearest subtraction per
+// element, before the amax). The shift is normally the token mean per channel,
+// which channel_mean_* computes: fp64 partial sums per CTA, then a fixed-order
+// sum over the CTAs, one fp64 division by S and one rounding to fp32.
 #include <mutex>
 
 #include "fmha_internal.h"
@@ -37,13 +43,29 @@ __device__ __forceinline__ void unpack8(const uint4& v, float (&x)[8]) {
   x[4] = bf16_lo(v.z); x[5] = bf16_hi(v.z); x[6] = bf16_lo(v.w); x[7] = bf16_hi(v.w);
 }
 
-__device__ __forceinline__ float amax8(const uint4& v) {
-  float x[8];
+// The 8 values of one 16-byte vector, minus the shift of its 8 channels when
+// shift_c (16-byte aligned) is not null.
+__device__ __forceinline__ void vals8(const uint4& v, const float* shift_c, float (&x)[8]) {
   unpack8(v, x);
+  if (shift_c != nullptr) {
+    const float4 a = __ldg(reinterpret_cast<const float4*>(shift_c));
+    const float4 c = __ldg(reinterpret_cast<const float4*>(shift_c + 4));
+    x[0] = __fsub_rn(x[0], a.x); x[1] = __fsub_rn(x[1], a.y); x[2] = __fsub_rn(x[2], a.z);
+    x[3] = __fsub_rn(x[3], a.w); x[4] = __fsub_rn(x[4], c.x); x[5] = __fsub_rn(x[5], c.y);
+    x[6] = __fsub_rn(x[6], c.z); x[7] = __fsub_rn(x[7], c.w);
+  }
+}
+
+__device__ __forceinline__ float amax8(const float (&x)[8]) {
   float m = 0.f;
 #pragma unroll
   for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(x[i]));
   return m;
+}
+
+// Shift of column vector c of head (b, h), or null when nothing is subtracted.
+__device__ __forceinline__ const float* shift_at(const QuantParams& p, int64_t bh, int c) {
+  return p.shift != nullptr ? p.shift + bh * p.D + c * 8 : nullptr;
 }
 
 __device__ __forceinline__ uint4 ld16(const uint16_t* p) { return __ldg(reinterpret_cast<const uint4*>(p)); }
@@ -73,9 +95,7 @@ __device__ __forceinline__ uint32_t code4(float a, float b, float c, float d, fl
 }
 
 template <bool kE4M3>
-__device__ __forceinline__ uint2 code8(const uint4& v, const float (&s)[8]) {
-  float x[8];
-  unpack8(v, x);
+__device__ __forceinline__ uint2 code8(const float (&x)[8], const float (&s)[8]) {
   return make_uint2(code4<kE4M3>(x[0], x[1], x[2], x[3], s[0], s[1], s[2], s[3]),
                     code4<kE4M3>(x[4], x[5], x[6], x[7], s[4], s[5], s[6], s[7]));
 }
@@ -108,6 +128,8 @@ __global__ void __launch_bounds__(kThreads) quant_token_block_kernel(const Quant
   const uint16_t* src = p.src + b * p.s_sb + static_cast<int64_t>(s0) * p.s_ss + h * p.s_sh;
   uint8_t* dst = p.dst + b * p.d_sb + static_cast<int64_t>(s0) * p.d_ss + h * p.d_sh;
 
+  const int64_t bh = static_cast<int64_t>(b) * p.H + h;
+
   uint4 cache[kCacheVecs];
   float amax = 0.f;
 #pragma unroll
@@ -116,12 +138,16 @@ __global__ void __launch_bounds__(kThreads) quant_token_block_kernel(const Quant
     if (v < nvec) {
       const int r = v / vpr, c = v - r * vpr;
       cache[i] = ld16(src + r * p.s_ss + c * 8);
-      amax = fmaxf(amax, amax8(cache[i]));
+      float x[8];
+      vals8(cache[i], shift_at(p, bh, c), x);
+      amax = fmaxf(amax, amax8(x));
     }
   }
   for (int v = threadIdx.x + kCacheVecs * kThreads; v < nvec; v += kThreads) {
     const int r = v / vpr, c = v - r * vpr;
-    amax = fmaxf(amax, amax8(ld16(src + r * p.s_ss + c * 8)));
+    float x[8];
+    vals8(ld16(src + r * p.s_ss + c * 8), shift_at(p, bh, c), x);
+    amax = fmaxf(amax, amax8(x));
   }
   amax = block_reduce_max(amax, red);
   const float scale = scale_from_amax<kE4M3>(amax);
@@ -133,14 +159,18 @@ __global__ void __launch_bounds__(kThreads) quant_token_block_kernel(const Quant
     const int v = threadIdx.x + i * kThreads;
     if (v < nvec) {
       const int r = v / vpr, c = v - r * vpr;
-      *reinterpret_cast<uint2*>(dst + r * p.d_ss + c * 8) = code8<kE4M3>(cache[i], s8);
+      float x[8];
+      vals8(cache[i], shift_at(p, bh, c), x);
+      *reinterpret_cast<uint2*>(dst + r * p.d_ss + c * 8) = code8<kE4M3>(x, s8);
     }
   }
   for (int v = threadIdx.x + kCacheVecs * kThreads; v < nvec; v += kThreads) {
     const int r = v / vpr, c = v - r * vpr;
-    *reinterpret_cast<uint2*>(dst + r * p.d_ss + c * 8) = code8<kE4M3>(ld16(src + r * p.s_ss + c * 8), s8);
+    float x[8];
+    vals8(ld16(src + r * p.s_ss + c * 8), shift_at(p, bh, c), x);
+    *reinterpret_cast<uint2*>(dst + r * p.d_ss + c * 8) = code8<kE4M3>(x, s8);
   }
-  if (threadIdx.x == 0) p.sf[(static_cast<int64_t>(b) * p.H + h) * p.nblk + blk] = scale;
+  if (threadIdx.x == 0) p.sf[bh * p.nblk + blk] = scale;
 }
 
 // Grid-wide kinds, pass 1: per-CTA amax over rows [chunk*rows_per_cta, ...) of
@@ -154,12 +184,13 @@ __global__ void __launch_bounds__(kThreads) quant_amax_kernel(const QuantParams 
   const int vpr = p.D >> 3;
   const int nvec = rows * vpr;
   const uint16_t* src = p.src + b * p.s_sb + static_cast<int64_t>(s0) * p.s_ss + h * p.s_sh;
+  const int64_t bh = static_cast<int64_t>(b) * p.H + h;
   if (p.kind == FMHA_SF_PER_CHANNEL) {
     float m[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     for (int v = threadIdx.x; v < nvec; v += kThreads) {
       const int r = v / vpr, c = v - r * vpr;
       float x[8];
-      unpack8(ld16(src + r * p.s_ss + c * 8), x);
+      vals8(ld16(src + r * p.s_ss + c * 8), shift_at(p, bh, c), x);
 #pragma unroll
       for (int i = 0; i < 8; ++i) m[i] = fmaxf(m[i], fabsf(x[i]));
     }
@@ -171,17 +202,19 @@ __global__ void __launch_bounds__(kThreads) quant_amax_kernel(const QuantParams 
       const int cv = ch >> 3, j = ch & 7;
       float a = 0.f;
       for (int k = 0; k < step; ++k) a = fmaxf(a, red[(cv + k * vpr) * 8 + j]);
-      atomicMax(p.ws + (static_cast<int64_t>(b) * p.H + h) * p.D + ch, __float_as_uint(a));
+      atomicMax(p.ws + bh * p.D + ch, __float_as_uint(a));
     }
   } else {
     float m = 0.f;
     for (int v = threadIdx.x; v < nvec; v += kThreads) {
       const int r = v / vpr, c = v - r * vpr;
-      m = fmaxf(m, amax8(ld16(src + r * p.s_ss + c * 8)));
+      float x[8];
+      vals8(ld16(src + r * p.s_ss + c * 8), shift_at(p, bh, c), x);
+      m = fmaxf(m, amax8(x));
     }
     m = block_reduce_max(m, red);
     if (threadIdx.x == 0) {
-      const int64_t g = p.kind == FMHA_SF_PER_HEAD ? static_cast<int64_t>(b) * p.H + h : 0;
+      const int64_t g = p.kind == FMHA_SF_PER_HEAD ? bh : 0;
       atomicMax(p.ws + g, __float_as_uint(m));
     }
   }
@@ -210,7 +243,9 @@ __global__ void __launch_bounds__(kThreads) quant_apply_kernel(const QuantParams
   }
   for (int v = threadIdx.x; v < nvec; v += kThreads) {
     const int r = v / vpr, c = v - r * vpr;
-    *reinterpret_cast<uint2*>(dst + r * p.d_ss + c * 8) = code8<kE4M3>(ld16(src + r * p.s_ss + c * 8), s8);
+    float x[8];
+    vals8(ld16(src + r * p.s_ss + c * 8), shift_at(p, bh, c), x);
+    *reinterpret_cast<uint2*>(dst + r * p.d_ss + c * 8) = code8<kE4M3>(x, s8);
   }
   if (chunk == 0) {
     if (p.kind == FMHA_SF_PER_CHANNEL) {
@@ -244,10 +279,66 @@ cudaError_t launch_quantize_t(const QuantParams& p, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+// Token mean, pass 1: CTA (chunk, h, b) sums rows [chunk * rows_per_cta, ...)
+// of (b, h) per channel in fp64. Each thread owns one column vector (256 is a
+// multiple of D / 8) and a fixed set of rows; the threads of a column vector
+// are then added in thread order, so the partial sums do not depend on timing.
+__global__ void __launch_bounds__(kThreads) channel_mean_partial_kernel(const QuantParams p) {
+  __shared__ double red[kThreads * 8];
+  const int chunk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  const int s0 = chunk * p.rows_per_cta;
+  const int rows = min(p.S - s0, p.rows_per_cta);
+  const int vpr = p.D >> 3;
+  const int cv = threadIdx.x % vpr, row_step = kThreads / vpr;
+  const uint16_t* src = p.src + b * p.s_sb + static_cast<int64_t>(s0) * p.s_ss + h * p.s_sh + cv * 8;
+  double acc[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
+#pragma unroll 4
+  for (int r = threadIdx.x / vpr; r < rows; r += row_step) {
+    float x[8];
+    unpack8(ld16(src + r * p.s_ss), x);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] += static_cast<double>(x[i]);
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) red[threadIdx.x * 8 + i] = acc[i];
+  __syncthreads();
+  const int64_t bh = static_cast<int64_t>(b) * p.H + h;
+  for (int ch = threadIdx.x; ch < p.D; ch += kThreads) {
+    const int c = ch >> 3, j = ch & 7;
+    double a = 0.0;
+    for (int k = 0; k < row_step; ++k) a += red[(c + k * vpr) * 8 + j];
+    p.partial[(bh * p.n_chunks + chunk) * p.D + ch] = a;
+  }
+}
+
+// Token mean, pass 2: one thread per (b, h, d) adds the chunks in order,
+// divides by S in fp64 and rounds once to fp32.
+__global__ void __launch_bounds__(kThreads) channel_mean_final_kernel(const QuantParams p) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;
+  if (i >= static_cast<int64_t>(p.B) * p.H * p.D) return;
+  const int64_t bh = i / p.D, ch = i - bh * p.D;
+  const double* part = p.partial + bh * p.n_chunks * p.D + ch;
+  double a = 0.0;
+  for (int c = 0; c < p.n_chunks; ++c) a += part[static_cast<int64_t>(c) * p.D];
+  p.mean[i] = __double2float_rn(__ddiv_rn(a, static_cast<double>(p.S)));
+}
+
 }  // namespace
 
 cudaError_t launch_quantize(bool to_e4m3, const QuantParams& p, cudaStream_t stream) {
   return to_e4m3 ? launch_quantize_t<true>(p, stream) : launch_quantize_t<false>(p, stream);
+}
+
+cudaError_t launch_channel_mean(const QuantParams& p, cudaStream_t stream) {
+  const int64_t n = static_cast<int64_t>(p.B) * p.H * p.D;
+  if (n == 0) return cudaSuccess;
+  if (p.S == 0) return cudaMemsetAsync(p.mean, 0, n * sizeof(float), stream);
+  dim3 grid(p.n_chunks, p.H, p.B);
+  channel_mean_partial_kernel<<<grid, kThreads, 0, stream>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  channel_mean_final_kernel<<<static_cast<unsigned>((n + kThreads - 1) / kThreads), kThreads, 0, stream>>>(p);
+  return cudaGetLastError();
 }
 
 // Built-in scratch for fmha_quantize_blockwise_noalloc: the amax accumulators

@@ -71,6 +71,11 @@ def load_library(path=None):
                                             i32, i32, i32, i32, vp, sz, vp]
     lib.fmha_quantize_workspace_bytes.argtypes = [i32, i32, i32, i32, i32]
     lib.fmha_quantize_workspace_bytes.restype = sz
+    lib.fmha_quantize_blockwise_shifted.argtypes = [ctypes.POINTER(_Tensor), vp, ctypes.POINTER(_Tensor),
+                                                    ctypes.POINTER(_Sf), i32, i32, i32, i32, vp, sz, vp]
+    lib.fmha_channel_mean.argtypes = [ctypes.POINTER(_Tensor), vp, i32, i32, i32, i32, vp, sz, vp]
+    lib.fmha_channel_mean_workspace_bytes.argtypes = [i32, i32, i32, i32]
+    lib.fmha_channel_mean_workspace_bytes.restype = sz
     lib.fmha_fwd.argtypes = [ctypes.POINTER(_Args), vp]
     lib.fmha_fwd_block_sparse.argtypes = [ctypes.POINTER(_Args), vp, i64, i64, vp]
     lib.fmha_fwd_paged.argtypes = [ctypes.POINTER(_Args), vp, i32, i32, i32, vp, i64, i64, vp]
@@ -86,7 +91,7 @@ def load_library(path=None):
     lib.fmha_last_error_message.restype = ctypes.c_char_p
     lib.fmha_set_wait_timeout_cycles.argtypes = [ctypes.c_uint64]
     for f in ("fmha_quantize_blockwise", "fmha_fwd", "fmha_fwd_block_sparse", "fmha_fwd_paged",
-              "fmha_get_device_error"):
+              "fmha_get_device_error", "fmha_quantize_blockwise_shifted", "fmha_channel_mean"):
         getattr(lib, f).restype = ctypes.c_int
     if path == LIB_PATH:
         _lib = lib
@@ -150,9 +155,16 @@ def scale_shape(kind, B, S, H, D, rows_per_block=None):
 
 
 def fmha_quantize_blockwise(x, out_dtype, kind, rows_per_block=None, out=None, scales=None, workspace=None,
-                            stream=None):
-    """BF16 x [B,S,H,D] -> (codes, fp32 scales). out_dtype: torch.int8 or torch.float8_e4m3fn."""
+                            stream=None, shift=None):
+    """BF16 x [B,S,H,D] -> (codes, fp32 scales). out_dtype: torch.int8 or torch.float8_e4m3fn.
+
+    shift (optional, contiguous fp32 [B, H, D] on the device): quantize
+    x - shift instead of x (K smoothing; see ``channel_mean``).
+    """
     lib = load_library()
+    if shift is not None and (shift.dtype != torch.float32 or not shift.is_contiguous()
+                              or tuple(shift.shape) != (x.shape[0], x.shape[2], x.shape[3])):
+        raise ValueError("shift must be a contiguous float32 [B, H, D] tensor")
     B, S, H, D = x.shape
     if out is None:
         out = torch.empty((B, S, H, D), dtype=out_dtype, device=x.device)
@@ -165,9 +177,41 @@ def fmha_quantize_blockwise(x, out_dtype, kind, rows_per_block=None, out=None, s
     sf = _Sf(scales.data_ptr(), SF_KINDS[kind], int(rows_per_block or 0))
     ws_ptr = workspace.data_ptr() if workspace is not None else None
     ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
-    _check(lib.fmha_quantize_blockwise(ctypes.byref(src), ctypes.byref(dst), ctypes.byref(sf), B, S, H, D,
-                                       ws_ptr, ws_bytes, _stream(stream)))
+    if shift is None:
+        _check(lib.fmha_quantize_blockwise(ctypes.byref(src), ctypes.byref(dst), ctypes.byref(sf), B, S, H, D,
+                                           ws_ptr, ws_bytes, _stream(stream)))
+    else:
+        _check(lib.fmha_quantize_blockwise_shifted(ctypes.byref(src), shift.data_ptr(), ctypes.byref(dst),
+                                                   ctypes.byref(sf), B, S, H, D, ws_ptr, ws_bytes, _stream(stream)))
     return out, scales
+
+
+def channel_mean_workspace_bytes(B, S, H, D):
+    return load_library().fmha_channel_mean_workspace_bytes(B, S, H, D)
+
+
+def channel_mean(x, out=None, workspace=None, stream=None):
+    """Token mean per (b, h, d) of BF16 x [B, S, H, D] -> fp32 [B, H, D] (fp64 sums)."""
+    lib = load_library()
+    B, S, H, D = x.shape
+    if out is None:
+        out = torch.empty((B, H, D), dtype=torch.float32, device=x.device)
+    need = lib.fmha_channel_mean_workspace_bytes(B, S, H, D)
+    if need and workspace is None:
+        workspace = torch.empty(need, dtype=torch.uint8, device=x.device)
+    src = _tensor(x)
+    ws_ptr = workspace.data_ptr() if workspace is not None else None
+    ws_bytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check(lib.fmha_channel_mean(ctypes.byref(src), out.data_ptr(), B, S, H, D, ws_ptr, ws_bytes,
+                                 _stream(stream)))
+    return out
+
+
+def quantize_smoothed(x, out_dtype, kind, rows_per_block=None, stream=None):
+    """SageAttention K smoothing: (codes, scales, mean) with codes * scales ~= x - mean."""
+    mean = channel_mean(x, stream=stream)
+    codes, scales = fmha_quantize_blockwise(x, out_dtype, kind, rows_per_block, stream=stream, shift=mean)
+    return codes, scales, mean
 
 
 def _args(q, k, v, out, sf_q, sf_k, sf_v, sf_p, softmax_scale, causal, lse, Skv=None, p_terms=1):
