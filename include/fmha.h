@@ -121,7 +121,12 @@ typedef struct {
  * Supported (q, k, v, o) dtype tuples: (BF16, BF16, BF16, BF16),
  * (BF16, BF16, E4M3, BF16) ("QK-BF16/PV-FP8", [BW-FP8]),
  * (E4M3, E4M3, E4M3, BF16) ("all-FP8", [BW-FP8]), (INT8, INT8, E4M3, BF16)
- * ("SageAttention", [DiT-Sage]). D must be 64 or 128 (128 for 8-bit Q/K).   */
+ * ("SageAttention", [DiT-Sage]). D must be 64 or 128 (128 for 8-bit Q/K).
+ * Any of these may instead write an E4M3 o (D = 128, not fmha_fwd_decode):
+ * o = E4M3(O / sf_o) rounded to nearest even and saturated to +-448. This is
+ * the FP8 output that [BW-FP8]'s reviewer notes mention, where their shared-
+ * memory-P schedule was limited to 16-bit outputs because of the TMA copy
+ * granularity. Here an E4M3 row of 128 bytes is one TMA box.               */
 typedef struct {
   fmha_tensor q, k, v, o;
   fmha_sf sf_q, sf_k, sf_v, sf_p;
@@ -134,6 +139,9 @@ typedef struct {
                       its own PV product (about 7 significant bits, twice the PV
                       tensor work). Must be 0 or 1 when V is BF16. */
   int32_t reserved; /* must be 0 */
+  fmha_sf sf_o;     /* o of dtype E4M3 only: PER_TENSOR dequantization multiplier
+                       of the output, O ~= code * sf_o[0], or NONE (= 1.0). Must
+                       be NONE for a BF16 o. */
 } fmha_args;
 
 /* Block quantizer: amax -> scale = amax / R -> codes ([DiT-Sage] section 2,

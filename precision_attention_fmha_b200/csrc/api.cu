@@ -275,10 +275,13 @@ fmha_status run_attention(const fmha_args* a, const uint8_t* mask, int64_t msb, 
   else if (dv == FMHA_E4M3) pv = PV_E4M3;
   else return fail(FMHA_ERR_UNSUPPORTED, "V dtype %d unsupported", dv);
   const bool tuple_ok = (qk == QK_BF16) || pv == PV_E4M3;
-  if (!tuple_ok || dout != FMHA_BF16)
+  if (!tuple_ok || (dout != FMHA_BF16 && dout != FMHA_E4M3))
     return fail(FMHA_ERR_UNSUPPORTED, "dtype tuple (q %d, k %d, v %d, o %d) unsupported", dq, dk, dv, dout);
   if (D == 64 && !(qk == QK_BF16 && pv == PV_BF16)) return fail(FMHA_ERR_UNSUPPORTED, "D=64 needs BF16 Q/K/V");
   const bool packed = dec != nullptr;
+  const bool o8 = dout == FMHA_E4M3;
+  if (o8 && D != 128) return fail(FMHA_ERR_UNSUPPORTED, "E4M3 O needs D = 128");
+  if (o8 && packed) return fail(FMHA_ERR_UNSUPPORTED, "decode: O must be BF16");
   const int group = Hq / Hkv;
   int group_shift = 0;
   if (packed) {
@@ -298,6 +301,7 @@ fmha_status run_attention(const fmha_args* a, const uint8_t* mask, int64_t msb, 
   if ((st = check_sf(a->sf_k, "sf_k", q8, q8, q8, 32, false)) != FMHA_OK) return st;
   if ((st = check_sf(a->sf_v, "sf_v", v8, v8, false, 1, v8)) != FMHA_OK) return st;
   if ((st = check_sf(a->sf_p, "sf_p", false, v8, v8, 128, false)) != FMHA_OK) return st;
+  if ((st = check_sf(a->sf_o, "sf_o", false, o8, false, 1, false)) != FMHA_OK) return st;
   if (a->reserved != 0) return fail(FMHA_ERR_INVALID_ARG, "args.reserved must be 0");
   if (a->p_terms < 0 || a->p_terms > 2) return fail(FMHA_ERR_INVALID_ARG, "p_terms must be 0, 1 or 2");
   if (a->p_terms == 2 && !v8) return fail(FMHA_ERR_INVALID_ARG, "p_terms = 2 needs an E4M3 V");
@@ -342,8 +346,9 @@ fmha_status run_attention(const fmha_args* a, const uint8_t* mask, int64_t msb, 
     const uint32_t box[4] = {uint32_t(128 / eqk), 1, 128, 1};
     if ((st = make_map(&tq, a->q.ptr, eqk, dims, strides, box, "q")) != FMHA_OK) return st;
     const int64_t ostr[3] = {a->o.stride_h, a->o.stride_s, a->o.stride_b};
-    const uint32_t obox[4] = {64, 1, 128, 1};
-    if ((st = make_map(&to, a->o.ptr, 2, dims, ostr, obox, "o")) != FMHA_OK) return st;
+    // BF16 O: 64-column (128-byte) boxes; E4M3 O: the whole 128-byte row.
+    const uint32_t obox[4] = {o8 ? 128u : 64u, 1, 128, 1};
+    if ((st = make_map(&to, a->o.ptr, o8 ? 1 : 2, dims, ostr, obox, "o")) != FMHA_OK) return st;
   }
   if (Skv == 0) {  // no key is ever loaded; any valid descriptor will do
     tk = tq;
@@ -386,6 +391,8 @@ fmha_status run_attention(const fmha_args* a, const uint8_t* mask, int64_t msb, 
   p.sf_p_nblk = ceil_div(Sq, p.sf_p_rpb);
   p.lse = a->lse;
   p.p_terms = a->p_terms == 2 ? 2 : 1;
+  p.o8 = o8 ? 1 : 0;
+  p.sf_o = a->sf_o.kind == FMHA_SF_PER_TENSOR ? a->sf_o.ptr : nullptr;
   p.mask = mask; p.mask_sb = msb; p.mask_sh = msh;
   if (paged) {
     p.page_table = pg->page_table; p.num_pages = pg->num_pages; p.page_size = pg->page_size;

@@ -12,9 +12,9 @@ cudaError_t launch_attention_bf16(int D, bool paged, const AttnParams& p, const 
                                   const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& to,
                                   cudaStream_t s) {
   if (D == 128)
-    return paged ? launch_attention_t<AttnCfg<128, QK_BF16, PV_BF16, true>>(p, tq, tk, tv, to, s)
-                 : launch_attention_t<AttnCfg<128, QK_BF16, PV_BF16, false>>(p, tq, tk, tv, to, s);
-  return paged ? launch_attention_t<AttnCfg<64, QK_BF16, PV_BF16, true>>(p, tq, tk, tv, to, s)
-               : launch_attention_t<AttnCfg<64, QK_BF16, PV_BF16, false>>(p, tq, tk, tv, to, s);
+    return paged ? launch_attention_variants<128, QK_BF16, PV_BF16, true>(p, tq, tk, tv, to, s)
+                 : launch_attention_variants<128, QK_BF16, PV_BF16, false>(p, tq, tk, tv, to, s);
+  return paged ? launch_attention_variants<64, QK_BF16, PV_BF16, true>(p, tq, tk, tv, to, s)
+               : launch_attention_variants<64, QK_BF16, PV_BF16, false>(p, tq, tk, tv, to, s);
 }
 }  // namespace fmha

@@ -10,10 +10,7 @@ extern "C" int fmha_trace_read_fp8(void* host, size_t bytes) {
 namespace fmha {
 cudaError_t launch_attention_fp8(int, bool paged, const AttnParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
                                  const CUtensorMap& tv, const CUtensorMap& to, cudaStream_t s) {
-  if (p.p_terms == 2)
-    return paged ? launch_attention_t<AttnCfg<128, QK_E4M3, PV_E4M3, true, true>>(p, tq, tk, tv, to, s)
-                 : launch_attention_t<AttnCfg<128, QK_E4M3, PV_E4M3, false, true>>(p, tq, tk, tv, to, s);
-  return paged ? launch_attention_t<AttnCfg<128, QK_E4M3, PV_E4M3, true>>(p, tq, tk, tv, to, s)
-               : launch_attention_t<AttnCfg<128, QK_E4M3, PV_E4M3, false>>(p, tq, tk, tv, to, s);
+  return paged ? launch_attention_variants<128, QK_E4M3, PV_E4M3, true>(p, tq, tk, tv, to, s)
+               : launch_attention_variants<128, QK_E4M3, PV_E4M3, false>(p, tq, tk, tv, to, s);
 }
 }  // namespace fmha

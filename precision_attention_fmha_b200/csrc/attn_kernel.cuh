@@ -59,7 +59,7 @@ static __device__ unsigned long long g_fmha_trace[FMHA_TRACE_SLOTS];  // one per
 
 namespace fmha {
 
-template <int D_, int QK_, int PV_, bool PAGED_, bool P2_ = false, bool PACKED_ = false>
+template <int D_, int QK_, int PV_, bool PAGED_, bool P2_ = false, bool PACKED_ = false, bool O8_ = false>
 struct AttnCfg {
   static constexpr int D = D_, QK = QK_, PV = PV_;
   static constexpr bool PAGED = PAGED_;
@@ -67,6 +67,9 @@ struct AttnCfg {
   static constexpr bool PACKED = PACKED_;
   static constexpr bool P2 = P2_;  // E4M3 P split into two terms (hi + lo), each with its own PV product
   static_assert(!P2 || PV == PV_E4M3, "two-term P needs an E4M3 V");
+  // E4M3 output: O / sf_o rounded to E4M3 (one 128-byte row per query row).
+  static constexpr bool O8 = O8_;
+  static_assert(!O8 || (D == 128 && !PACKED), "E4M3 O is built for D = 128 tiles");
   static constexpr int BM = 128, BN = 128;
   static constexpr int QK_ELEM = QK == QK_BF16 ? 2 : 1;
   static constexpr int V_ELEM = PV == PV_BF16 ? 2 : 1;
@@ -971,8 +974,50 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, 
   const float inv_l = l > 0.f ? sfv / l : 0.f;
   const uint32_t stage0 = smem_addr(sQx);
   constexpr uint32_t TILE_THREADS = 128 * NH;
+  if constexpr (C::O8) {
+    // E4M3 output: the whole 128-column row is 128 bytes, one swizzled
+    // 128 x 128-byte chunk (the size and layout of a 64-column BF16 chunk),
+    // written by one TMA store. Column c of the row is O[c] / l * sf_v / sf_o.
+    const float inv_lo = inv_l / (p.sf_o != nullptr ? __ldg(p.sf_o) : 1.f);
+    const uint32_t base = stage0 + r * 128;
 #pragma unroll 1
-  for (int c64 = 0; c64 < C::D / 64; ++c64) {
+    for (int sc = 0; sc < C::D / 32; ++sc) {
+      if (sc / OB != h) continue;  // warp-uniform: another thread of this row owns these columns
+      uint32_t o[32];
+      if (have_o) {
+        tmem_ld32(tO + 32 * sc, o);
+        tmem_wait_ld();
+        reg_fence(o);
+      }
+      uint32_t pk[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        float v[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int col = 4 * j + e;
+          v[e] = have_o ? __uint_as_float(o[col]) * inv_lo : 0.f;
+          if (C::PV == PV_E4M3 && p.sf_v_kind == FMHA_SF_PER_CHANNEL) v[e] *= misc->sf_v[32 * sc + col];
+        }
+        pk[j] = pack_e4m3x2(v[0], v[1]) | (pack_e4m3x2(v[2], v[3]) << 16);
+      }
+#pragma unroll
+      for (int kk = 0; kk < 2; ++kk) {
+        const uint32_t addr = base + (((2 * sc + kk) ^ (r & 7)) << 4);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[4 * kk]), "r"(pk[4 * kk + 1]),
+                     "r"(pk[4 * kk + 2]), "r"(pk[4 * kk + 3])
+                     : "memory");
+      }
+    }
+    fence_proxy_async_smem();
+    named_bar_sync(1 + x, TILE_THREADS);
+    if (lead && ok) {
+      tma_store_4d(tmO, stage0, 0, t.h, t.q0, b);
+      bulk_commit();
+    }
+  }
+#pragma unroll 1
+  for (int c64 = 0; c64 < (C::O8 ? 0 : C::D / 64); ++c64) {
     // 32-column blocks of this 64-column chunk held by this thread (its O
     // columns are [32 * OB * h, 32 * OB * (h + 1))); warp-uniform.
     const bool mine[2] = {(2 * c64) / OB == h, (2 * c64 + 1) / OB == h};
@@ -1275,6 +1320,21 @@ cudaError_t launch_attention_t(const AttnParams& p, const CUtensorMap& tq, const
   const long long blocks = static_cast<long long>(p.n_units) * head_units * p.B;
   kern<<<static_cast<unsigned>(blocks), C::THREADS, C::SMEM_BYTES, stream>>>(p, tq, tk, tv, to);
   return cudaGetLastError();
+}
+
+// The two-term-P and E4M3-output variants of one (D, QK, PV, PAGED) kernel.
+template <int D, int QK, int PV, bool PAGED>
+cudaError_t launch_attention_variants(const AttnParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
+                                      const CUtensorMap& tv, const CUtensorMap& to, cudaStream_t s) {
+  if constexpr (PV == PV_E4M3) {
+    if (p.p_terms == 2)
+      return p.o8 ? launch_attention_t<AttnCfg<D, QK, PV, PAGED, true, false, true>>(p, tq, tk, tv, to, s)
+                  : launch_attention_t<AttnCfg<D, QK, PV, PAGED, true>>(p, tq, tk, tv, to, s);
+  }
+  if constexpr (D == 128) {
+    if (p.o8) return launch_attention_t<AttnCfg<D, QK, PV, PAGED, false, false, true>>(p, tq, tk, tv, to, s);
+  }
+  return launch_attention_t<AttnCfg<D, QK, PV, PAGED>>(p, tq, tk, tv, to, s);
 }
 
 }  // namespace fmha

@@ -49,6 +49,8 @@ struct AttnParams {
   // paged K/V (page_table == nullptr: contiguous)
   const int32_t* page_table; int32_t num_pages, page_size, max_pages_per_seq;
   int32_t p_terms;      // 1 or 2 E4M3 terms for P (E4M3 V only)
+  int32_t o8;           // 1: O is written as E4M3(O / sf_o) (D = 128, not packed)
+  const float* sf_o;    // nullable per-tensor output scale (1.0 when NULL)
   // GQA-packed query tiles (decode shapes): row r of a 128-row unit is query
   // token r >> group_shift of head (hkv * group + (r & (group - 1))); n_units
   // then counts pairs of 128-row units of the Sq * group packed rows.

@@ -66,7 +66,12 @@ def _args(D=128, dq=fmha.BF16, dv=fmha.BF16, ptr=0x10000, Hq=4, Hkv=2):
     (lambda a: setattr(a.q, "ptr", 0), 1),
     (lambda a: setattr(a.q, "ptr", 0x10008), 1),
     (lambda a: setattr(a.k, "stride_s", 4 * 128 + 4), 1),
-    (lambda a: setattr(a.o, "dtype", fmha.E4M3), 2),
+    (lambda a: (setattr(a.o, "dtype", fmha.E4M3), setattr(a, "D", 64)), 2),  # E4M3 O needs D = 128
+    (lambda a: setattr(a.o, "dtype", fmha.INT8), 2),
+    (lambda a: (setattr(a.sf_o, "kind", 1), setattr(a.sf_o, "ptr", 0x20000)), 2),  # sf_o with a BF16 O
+    (lambda a: (setattr(a.o, "dtype", fmha.E4M3), setattr(a.sf_o, "kind", 2),
+                setattr(a.sf_o, "ptr", 0x20000)), 2),  # per-head sf_o
+    (lambda a: (setattr(a.o, "dtype", fmha.E4M3), setattr(a.sf_o, "kind", 1)), 1),  # sf_o.ptr NULL
     (lambda a: setattr(a.v, "dtype", fmha.INT8), 2),
     (lambda a: setattr(a.q, "reserved", 1), 1),
     (lambda a: setattr(a.sf_q, "kind", 1), 2),  # scale on a BF16 operand
@@ -117,6 +122,13 @@ def test_nvfp4_argument_checks(lib):
     assert f(src, 64, 4, 64, codes, 32, sb, 3, st, 0, None) == 1       # block-scale row stride
     assert f(None, 64, 4, 64, codes, 32, sb, 4, st, 0, None) == 1      # NULL
     assert f(src, 64, 0, 64, codes, 32, sb, 4, st, 0, None) == 0       # nothing to do
+
+
+def test_decode_rejects_e4m3_output(lib):
+    a = _args()
+    a.B, a.Hq, a.Hkv, a.Sq, a.Skv, a.D = 1, 4, 2, 1, 256, 128
+    a.o.dtype = fmha.E4M3
+    assert lib.fmha_fwd_decode(ctypes.byref(a), None, 0, 0, 0, None, 0, 0, 0, None, 0, None) == 2
 
 
 def test_decode_plan_on_host(lib):
