@@ -37,6 +37,8 @@ WORKLOADS = {
     "dense_pv8_s32768": ("pv8", 1, 40, 40, 32768, 128, False),
     "dense_pv8_s16384": ("pv8", 1, 40, 40, 16384, 128, False),
     "dense_pv8_s4096": ("pv8", 1, 40, 40, 4096, 128, False),
+    # the same with an E4M3 output, O / sf_o with sf_o = V's per-tensor scale (|O| <= max |V|)
+    "dense_pv8_o8_s32768": ("pv8_o8", 1, 40, 40, 32768, 128, False),
     "dense_bf16_s16384": ("bf16", 1, 40, 40, 16384, 128, False),
     "dense_bf16_s4096": ("bf16", 1, 40, 40, 4096, 128, False),
     "tiny_bf16": ("bf16", 1, 1, 1, 256, 64, False),
@@ -48,8 +50,12 @@ WORKLOADS = {
     "decode_paged_s16384": ("decode_paged", 4, 64, 8, 16384, 128, False),
     # per-token NVFP4 quantization of S tokens x D channels (B, H unused)
     "nvfp4_t16384_k4096": ("nvfp4", 1, 1, 1, 16384, 4096, False),
+    # SageAttention K smoothing of the Sage workload's K: token mean per channel + shifted INT8 quantizer
+    "sage_k_smooth_s16384": ("smooth_k", 1, 24, 24, 16384, 128, False),
 }
 DEFAULT_WORKLOAD = "dense_pv8_s32768"
+L2_BYTES = 126 * 2**20          # B200 L2
+L2_FLUSH_BYTES = 512 * 2**20    # written between timed steps when the inputs fit in L2 (~80 us)
 
 
 def load_peaks():
@@ -142,12 +148,12 @@ class Work:
             self.host = dict(zip(("q", "k", "v"), w))
             self.peak, self.peak_note, self.dtype = bf16_peak, "bf16 burst", "bf16"
             self.quant = []
-        elif kind == "pv8":
+        elif kind in ("pv8", "pv8_o8"):
             w = workloads.dense_pv8(S=S, B=B, H=Hq, D=D)
             self.host = {n: w[n] for n in ("q", "k", "v")}
             self.peak = 1.0 / (0.5 / bf16_peak + 0.5 / (2.0 * bf16_peak))
             self.peak_note = f"bf16 burst {bf16_peak} for QK^T, 2x (nominal E4M3 ratio) for PV, time-weighted"
-            self.dtype = "bf16,e4m3"
+            self.dtype = "bf16,e4m3" if kind == "pv8" else "bf16,e4m3,o:e4m3"
             self.quant = [("v", E4, "per_tensor", None)]
         elif kind == "fp8":
             w = workloads.all_fp8(S=S, B=B, H=Hq, D=D)
@@ -173,7 +179,8 @@ class Work:
         self.host = {n: t.contiguous().pin_memory() for n, t in self.host.items()}
         self.dev_in = {n: t.to(dev) for n, t in self.host.items()}
         self.Sq = self.host["q"].shape[1]
-        self.o = torch.empty((B, self.Sq, Hq, D), dtype=torch.bfloat16, device=dev)
+        self.o8 = kind == "pv8_o8"
+        self.o = torch.empty((B, self.Sq, Hq, D), dtype=E4 if self.o8 else torch.bfloat16, device=dev)
         # density = kept score elements / (Sq * Skv)
         self.ws = None
         if kind == "sparse_paged":
@@ -201,6 +208,10 @@ class Work:
             self.qbuf[name] = (torch.empty(x.shape, dtype=dt, device=dev), torch.empty(shp, dtype=torch.float32,
                                device=dev), torch.empty(max(4, fmha.quantize_workspace_bytes(gran, B, S, x.shape[2], D)),
                                                         dtype=torch.uint8, device=dev), gran, rpb, dt)
+        # bytes one step reads: all inputs, or for decode the kept K/V blocks
+        touched = (self.hbm_bytes if kind == "decode_paged"
+                   else sum(t.numel() * t.element_size() for t in self.host.values()))
+        self.fits_l2 = touched <= L2_BYTES
         self.sf_p = None
         self.p_terms = 2 if kind == "sage" else 1  # Sage: P as two E4M3 terms (the tested configuration)
         if kind == "sage":  # per-row-block P scale: P stored as 16 p
@@ -230,15 +241,19 @@ class Work:
         for name, (out, sc, ws, gran, rpb, dt) in self.qbuf.items():
             ops[name] = out
             sfs["sf_" + name] = S_(sc, gran, rpb or 0)
+        if self.o8:  # O is a convex combination of V's rows: V's scale keeps O / sf_o within +-448
+            sfs["sf_o"] = S_(self.qbuf["v"][1], "per_tensor", 0)
         f.fmha_fwd(ops["q"], ops["k"], ops["v"], out=self.o, softmax_scale=self.scale, causal=self.causal,
                    sf_p=self.sf_p, p_terms=self.p_terms, **sfs)
 
     def config(self, world):
-        c = {"workload": self.kind if self.kind != "pv8" else "dense_pv8", "B": self.B, "Hq": self.Hq,
+        c = {"workload": {"pv8": "dense_pv8", "pv8_o8": "dense_pv8_o8"}.get(self.kind, self.kind), "B": self.B,
+             "Hq": self.Hq,
              "Hkv": self.Hkv, "Sq": self.Sq, "Skv": self.S, "D": self.D, "causal": self.causal,
              "density": round(self.density, 6),
              "quantized_in_step": [f"{n}:{g}" for n, _, g, _ in self.quant], "p_terms": self.p_terms,
-             "l2": "inputs larger than L2" if self.host["q"].numel() * 2 > 126 * 2**20 else "inputs fit in L2",
+             "l2": "inputs fit in L2: flushed before each step (512 MiB write, outside the timed events)"
+                   if self.fits_l2 else "inputs larger than L2",
              "parallelism": f"replicas{world}"}
         return c
 
@@ -363,23 +378,18 @@ def run_ours(args):
     time.sleep(0.3)
     barrier(world)
     torch.cuda.synchronize()
-    if W.kind == "decode_paged":
-        # A decode step (~30 us on the GPU) is shorter than the host call that
-        # launches it, so the K steps are captured once in a CUDA graph and the
-        # graph replay is timed: device time with no host gaps.
-        graph = torch.cuda.CUDAGraph()
-        side = torch.cuda.Stream()
-        side.wait_stream(stream)
-        with torch.cuda.stream(side):
-            with torch.cuda.graph(graph, stream=side):
-                for i in range(K):
-                    W.attn(W.dev_in)
-        stream.wait_stream(side)
-        graph.replay()
-        torch.cuda.synchronize()
-        t0.record(stream)
-        graph.replay()
-        t1.record(stream)
+    if W.fits_l2:
+        # The inputs fit in L2: each step is timed alone, after a write of
+        # twice the L2 size that evicts them (outside the step's events). The
+        # flush kernel is still running when the step is queued behind it, so
+        # no host launch gap falls inside the events.
+        flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        for i in range(K):
+            flush.zero_()
+            attn_ev[i][0].record(stream)
+            W.prep(W.dev_in)
+            W.attn(W.dev_in)
+            attn_ev[i][1].record(stream)
     else:
         t0.record(stream)
         for i in range(K):
@@ -392,8 +402,11 @@ def run_ours(args):
     barrier(world)
     clk = clocks.stop()
     fmha.get_device_error()
-    ms = t0.elapsed_time(t1) / K
-    attn_ms = ms if W.kind == "decode_paged" else statistics.mean(a.elapsed_time(b) for a, b in attn_ev)
+    if W.fits_l2:  # prep + attention between each step's events
+        ms = attn_ms = statistics.mean(a.elapsed_time(b) for a, b in attn_ev)
+    else:
+        ms = t0.elapsed_time(t1) / K
+        attn_ms = statistics.mean(a.elapsed_time(b) for a, b in attn_ev)
     ms = max_over_ranks(ms, world)
     attn_ms = max_over_ranks(attn_ms, world)
 
@@ -485,7 +498,7 @@ def oracle_sample(host, kind, B, Hq, Hkv, S, D, causal, rows):
         q32 = host["q"][:1, :rows, :1].to(torch.float32).numpy()
         k32 = host["k"][:1, :, :1].to(torch.float32).numpy()
         v32 = host["v"][:1, :, :1].to(torch.float32).numpy()
-        spec = {"bf16": {}, "pv8": {"v": ("e4m3", "per_tensor", None)},
+        spec = {"bf16": {}, "pv8": {"v": ("e4m3", "per_tensor", None)}, "pv8_o8": {"v": ("e4m3", "per_tensor", None)},
                 "fp8": {n: ("e4m3", "per_head", None) for n in "qkv"},
                 "sage": {"q": ("int8", "per_token_block", 128), "k": ("int8", "per_token_block", 64),
                          "v": ("e4m3", "per_channel", None)}}[kind]
@@ -529,6 +542,7 @@ def run_reference(args):
     kind, B, Hq, Hkv, S, D, causal = WORKLOADS[args.workload]
     gen = {"bf16": lambda: dict(zip("qkv", workloads.normal_qkv(workloads.SEED_BASE + 1 + S, B, S, S, Hq, Hkv, D))),
            "pv8": lambda: workloads.dense_pv8(S=S, B=B, H=Hq, D=D),
+           "pv8_o8": lambda: workloads.dense_pv8(S=S, B=B, H=Hq, D=D),
            "fp8": lambda: workloads.all_fp8(S=S, B=B, H=Hq, D=D),
            "sage": lambda: workloads.sage(S=S, B=B, H=Hq, D=D),
            "sparse_paged": lambda: workloads.sparse_paged(S=S, B=B, Hq=Hq, Hkv=Hkv, D=D),
@@ -555,6 +569,136 @@ def run_reference(args):
         "e2e": {"value": round(val, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
+
+
+def run_smooth(args):
+    """SageAttention K smoothing of the Sage workload's K: channel mean + shifted INT8 quantizer. HBM-bound."""
+    from precision_attention_fmha_b200 import fmha, workloads
+
+    world, rank, local = dist_setup(args.gpus)
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    _, B, H, _, S, D, _ = WORKLOADS[args.workload]
+    kh = workloads.sage(S=S, B=B, H=H, D=D)["k"].contiguous().pin_memory()
+    k = kh.to(dev)
+    mean = torch.empty((B, H, D), dtype=torch.float32, device=dev)
+    mws = torch.empty(max(16, fmha.channel_mean_workspace_bytes(B, S, H, D)), dtype=torch.uint8, device=dev)
+    codes = torch.empty(k.shape, dtype=torch.int8, device=dev)
+    scales = torch.empty(fmha.scale_shape("per_token_block", B, S, H, D, 64), dtype=torch.float32, device=dev)
+
+    def step(inp):
+        fmha.channel_mean(inp, out=mean, workspace=mws)
+        fmha.fmha_quantize_blockwise(inp, torch.int8, "per_token_block", 64, out=codes, scales=scales, shift=mean)
+
+    for _ in range(args.warmup):
+        step(k)
+    fmha.get_device_error()
+    K_ = args.steps
+    stream = torch.cuda.current_stream()
+    fits_l2 = k.numel() * 2 <= L2_BYTES
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev) if fits_l2 else None
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K_)]
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    for i in range(K_):  # each step alone, L2 flushed before it when K fits there
+        if flush is not None:
+            flush.zero_()
+        evs[i][0].record(stream)
+        step(k)
+        evs[i][1].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in evs), world)
+    # mean: K read once; quantizer: K read once, codes + scales written; mean written once
+    out_bytes = codes.numel() + scales.numel() * 4 + mean.numel() * 4
+    algo = 2 * k.numel() * 2 + out_bytes
+    _, hbm, src = load_peaks()
+    gbs = algo / (ms * 1e-3) / 1e9
+    oh = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (codes, scales, mean)]
+    Ke = max(1, min(K_, 10))
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(Ke):
+        step(kh.to(dev, non_blocking=True))
+        for h, d in zip(oh, (codes, scales, mean)):
+            h.copy_(d, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / Ke, world)
+    fmha.get_device_error()
+    line = {
+        "metric": "K smoothing GB/s (token mean per channel + INT8 quantization of K - mean: 4 B read + 1 B written "
+                  "per element)",
+        "value": round(world * gbs, 1), "unit": "GB/s", "n_gpus": world, "steps": K_, "warmup": args.warmup,
+        "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16->int8", "data": "synthetic (seeded; the Sage workload's K, N(0,1) + per-channel N(0,2) bias)",
+        "config": {"workload": "sage_k_smooth", "B": B, "H": H, "S": S, "D": D, "k_scale": "per 64-token block",
+                   "l2": "inputs fit in L2: flushed before each step (512 MiB write, outside the timed events)"
+                   if fits_l2 else "inputs larger than L2",
+                   "parallelism": f"replicas{world}"},
+        "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": round(hbm, 1), "unit": "GB/s",
+                     "frac": round(gbs / hbm, 4), "traffic": None, "peak_note": f"{src}: HBM copy bandwidth",
+                     "algorithmic_bytes": int(algo),
+                     "kernel": "channel_mean_partial_kernel + channel_mean_final_kernel + quant_token_block_kernel",
+                     "kernel_ms": round(ms, 5)},
+        "e2e": {"value": round(world * algo / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
+                "h2d_bytes_per_step": k.numel() * 2, "d2h_bytes_per_step": out_bytes, "steps": Ke},
+        "gpu_launches": 3 * K_,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        dt, nbytes = smooth_oracle_sample(kh, heads=2)
+        line["cpu_baseline"] = {"value": round(nbytes / dt / 1e9, 6), "unit": "GB/s", "cores": cpu_cores(),
+                                "kind": "oracle", "sample": f"heads 0..1 of {H}, NumPy oracle, {dt:.2f} s"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    teardown(world)
+
+
+def smooth_oracle_sample(kh, heads):
+    """The oracle's channel mean + shifted quantizer on the first `heads` heads: (seconds, algorithmic bytes)."""
+    from oracle import quant as oq
+
+    x = kh[:, :, :heads].to(torch.float32).numpy()
+    t = time.perf_counter()
+    mu = oq.channel_mean(x)
+    oq.quantize_blockwise(x, "int8", "per_token_block", 64, shift=mu)
+    dt = time.perf_counter() - t
+    return dt, x.size * 5
+
+
+def run_reference_smooth(args):
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    from precision_attention_fmha_b200 import workloads
+
+    _, B, H, _, S, D, _ = WORKLOADS[args.workload]
+    kh = workloads.sage(S=S, B=B, H=H, D=D)["k"].contiguous()
+    heads = 2  # a bounded sample of the H heads per step
+    for _ in range(args.warmup):
+        smooth_oracle_sample(kh, heads)
+    times, nbytes = [], 0
+    for _ in range(args.steps):
+        dt, nbytes = smooth_oracle_sample(kh, heads)
+        times.append(dt)
+    ms = 1e3 * sum(times) / len(times)
+    val = nbytes / (ms * 1e-3) / 1e9
+    print(json.dumps({
+        "impl": "reference", "metric": "K smoothing GB/s (token mean per channel + INT8 quantization of K - mean: "
+                                       "4 B read + 1 B written per element)",
+        "value": round(val, 6), "unit": "GB/s", "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded; the Sage workload's K)",
+        "config": {"workload": args.workload, "B": B, "H": H, "S": S, "D": D},
+        "cpu_baseline": {"value": round(val, 6), "unit": "GB/s", "cores": cpu_cores(), "kind": "oracle",
+                         "sample": f"heads 0..{heads - 1} of {H} per step, NumPy oracle"},
+        "e2e": {"value": round(val, 6), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}), flush=True)
 
 
 def run_reference_nvfp4(args):
@@ -636,11 +780,11 @@ def main():
         return
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
-    nvfp4 = WORKLOADS[args.workload][0] == "nvfp4"
+    kind = WORKLOADS[args.workload][0]
     if args.impl == "reference":
-        run_reference_nvfp4(args) if nvfp4 else run_reference(args)
+        {"nvfp4": run_reference_nvfp4, "smooth_k": run_reference_smooth}.get(kind, run_reference)(args)
     else:
-        run_nvfp4(args) if nvfp4 else run_ours(args)
+        {"nvfp4": run_nvfp4, "smooth_k": run_smooth}.get(kind, run_ours)(args)
 
 
 if __name__ == "__main__":

@@ -450,8 +450,9 @@ fmha_status run_attention(const fmha_args* a, const uint8_t* mask, int64_t msb, 
   return ok_status();
 }
 
-// Token rows one CTA of the channel-mean kernel sums: 16 KB of BF16 input.
-int mean_rows_per_cta(int D) { return D >= 8 ? (2048 / (D / 8) > 0 ? 2048 / (D / 8) : 1) : 1; }
+// Token rows one CTA of the channel-mean kernel sums: 128 KB of BF16 input
+// (few partials for the final sum; still several CTAs per SM at 16 K tokens).
+int mean_rows_per_cta(int D) { return D >= 8 ? 65536 / D : 1; }
 
 fmha_status quantize_impl(const fmha_tensor* src, const float* shift, const fmha_tensor* dst, const fmha_sf* sf,
                           int32_t B, int32_t S, int32_t H, int32_t D, void* workspace, size_t workspace_bytes,

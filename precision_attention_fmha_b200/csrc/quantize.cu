@@ -292,7 +292,7 @@ __global__ void __launch_bounds__(kThreads) channel_mean_partial_kernel(const Qu
   const int cv = threadIdx.x % vpr, row_step = kThreads / vpr;
   const uint16_t* src = p.src + b * p.s_sb + static_cast<int64_t>(s0) * p.s_ss + h * p.s_sh + cv * 8;
   double acc[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
-#pragma unroll 4
+#pragma unroll 8
   for (int r = threadIdx.x / vpr; r < rows; r += row_step) {
     float x[8];
     unpack8(ld16(src + r * p.s_ss), x);
@@ -319,6 +319,7 @@ __global__ void __launch_bounds__(kThreads) channel_mean_final_kernel(const Quan
   const int64_t bh = i / p.D, ch = i - bh * p.D;
   const double* part = p.partial + bh * p.n_chunks * p.D + ch;
   double a = 0.0;
+#pragma unroll 8
   for (int c = 0; c < p.n_chunks; ++c) a += part[static_cast<int64_t>(c) * p.D];
   p.mean[i] = __double2float_rn(__ddiv_rn(a, static_cast<double>(p.S)));
 }

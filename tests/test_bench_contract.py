@@ -36,8 +36,13 @@ def test_nvfp4_reference_arm_line():
     assert d["impl"] == "reference" and d["unit"] == "GB/s" and d["value"] > 0
 
 
+def test_smooth_reference_arm_line():
+    d = run_bench("--impl", "reference", "--workload", "sage_k_smooth_s16384", "--steps", "1", "--warmup", "1")
+    assert d["impl"] == "reference" and d["unit"] == "GB/s" and d["value"] > 0
+
+
 @pytest.mark.gpu
-@pytest.mark.parametrize("workload", ["tiny_bf16", "decode_paged_s16384"])
+@pytest.mark.parametrize("workload", ["tiny_bf16", "decode_paged_s16384", "sage_k_smooth_s16384"])
 def test_our_arm_line(workload):
     d = run_bench("--workload", workload, "--steps", "3", "--warmup", "3")
     for k in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
