@@ -765,6 +765,66 @@ def probe_peaks():
     print(json.dumps({"probe": "library GEMM peaks, 8192^3, TFLOP/s (TOP/s for int8)", **out}), flush=True)
 
 
+def quant_probe(capture=False):
+    """Block-quantizer calls on the Sage workload's K and Q (B1 H24 S16384 D128),
+    each timed alone after an L2 flush: INT8 / E4M3 per 64-token block, INT8 per
+    64-token block with the K-smoothing shift, INT8 per 128-token block, and the
+    channel mean. With capture=True it makes only two calls, INT8 per 64-token
+    block without and then with the shift (a short program for ncu)."""
+    from precision_attention_fmha_b200 import fmha, workloads
+
+    dev = torch.device("cuda")
+    w = workloads.sage()
+    k = w["k"].to(dev)
+    B, S, H, D = k.shape
+    mean = torch.empty((B, H, D), dtype=torch.float32, device=dev)
+    ws = torch.empty(max(16, fmha.channel_mean_workspace_bytes(B, S, H, D)), dtype=torch.uint8, device=dev)
+    codes = torch.empty(k.shape, dtype=torch.int8, device=dev)
+    sc64 = torch.empty(fmha.scale_shape("per_token_block", B, S, H, D, 64), dtype=torch.float32, device=dev)
+    fmha.channel_mean(k, out=mean, workspace=ws)
+    if capture:
+        fmha.fmha_quantize_blockwise(k, torch.int8, "per_token_block", 64, out=codes, scales=sc64)
+        fmha.fmha_quantize_blockwise(k, torch.int8, "per_token_block", 64, out=codes, scales=sc64, shift=mean)
+        torch.cuda.synchronize()
+        fmha.get_device_error()
+        return
+    q = w["q"].to(dev)
+    codes_e = torch.empty(k.shape, dtype=torch.float8_e4m3fn, device=dev)
+    sc128 = torch.empty(fmha.scale_shape("per_token_block", B, S, H, D, 128), dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def timed(fn, n=20):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        total = 0.0
+        for _ in range(n):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            total += a.elapsed_time(b)
+        return round(total / n * 1000, 2)
+
+    res = {
+        "probe": "block quantizer on the Sage workload's K / Q, us per call, L2 flushed before each",
+        "channel_mean": timed(lambda: fmha.channel_mean(k, out=mean, workspace=ws)),
+        "int8_per64": timed(lambda: fmha.fmha_quantize_blockwise(k, torch.int8, "per_token_block", 64, out=codes,
+                                                                scales=sc64)),
+        "int8_per64_shift": timed(lambda: fmha.fmha_quantize_blockwise(k, torch.int8, "per_token_block", 64,
+                                                                      out=codes, scales=sc64, shift=mean)),
+        "e4m3_per64": timed(lambda: fmha.fmha_quantize_blockwise(k, torch.float8_e4m3fn, "per_token_block", 64,
+                                                                out=codes_e, scales=sc64)),
+        "int8_per128_q": timed(lambda: fmha.fmha_quantize_blockwise(q, torch.int8, "per_token_block", 128,
+                                                                   out=codes, scales=sc128)),
+        "algorithmic_bytes_per_call": k.numel() * 3,
+    }
+    fmha.get_device_error()
+    print(json.dumps(res), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -774,9 +834,14 @@ def main():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--probe-peaks", action="store_true", help="print library GEMM peaks (bf16, E4M3, INT8) and exit")
+    ap.add_argument("--quant-probe", choices=["time", "capture"],
+                    help="time the block quantizer on the Sage workload's K / Q ('capture': two calls, for ncu)")
     args = ap.parse_args()
     if args.probe_peaks:
         probe_peaks()
+        return
+    if args.quant_probe:
+        quant_probe(capture=args.quant_probe == "capture")
         return
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
