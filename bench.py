@@ -21,6 +21,7 @@ import math
 import os
 import statistics
 import subprocess
+import tempfile
 import sys
 import time
 
@@ -82,7 +83,9 @@ class ClockSampler:
     def __init__(self, gpu_index):
         self.gpu_index = gpu_index
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_bench_{os.getpid()}.csv")
+        # raw samples go to a scratch file (set CLOCKS_CSV_DIR to keep them); the summary is in the JSON line
+        self.path = os.path.join(os.environ.get("CLOCKS_CSV_DIR") or tempfile.gettempdir(),
+                                 f"clocks_bench_{os.getpid()}.csv")
 
     def start(self):
         try:

@@ -27,10 +27,11 @@
 // tile's S columns are free once the softmax has loaded them: QK^T of the next
 // KV tile overlaps the softmax, and the two softmax warpgroups take turns in
 // their exp2 phases.
-// The epilogue scales O by 1/l (and the V / P scale factors), converts to BF16,
-// stages 64-column halves in the dead Q buffer and writes them with TMA stores
-// ("FlashInfer DeepSeek-V4 sparse-MLA: Cake backend", section 1: output through
-// a TMA descriptor passed as a grid constant).
+// The epilogue scales O by 1/l (and the V / P scale factors), converts to BF16
+// (64-column halves) or E4M3 (O / sf_o, one 128-byte row per query row), stages
+// the result in the dead Q buffer and writes it with TMA stores ("FlashInfer
+// DeepSeek-V4 sparse-MLA: Cake backend", section 1: output through a TMA
+// descriptor passed as a grid constant).
 //
 // Every wait is bounded: on expiry the thread sets the device error word and a
 // CTA-wide abort flag; all roles then fall through to a teardown that drains
