@@ -33,7 +33,10 @@ namespace fmha {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kCacheVecs = 8;  // 8 x 16 B per thread: a 128 x 128 bf16 block stays in registers
+// 16-byte vectors a thread keeps in registers between the amax and the code
+// pass: 8 hold a 128 x 128 BF16 block, 4 a 64 x 128 block. The smaller cache
+// lets four CTAs share an SM's registers (more loads in flight).
+constexpr int kCacheVecsMax = 8;
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
@@ -117,8 +120,8 @@ __device__ __forceinline__ float block_reduce_max(float v, float* red) {
 }
 
 // One CTA per (token block, h, b).
-template <bool kE4M3>
-__global__ void __launch_bounds__(kThreads) quant_token_block_kernel(const QuantParams p) {
+template <bool kE4M3, int kCacheVecs>
+__global__ void __launch_bounds__(kThreads, kCacheVecs <= 4 ? 4 : 0) quant_token_block_kernel(const QuantParams p) {
   __shared__ float red[kThreads / 32];
   const int blk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int s0 = blk * p.rpb;
@@ -264,7 +267,10 @@ template <bool kE4M3>
 cudaError_t launch_quantize_t(const QuantParams& p, cudaStream_t stream) {
   if (p.kind == FMHA_SF_PER_TOKEN_BLOCK) {
     dim3 grid(p.nblk, p.H, p.B);
-    quant_token_block_kernel<kE4M3><<<grid, kThreads, 0, stream>>>(p);
+    if (static_cast<int64_t>(p.rpb) * (p.D >> 3) <= 4 * kThreads)
+      quant_token_block_kernel<kE4M3, 4><<<grid, kThreads, 0, stream>>>(p);
+    else
+      quant_token_block_kernel<kE4M3, kCacheVecsMax><<<grid, kThreads, 0, stream>>>(p);
     return cudaGetLastError();
   }
   const size_t groups = p.kind == FMHA_SF_PER_CHANNEL ? static_cast<size_t>(p.B) * p.H * p.D
