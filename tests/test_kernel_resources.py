@@ -1,0 +1,78 @@
+"""Register and spill budgets of the kernels, from ptxas's resource report (CPU only).
+
+The occupancy the kernels are designed for depends on these numbers:
+
+* the token-block quantizer's 4-vector variant (64 x 128 blocks) must fit in
+  64 registers, so that 4 CTAs of 256 threads share an SM's 65,536 registers;
+* the channel-mean kernels must not spill;
+* the attention kernel runs 384 threads per CTA, one CTA per SM, and its
+  setmaxnreg split assumes a launch of at most 168 registers per thread
+  (384 x 168 = 64,512). Its spills must stay a few bytes.
+
+nvcc compiles for sm_100a without a GPU. Only ptxas's printed summary
+(`-Xptxas -v`) is read.
+"""
+
+import os
+import re
+import subprocess
+
+import pytest
+
+from precision_attention_fmha_b200 import build as build_mod
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+CSRC = os.path.join(ROOT, "precision_attention_fmha_b200", "csrc")
+
+
+def resources(src, tmp_path):
+    cmd = [build_mod.nvcc()] + build_mod.ARCH + [f for f in build_mod.FLAGS] + [
+        "-c", os.path.join(CSRC, src), "-o", str(tmp_path / (src + ".o"))]
+    r = subprocess.run(cmd, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    out = {}
+    name = None
+    for line in (r.stdout + r.stderr).splitlines():
+        m = re.search(r"Compiling entry function '([^']+)'", line)
+        if m:
+            name = m.group(1)
+            out[name] = {"regs": None, "spill_st": 0, "spill_ld": 0}
+            continue
+        if name is None:
+            continue
+        m = re.search(r"(\d+) bytes spill stores, (\d+) bytes spill loads", line)
+        if m:
+            out[name]["spill_st"], out[name]["spill_ld"] = int(m.group(1)), int(m.group(2))
+        m = re.search(r"Used (\d+) registers", line)
+        if m:
+            out[name]["regs"] = int(m.group(1))
+    return out
+
+
+@pytest.fixture(scope="module")
+def quant_res(tmp_path_factory):
+    return resources("quantize.cu", tmp_path_factory.mktemp("ptxas"))
+
+
+def test_token_block_quantizer_small_cache_fits_four_ctas(quant_res):
+    small = {n: r for n, r in quant_res.items() if re.search(r"quant_token_block_kernelILb[01]ELi4E", n)}
+    assert len(small) == 2, sorted(quant_res)  # INT8 and E4M3
+    for n, r in small.items():
+        assert r["regs"] is not None and r["regs"] <= 64, (n, r)
+        assert r["spill_st"] == 0 and r["spill_ld"] == 0, (n, r)
+
+
+def test_quantizer_and_mean_kernels_do_not_spill(quant_res):
+    assert any("channel_mean_partial_kernel" in n for n in quant_res)
+    assert any("channel_mean_final_kernel" in n for n in quant_res)
+    for n, r in quant_res.items():
+        assert r["spill_st"] == 0 and r["spill_ld"] == 0, (n, r)
+
+
+def test_attention_kernel_register_budget(tmp_path):
+    res = resources("attn_pv8.cu", tmp_path)
+    attn = {n: r for n, r in res.items() if "attn_fwd_kernel" in n}
+    assert len(attn) >= 4
+    for n, r in attn.items():
+        assert r["regs"] is not None and r["regs"] <= 168, (n, r)
+        assert r["spill_st"] <= 64 and r["spill_ld"] <= 64, (n, r)
