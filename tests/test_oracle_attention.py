@@ -67,6 +67,21 @@ def test_brute_force_tiny(causal, Sq, Skv):
         assert np.allclose(lse[fin], lseb[fin], atol=1e-12)
 
 
+@pytest.mark.parametrize("causal", [False, True])
+def test_brute_force_qk_dim_differs_from_v_dim(causal):
+    # The QK head dim and the V head dim are separate (192 / 128 in the wider
+    # head-dim variant, 12 / 8 here): O takes V's width, scores sum over QK's.
+    rng = np.random.default_rng(31)
+    B, Sq, Skv, Hq, Hkv, Dqk, Dv = 1, 9, 13, 4, 2, 12, 8
+    q, k, v = _rand(rng, B, Sq, Hq, Dqk), _rand(rng, B, Skv, Hkv, Dqk), _rand(rng, B, Skv, Hkv, Dv)
+    o, lse = A.attention(q, k, v, 1 / math.sqrt(Dqk), causal)
+    ob, lseb = _brute(q, k, v, 1 / math.sqrt(Dqk), causal, None, 4)
+    assert o.shape == (B, Sq, Hq, Dv)
+    assert np.allclose(o, ob, atol=1e-13, rtol=1e-12)
+    fin = np.isfinite(lseb)
+    assert np.allclose(lse[fin], lseb[fin], atol=1e-12)
+
+
 def test_two_key_closed_form():
     q = np.array([1.0, 0.0]).reshape(1, 1, 1, 2)
     k = np.array([[1.0, 0.0], [0.0, 1.0]]).reshape(1, 2, 1, 2)
