@@ -16,6 +16,7 @@ import pytest
 import torch
 
 from oracle import attention as oa
+from oracle import e4m3 as oe
 from oracle import quant as oq
 from precision_attention_fmha_b200 import fmha, workloads
 from precision_attention_fmha_b200.fmha import Scale
@@ -49,11 +50,20 @@ def oracle_head(x_bf16, b, h, spec, full_x=None):
     return deq[0, :, 0], codes[0, :, 0]
 
 
-def check_rows(mode, got_rows, ref_rows):
-    """got/ref: dict (b, h) -> [n, D] arrays."""
+def check_rows(mode, got_rows, ref_rows, sf_o=None):
+    """got/ref: dict (b, h) -> [n, D] arrays. sf_o: the output scale of an E4M3
+    output, whose rounding (2^-4 relative, 2^-10 sf_o absolute) adds to the
+    8-bit tolerance, with cos >= 0.998."""
     for key in ref_rows:
         g, r = got_rows[key], ref_rows[key]
         assert np.all(np.isfinite(g)), f"non-finite output at {key}"
+        if sf_o is not None:
+            bound = 2.0 ** -4 * np.abs(r) + 2.0 ** -10 * sf_o + Q8_ATOL * max(1.0, np.abs(r).max())
+            worst = np.argmax(np.abs(g - r) - bound)
+            assert np.all(np.abs(g - r) <= bound), f"{key}: err {np.abs(g - r).flat[worst]:.3e}"
+            c = cos_per_head(g[None, :, None, :], r[None, :, None, :])[0]
+            assert c >= 0.998, f"{key}: cos {c:.6f}"
+            continue
         err = np.abs(g - r).max()
         if mode == "bf16":
             assert err <= BF16_ATOL, f"{key}: max-abs {err:.3e}"
@@ -64,8 +74,9 @@ def check_rows(mode, got_rows, ref_rows):
             assert c >= Q8_COS, f"{key}: cos {c:.6f}"
 
 
-def run_case(mode, q, k, v, specs, heads, causal=False, sf_p=None, p_terms=1):
-    """Quantize on the GPU exactly as bench.py does, run attention, compare sampled rows."""
+def run_case(mode, q, k, v, specs, heads, causal=False, sf_p=None, p_terms=1, o8=False):
+    """Quantize on the GPU exactly as bench.py does, run attention, compare sampled rows.
+    o8: E4M3 output with V's per-tensor scale as sf_o (bench.py's E4M3-output workload)."""
     B, Sq, Hq, D = q.shape
     Skv = k.shape[1]
     group = Hq // k.shape[2]
@@ -75,8 +86,13 @@ def run_case(mode, q, k, v, specs, heads, causal=False, sf_p=None, p_terms=1):
         out, kind, rpb = spec
         c, sc = fmha.fmha_quantize_blockwise(ops[name], TDT[out], kind, rpb)
         ops[name], sfs["sf_" + name] = c, Scale(sc, kind, rpb or 0)
+    extra, sf_o = {}, None
+    if o8:
+        extra = {"out": torch.empty((B, Sq, Hq, v.shape[3]), dtype=torch.float8_e4m3fn, device=DEV),
+                 "sf_o": sfs["sf_v"]}
+        sf_o = float(sfs["sf_v"].tensor.reshape(-1)[0].item())
     o = fmha.fmha_fwd(ops["q"], ops["k"], ops["v"], softmax_scale=1 / math.sqrt(D), causal=causal, sf_p=sf_p,
-                      p_terms=p_terms, **sfs)
+                      p_terms=p_terms, **sfs, **extra)
     fmha.get_device_error()
     got, ref = {}, {}
     for (b, h) in heads:
@@ -92,14 +108,22 @@ def run_case(mode, q, k, v, specs, heads, causal=False, sf_p=None, p_terms=1):
         rows = sample_rows(Sq, seed=b * 131 + h)
         ro, _ = oa.attention_rows(opr["q"][rows], rows, opr["k"], opr["v"], 1 / math.sqrt(D), Sq, causal)
         ref[(b, h)] = ro
-        got[(b, h)] = f64(o[b, rows, h, :])
-    check_rows(mode, got, ref)
+        if o8:
+            got[(b, h)] = oe.decode(o.view(torch.uint8)[b, rows, h, :].cpu().numpy()) * sf_o
+        else:
+            got[(b, h)] = f64(o[b, rows, h, :])
+    check_rows(mode, got, ref, sf_o)
 
 
 @pytest.mark.parametrize("S", [4096, 16384, 32768])
 def test_dense_pv8_full_size(S):
     w = workloads.dense_pv8(S=S)
     run_case("pv8", w["q"], w["k"], w["v"], {"v": ("e4m3", "per_tensor", None)}, heads=[(0, 0), (0, 17), (0, 39)])
+
+
+def test_dense_pv8_e4m3_output_full_size():
+    w = workloads.dense_pv8(S=32768)
+    run_case("pv8", w["q"], w["k"], w["v"], {"v": ("e4m3", "per_tensor", None)}, heads=[(0, 0), (0, 39)], o8=True)
 
 
 @pytest.mark.parametrize("causal", [False, True])
