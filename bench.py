@@ -47,6 +47,8 @@ WORKLOADS = {
     "all_fp8_s8192_causal": ("fp8", 2, 32, 32, 8192, 128, True),
     "sage_s16384": ("sage", 1, 24, 24, 16384, 128, False),
     "sparse_paged_s16384": ("sparse_paged", 4, 64, 8, 16384, 128, False),
+    # the same mask, Q and K/V values with K/V contiguous [B, S, Hkv, D] (the paged-overhead control)
+    "sparse_contig_s16384": ("sparse_contig", 4, 64, 8, 16384, 128, False),
     # decode step: one query token per sequence against S cached tokens (S is Skv)
     "decode_paged_s16384": ("decode_paged", 4, 64, 8, 16384, 128, False),
     # per-token NVFP4 quantization of S tokens x D channels (B, H unused)
@@ -141,6 +143,7 @@ class Work:
 
     def __init__(self, name, dev, fmha, workloads, Scale):
         kind, B, Hq, Hkv, S, D, causal = WORKLOADS[name]
+        self.name = name
         self.kind, self.B, self.Hq, self.Hkv, self.S, self.D, self.causal = kind, B, Hq, Hkv, S, D, causal
         self.dev, self.fmha, self.Scale = dev, fmha, Scale
         bf16_peak, _, src = load_peaks()
@@ -178,6 +181,11 @@ class Work:
                          "mask": w["mask"]}
             self.peak, self.peak_note, self.dtype = bf16_peak, "bf16 burst", "bf16"
             self.quant = []
+        elif kind == "sparse_contig":
+            w = workloads.sparse_paged(S=S, B=B, Hq=Hq, Hkv=Hkv, D=D)
+            self.host = {"q": w["q"], "k": w["k"], "v": w["v"], "mask": w["mask"]}
+            self.peak, self.peak_note, self.dtype = bf16_peak, "bf16 burst", "bf16"
+            self.quant = []
         self.scale = 1.0 / math.sqrt(D)
         self.host = {n: t.contiguous().pin_memory() for n, t in self.host.items()}
         self.dev_in = {n: t.to(dev) for n, t in self.host.items()}
@@ -186,7 +194,7 @@ class Work:
         self.o = torch.empty((B, self.Sq, Hq, D), dtype=E4 if self.o8 else torch.bfloat16, device=dev)
         # density = kept score elements / (Sq * Skv)
         self.ws = None
-        if kind == "sparse_paged":
+        if kind in ("sparse_paged", "sparse_contig"):
             kept = float(self.host["mask"].to(torch.float64).sum())
             self.density = kept * 128 * 128 / (B * Hkv * S * S)
             self.flop = 4.0 * B * Hq * S * S * D * self.density
@@ -235,6 +243,9 @@ class Work:
             f.fmha_fwd_paged(inp["q"], inp["k_pool"], inp["v_pool"], inp["page_table"], self.S, mask=inp["mask"],
                              out=self.o, softmax_scale=self.scale)
             return
+        if self.kind == "sparse_contig":
+            f.fmha_fwd_block_sparse(inp["q"], inp["k"], inp["v"], inp["mask"], out=self.o, softmax_scale=self.scale)
+            return
         if self.kind == "decode_paged":
             f.fmha_fwd_decode(inp["q"], inp["k_pool"], inp["v_pool"], page_table=inp["page_table"], Skv=self.S,
                               mask=inp["mask"], workspace=self.ws, out=self.o, softmax_scale=self.scale)
@@ -250,7 +261,7 @@ class Work:
                    sf_p=self.sf_p, p_terms=self.p_terms, **sfs)
 
     def config(self, world):
-        c = {"workload": {"pv8": "dense_pv8", "pv8_o8": "dense_pv8_o8"}.get(self.kind, self.kind), "B": self.B,
+        c = {"workload": self.name, "B": self.B,
              "Hq": self.Hq,
              "Hkv": self.Hkv, "Sq": self.Sq, "Skv": self.S, "D": self.D, "causal": self.causal,
              "density": round(self.density, 6),
@@ -332,7 +343,7 @@ def run_nvfp4(args):
         "value": round(world * gbs, 1), "unit": "GB/s", "n_gpus": world, "steps": K_, "warmup": args.warmup,
         "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16->e2m1", "data": "synthetic (seeded N(0,1), BF16)",
-        "config": {"workload": "nvfp4_per_token", "tokens": T, "K": K, "l2": "inputs fit in L2" if x.numel() * 2 <= 126 * 2**20
+        "config": {"workload": args.workload, "tokens": T, "K": K, "l2": "inputs fit in L2" if x.numel() * 2 <= 126 * 2**20
                    else "inputs larger than L2", "parallelism": f"replicas{world}"},
         "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": round(hbm, 1), "unit": "GB/s",
                      "frac": round(gbs / hbm, 4), "traffic": None, "peak_note": f"{src}: HBM copy bandwidth",
@@ -490,7 +501,13 @@ def oracle_sample(host, kind, B, Hq, Hkv, S, D, causal, rows):
         oa.attention(q, k, v, 1.0 / math.sqrt(D), False, mask)
         dt = time.perf_counter() - t0 + t
         return dt, 4.0 * q.shape[0] * q.shape[1] * G * float(mask.sum()) / q.shape[0] * 128 * D
-    if kind == "sparse_paged":
+    if kind == "sparse_contig":
+        k = host["k"][:1, :, :1].to(torch.float64).numpy()
+        v = host["v"][:1, :, :1].to(torch.float64).numpy()
+        q = host["q"][:1, :rows, :1].to(torch.float64).numpy()
+        mask = host["mask"][:1, :1].numpy()
+        mask = mask[:, :, : -(-rows // 128)]
+    elif kind == "sparse_paged":
         pt = host["page_table"].numpy()[:1]
         k = oa.gather_paged(host["k_pool"][:, :, :1].to(torch.float64).numpy(), pt, S)
         v = oa.gather_paged(host["v_pool"][:, :, :1].to(torch.float64).numpy(), pt, S)
@@ -549,6 +566,7 @@ def run_reference(args):
            "fp8": lambda: workloads.all_fp8(S=S, B=B, H=Hq, D=D),
            "sage": lambda: workloads.sage(S=S, B=B, H=Hq, D=D),
            "sparse_paged": lambda: workloads.sparse_paged(S=S, B=B, Hq=Hq, Hkv=Hkv, D=D),
+           "sparse_contig": lambda: workloads.sparse_paged(S=S, B=B, Hq=Hq, Hkv=Hkv, D=D),
            "decode_paged": lambda: workloads.decode_paged(S=S, B=B, Hq=Hq, Hkv=Hkv, D=D)}[kind]
     host = gen()
     rows = 256
@@ -641,7 +659,7 @@ def run_smooth(args):
         "value": round(world * gbs, 1), "unit": "GB/s", "n_gpus": world, "steps": K_, "warmup": args.warmup,
         "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16->int8", "data": "synthetic (seeded; the Sage workload's K, N(0,1) + per-channel N(0,2) bias)",
-        "config": {"workload": "sage_k_smooth", "B": B, "H": H, "S": S, "D": D, "k_scale": "per 64-token block",
+        "config": {"workload": args.workload, "B": B, "H": H, "S": S, "D": D, "k_scale": "per 64-token block",
                    "l2": "inputs fit in L2: flushed before each step (512 MiB write, outside the timed events)"
                    if fits_l2 else "inputs larger than L2",
                    "parallelism": f"replicas{world}"},
@@ -732,102 +750,6 @@ def run_reference_nvfp4(args):
         "e2e": {"value": round(val, 6), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}), flush=True)
 
 
-def probe_peaks():
-    """Library GEMM peaks on this GPU (8192^3, best of 10, CUDA events): bf16
-    torch.matmul, E4M3 torch._scaled_mm (fp32 scales, bf16 out), INT8
-    torch._int_mm. Context for the 8-bit rooflines; the reported peaks stay
-    MEASURED_PEAKS.json's bf16 burst with the nominal 2x ratio for 8-bit."""
-    dev = torch.device("cuda")
-    n = 8192
-    a = torch.randn(n, n, device=dev, dtype=torch.bfloat16)
-    b = torch.randn(n, n, device=dev, dtype=torch.bfloat16)
-    a8, b8 = a.to(torch.float8_e4m3fn), b.to(torch.float8_e4m3fn).t().contiguous().t()
-    one = torch.ones((), device=dev, dtype=torch.float32)
-    ai = torch.randint(-100, 100, (n, n), device=dev, dtype=torch.int8)
-    bi = torch.randint(-100, 100, (n, n), device=dev, dtype=torch.int8).t().contiguous().t()
-    runs = {"bf16_matmul": lambda: a @ b,
-            "e4m3_scaled_mm": lambda: torch._scaled_mm(a8, b8, scale_a=one, scale_b=one, out_dtype=torch.bfloat16),
-            "int8_int_mm": lambda: torch._int_mm(ai, bi)}
-    out = {}
-    for name, f in runs.items():
-        try:
-            for _ in range(3):
-                f()
-            torch.cuda.synchronize()
-            best = 1e30
-            for _ in range(10):
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                e0.record()
-                f()
-                e1.record()
-                torch.cuda.synchronize()
-                best = min(best, e0.elapsed_time(e1))
-            out[name] = round(2.0 * n ** 3 / (best * 1e-3) / 1e12, 1)
-        except Exception as e:  # a dtype path this torch build lacks
-            out[name] = f"unavailable: {type(e).__name__}: {e}"[:160]
-    print(json.dumps({"probe": "library GEMM peaks, 8192^3, TFLOP/s (TOP/s for int8)", **out}), flush=True)
-
-
-def quant_probe(capture=False):
-    """Block-quantizer calls on the Sage workload's K and Q (B1 H24 S16384 D128),
-    each timed alone after an L2 flush: INT8 / E4M3 per 64-token block, INT8 per
-    64-token block with the K-smoothing shift, INT8 per 128-token block, and the
-    channel mean. With capture=True it makes only two calls, INT8 per 64-token
-    block without and then with the shift (a short program for ncu)."""
-    from precision_attention_fmha_b200 import fmha, workloads
-
-    dev = torch.device("cuda")
-    w = workloads.sage()
-    k = w["k"].to(dev)
-    B, S, H, D = k.shape
-    mean = torch.empty((B, H, D), dtype=torch.float32, device=dev)
-    ws = torch.empty(max(16, fmha.channel_mean_workspace_bytes(B, S, H, D)), dtype=torch.uint8, device=dev)
-    codes = torch.empty(k.shape, dtype=torch.int8, device=dev)
-    sc64 = torch.empty(fmha.scale_shape("per_token_block", B, S, H, D, 64), dtype=torch.float32, device=dev)
-    fmha.channel_mean(k, out=mean, workspace=ws)
-    if capture:
-        fmha.fmha_quantize_blockwise(k, torch.int8, "per_token_block", 64, out=codes, scales=sc64)
-        fmha.fmha_quantize_blockwise(k, torch.int8, "per_token_block", 64, out=codes, scales=sc64, shift=mean)
-        torch.cuda.synchronize()
-        fmha.get_device_error()
-        return
-    q = w["q"].to(dev)
-    codes_e = torch.empty(k.shape, dtype=torch.float8_e4m3fn, device=dev)
-    sc128 = torch.empty(fmha.scale_shape("per_token_block", B, S, H, D, 128), dtype=torch.float32, device=dev)
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-
-    def timed(fn, n=20):
-        for _ in range(3):
-            fn()
-        torch.cuda.synchronize()
-        total = 0.0
-        for _ in range(n):
-            flush.zero_()
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record()
-            fn()
-            b.record()
-            torch.cuda.synchronize()
-            total += a.elapsed_time(b)
-        return round(total / n * 1000, 2)
-
-    res = {
-        "probe": "block quantizer on the Sage workload's K / Q, us per call, L2 flushed before each",
-        "channel_mean": timed(lambda: fmha.channel_mean(k, out=mean, workspace=ws)),
-        "int8_per64": timed(lambda: fmha.fmha_quantize_blockwise(k, torch.int8, "per_token_block", 64, out=codes,
-                                                                scales=sc64)),
-        "int8_per64_shift": timed(lambda: fmha.fmha_quantize_blockwise(k, torch.int8, "per_token_block", 64,
-                                                                      out=codes, scales=sc64, shift=mean)),
-        "e4m3_per64": timed(lambda: fmha.fmha_quantize_blockwise(k, torch.float8_e4m3fn, "per_token_block", 64,
-                                                                out=codes_e, scales=sc64)),
-        "int8_per128_q": timed(lambda: fmha.fmha_quantize_blockwise(q, torch.int8, "per_token_block", 128,
-                                                                   out=codes, scales=sc128)),
-        "algorithmic_bytes_per_call": k.numel() * 3,
-    }
-    fmha.get_device_error()
-    print(json.dumps(res), flush=True)
-
-
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -836,16 +758,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(WORKLOADS))
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--probe-peaks", action="store_true", help="print library GEMM peaks (bf16, E4M3, INT8) and exit")
-    ap.add_argument("--quant-probe", choices=["time", "capture"],
-                    help="time the block quantizer on the Sage workload's K / Q ('capture': two calls, for ncu)")
     args = ap.parse_args()
-    if args.probe_peaks:
-        probe_peaks()
-        return
-    if args.quant_probe:
-        quant_probe(capture=args.quant_probe == "capture")
-        return
     if args.warmup < 3 and args.impl == "ours":
         args.warmup = 3
     kind = WORKLOADS[args.workload][0]

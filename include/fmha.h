@@ -153,6 +153,8 @@ typedef struct {
  * 1.0 when amax == 0); code = RN(fp32(x) / scale) (IEEE division), INT8
  * rounded half-to-even and clamped to [-127, 127], E4M3 rounded to nearest
  * even with saturation to +-448. Inputs must be finite.
+ * S == 0 writes no code; the grid-wide kinds then write scale 1.0 into every
+ * group. H and B must be at most 65535 (FMHA_ERR_UNSUPPORTED otherwise).
  * PER_TOKEN_BLOCK needs no workspace. The other kinds reduce amax across the
  * whole grid and need `workspace`: a device buffer of at least
  * fmha_quantize_workspace_bytes(...) bytes, 4-byte aligned, owned by the
@@ -180,7 +182,10 @@ size_t fmha_quantize_workspace_bytes(int32_t sf_kind, int32_t B, int32_t S, int3
  *    FMHA_ERR_INVALID_ARG with the sizes in fmha_last_error_message().
  *  - The first call on a device (that device current) looks up the array's
  *    device address with cudaGetSymbolAddress; make that first call before
- *    any stream capture.
+ *    any stream capture. The address is kept for the life of the process:
+ *    after cudaDeviceReset the library's module is loaded again and the kept
+ *    address is stale, so do not call this entry point (nor any other that
+ *    uses the device error word) after a device reset.
  *  - All calls share the one array. It keeps the last call's contents; each
  *    call clears the part it uses before use. Calls that overlap on the GPU
  *    (for example on two streams at once) race and give wrong scales: order

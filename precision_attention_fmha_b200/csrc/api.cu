@@ -546,6 +546,8 @@ fmha_status quantize_impl(const fmha_tensor* src, const float* shift, const fmha
   if (kind == FMHA_SF_PER_CHANNEL && (256 % (D / 8)) != 0)
     return fail(FMHA_ERR_UNSUPPORTED, "per-channel scales need D a power of two in [8, 2048]");
   if (B == 0 || H == 0) return ok_status();
+  if (H > 65535 || B > 65535) return fail(FMHA_ERR_UNSUPPORTED, "grid too large: H and B must be <= 65535");
+  if (kind == FMHA_SF_PER_TOKEN_BLOCK && S == 0) return ok_status();  // no block, no scale
   if (sf->ptr == nullptr || (reinterpret_cast<uintptr_t>(sf->ptr) & 3u))
     return fail(FMHA_ERR_INVALID_ARG, "sf.ptr is NULL or misaligned");
   if (S > 0) {
@@ -557,7 +559,6 @@ fmha_status quantize_impl(const fmha_tensor* src, const float* shift, const fmha
     for (int i = 0; i < 3; ++i)
       if (ds[i] % 8 != 0) return fail(FMHA_ERR_INVALID_ARG, "dst strides must be multiples of 8 bytes");
   }
-  if (kind == FMHA_SF_PER_TOKEN_BLOCK && S == 0) return ok_status();
   const size_t need = fmha_quantize_workspace_bytes(kind, B, S, H, D);
   if (need > 0) {
     if (workspace == nullptr || workspace_bytes < need)

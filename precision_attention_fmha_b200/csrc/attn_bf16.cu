@@ -1,12 +1,6 @@
 // BF16 Q/K/V instantiations of the attention kernel (D = 64, 128; contiguous and paged K/V).
 #include "attn_kernel.cuh"
 
-#ifdef FMHA_TRACE
-extern "C" int fmha_trace_read_bf16(void* host, size_t bytes) {
-  return (int)cudaMemcpyFromSymbol(host, g_fmha_trace, bytes);
-}
-#endif
-
 namespace fmha {
 cudaError_t launch_attention_bf16(int D, bool paged, const AttnParams& p, const CUtensorMap& tq,
                                   const CUtensorMap& tk, const CUtensorMap& tv, const CUtensorMap& to,

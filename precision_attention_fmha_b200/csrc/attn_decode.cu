@@ -4,12 +4,6 @@
 // ranges, and the merge of the splits' partial outputs by their log-sum-exp.
 #include "attn_kernel.cuh"
 
-#ifdef FMHA_TRACE
-extern "C" int fmha_trace_read_decode(void* host, size_t bytes) {
-  return (int)cudaMemcpyFromSymbol(host, g_fmha_trace, bytes);
-}
-#endif
-
 namespace fmha {
 
 cudaError_t launch_attention_packed(int qk, int pv, bool paged, const AttnParams& p, const CUtensorMap& tq,

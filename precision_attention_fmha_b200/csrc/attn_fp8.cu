@@ -1,12 +1,6 @@
 // All-E4M3 (Q, K, V) instantiations of the attention kernel (D = 128).
 #include "attn_kernel.cuh"
 
-#ifdef FMHA_TRACE
-extern "C" int fmha_trace_read_fp8(void* host, size_t bytes) {
-  return (int)cudaMemcpyFromSymbol(host, g_fmha_trace, bytes);
-}
-#endif
-
 namespace fmha {
 cudaError_t launch_attention_fp8(int, bool paged, const AttnParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
                                  const CUtensorMap& tv, const CUtensorMap& to, cudaStream_t s) {

@@ -41,23 +41,6 @@
 #include "fmha_internal.h"
 #include "ptx_sm100.cuh"
 
-// Optional phase tracing for one CTA (build with -DFMHA_TRACE=<cta index>):
-// clock64 stamps of each role's phases go to a device array that the host
-// reads with fmha_trace_read(). Off in normal builds.
-#ifdef FMHA_TRACE
-#define FMHA_TRACE_SLOTS (1 << 16)
-static __device__ unsigned long long g_fmha_trace[FMHA_TRACE_SLOTS];  // one per translation unit
-#define TRACE(slot, cond)                                                                   \
-  do {                                                                                      \
-    if (blockIdx.x == (FMHA_TRACE) && (cond) && (slot) < FMHA_TRACE_SLOTS)                  \
-      g_fmha_trace[(slot)] = static_cast<unsigned long long>(clock64());                    \
-  } while (0)
-#else
-#define TRACE(slot, cond) \
-  do {                    \
-  } while (0)
-#endif
-
 namespace fmha {
 
 template <int D_, int QK_, int PV_, bool PAGED_, bool P2_ = false, bool PACKED_ = false, bool O8_ = false>
@@ -323,9 +306,7 @@ __device__ void attn_load_role(const AttnParams& p, const TileInfo t0, const Til
       const int s = slot_it % C::STAGES;
       const uint32_t ph = (slot_it / C::STAGES) & 1;
       ++slot_it;
-      TRACE(32768 + u * 8 + kv * 4 + 0, lane == 0);
       if (!(ok = __all_sync(FULL, w.wait(smem_addr(&misc->kv_empty[s]), ph ^ 1)))) break;
-      TRACE(32768 + u * 8 + kv * 4 + 1, lane == 0);
       const uint32_t full = smem_addr(&misc->kv_full[s]);
       const int chunks = kv == 0 ? C::QK_CHUNKS : C::V_CHUNKS;
       const int chunk_elems = kv == 0 ? C::QK_CHUNK_ELEMS : C::V_CHUNK_ELEMS;
@@ -445,7 +426,6 @@ __device__ void attn_mma_role(const AttnParams& p, const TileInfo t0, const Tile
   for (int u = min(t0.u0, t1.u0); u < n_u && ok; ++u) {
     const bool kx[2] = {keep_tile<C>(p, t0, b, hkv, u, misc), keep_tile<C>(p, t1, b, hkv, u, misc)};
     if (!kx[0] && !kx[1]) continue;
-    TRACE(16384 + u * 16 + 15, leader);
     const int ks = slot_it % C::STAGES;
     const uint32_t kph = (slot_it / C::STAGES) & 1;
     ++slot_it;
@@ -463,9 +443,7 @@ __device__ void attn_mma_role(const AttnParams& p, const TileInfo t0, const Tile
       for (int x = 0; x < 2 && ok; ++x) {
         if (kx[x] != (pass == 0)) continue;
         if (pend[x] >= 0) {
-          TRACE(16384 + u * 16 + x * 8 + 0, leader);
           if (!(ok = __all_sync(FULL, w.wait(smem_addr(&misc->p_full[x]), pv_cnt[x] & 1)))) break;
-          TRACE(16384 + u * 16 + x * 8 + 1, leader);
           tc_fence_after();
           if (leader) {
             issue_pv<C>(tmem + o_col[x], tmem + s_col[x], v_lo0 + pend[x] * (C::SLOT >> 4), hi, pv_cnt[x] > 0);
@@ -473,7 +451,6 @@ __device__ void attn_mma_role(const AttnParams& p, const TileInfo t0, const Tile
               issue_pv<C>(tmem + o_col[x], tmem + s_col[x] + 32, v_lo0 + pend[x] * (C::SLOT >> 4), hi, 1u);
           }
           __syncwarp();
-          TRACE(16384 + u * 16 + x * 8 + 2, leader);
           ++pv_cnt[x];
           pend[x] = -1;
         }
@@ -483,13 +460,11 @@ __device__ void attn_mma_role(const AttnParams& p, const TileInfo t0, const Tile
             tc_fence_after();
             k_ready = true;
           }
-          TRACE(16384 + u * 16 + x * 8 + 3, leader);
           if (leader) {
             issue_qk<C>(tmem + s_col[x], x ? q_lo1 : q_lo0, k_lo0 + ks * (C::SLOT >> 4), hi);
             tc_commit(smem_addr(&misc->s_full[x]));
           }
           __syncwarp();
-          TRACE(16384 + u * 16 + x * 8 + 5, leader);
         }
       }
     }
@@ -500,7 +475,6 @@ __device__ void attn_mma_role(const AttnParams& p, const TileInfo t0, const Tile
     }
     __syncwarp();
     if (!(ok = __all_sync(FULL, w.wait(smem_addr(&misc->kv_full[vs]), vph)))) break;
-    TRACE(16384 + u * 16 + 7, leader);
     tc_fence_after();
     pend[0] = kx[0] ? vs : -1;
     pend[1] = kx[1] ? vs : -1;
@@ -576,7 +550,6 @@ __device__ void attn_mma_role_psmem(const AttnParams& p, const TileInfo t0, cons
         if (!(ok = __all_sync(FULL, w.wait(smem_addr(&misc->s_free[x]), (s_cnt[x] - 1) & 1)))) return;
         tc_fence_after();
       }
-      TRACE(16384 + u * 16 + 10 + x, leader);
       if (leader) {
         issue_qk<C>(tmem + s_col[x], x ? q_lo1 : q_lo0, k_lo0 + ks * (C::SLOT >> 4), hi);
         tc_commit(smem_addr(&misc->s_full[x]));
@@ -601,7 +574,6 @@ __device__ void attn_mma_role_psmem(const AttnParams& p, const TileInfo t0, cons
     }
   }
   while (u < n_u && ok) {
-    TRACE(16384 + u * 16 + 0, leader);
     const int vph_it = slot_it - 1;  // ring position of V_u
     const uint32_t vph = (vph_it / C::STAGES) & 1;
     const int nu = next_kept(u + 1);
@@ -614,22 +586,17 @@ __device__ void attn_mma_role_psmem(const AttnParams& p, const TileInfo t0, cons
       ++slot_it;
       if (!(ok = __all_sync(FULL, w.wait(smem_addr(&misc->kv_full[nks]), nkph)))) break;
       tc_fence_after();
-      TRACE(16384 + u * 16 + 1, leader);
       issue_s(nu, nks);
       if (!ok) break;
       if (leader) tc_commit(smem_addr(&misc->kv_empty[nks]));
       __syncwarp();
     }
-    TRACE(16384 + u * 16 + 2, leader);
     if (!(ok = __all_sync(FULL, w.wait(smem_addr(&misc->kv_full[vs]), vph)))) break;
-    TRACE(16384 + u * 16 + 3, leader);
     tc_fence_after();
 #pragma unroll
     for (int x = 0; x < 2; ++x) {
       if (!keep_tile<C>(p, x ? t1 : t0, b, hkv, u, misc)) continue;
-      TRACE(16384 + u * 16 + 4 + x * 3, leader);
       if (!(ok = __all_sync(FULL, w.wait(smem_addr(&misc->p_full[x]), pv_cnt[x] & 1)))) break;
-      TRACE(16384 + u * 16 + 5 + x * 3, leader);
       tc_fence_after();
       if (leader) {
         const uint32_t plo = x ? p_lo1 : p_lo0;
@@ -639,7 +606,6 @@ __device__ void attn_mma_role_psmem(const AttnParams& p, const TileInfo t0, cons
         tc_commit(smem_addr(&misc->pv_done[x]));
       }
       __syncwarp();
-      TRACE(16384 + u * 16 + 6 + x * 3, leader);
       ++pv_cnt[x];
     }
     if (!ok) break;
@@ -728,11 +694,9 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, 
   bool ok = true;
   for (int u = t.u0; u < t.n_kv; ++u) {
     if (!keep_tile<C>(p, t, b, hkv, u, misc)) continue;
-    TRACE(x * 8192 + it * 16 + 0, lead);
     // A failed wait does not leave the loop here: the exchange below does, for
     // both threads of the row at once (the work in between is harmless).
     ok = __all_sync(FULL, w.wait(smem_addr(&misc->s_full[x]), it & 1)) && ok;
-    TRACE(x * 8192 + it * 16 + 1, lead);
     tc_fence_after();
 
     // Column factors: K scale per 32-key chunk (token-block K scales), times cq.
@@ -759,7 +723,6 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, 
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_addr(&misc->s_free[x]));
     }
-    TRACE(x * 8192 + it * 16 + 2, lead);
     float f[NC][32];
 #pragma unroll
     for (int c = 0; c < NC; ++c)
@@ -827,13 +790,11 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, 
     // walk the same KV tiles) the warpgroups alternate their exponential
     // phases, so that one exponentiates while the other loads, reduces and
     // packs. Tile 0 goes first.
-    TRACE(x * 8192 + it * 16 + 3, lead);
     if (x == 0 ? (it >= 1 && it < n_turns) : (it < n_turns)) {
       ok = __all_sync(FULL, w.wait(smem_addr(&misc->exp_done[x ^ 1]), (x == 0 ? it - 1 : it) & 1)) && ok;
 #pragma unroll
       for (int c = 0; c < NC; ++c) reg_fence(f[c]);
     }
-    TRACE(x * 8192 + it * 16 + 4, lead);
     const float mb = (m == -INFINITY ? 0.f : m) - log2g;
 #pragma unroll
     for (int c = 0; c < NC; ++c)
@@ -849,7 +810,6 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, 
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_addr(&misc->exp_done[x]));
     }
-    TRACE(x * 8192 + it * 16 + 5, lead);
     float rs = 0.f;
     if constexpr (C::PV == PV_BF16) {
       // BF16 P of this thread's columns goes over TMEM columns [32 * NC/2 * h, ...)
@@ -913,14 +873,12 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, 
 #pragma unroll
         for (int c = 1; c < NC; ++c) rs += racc[c];
       }
-      TRACE(x * 8192 + it * 16 + 6, lead);
       if constexpr (C::PSMEM) {
         // The previous PV must be done before P (single buffer) or O is rewritten.
         if (it > 0) {
           ok = __all_sync(FULL, w.wait(smem_addr(&misc->pv_done[x]), (it - 1) & 1)) && ok;
           tc_fence_after();
         }
-        TRACE(x * 8192 + it * 16 + 7, lead);
         rescale_o();
         // Row r of the 128 x 128-byte P tile, 16-byte chunks XOR-swizzled by r % 8
         // (the 128-byte swizzle the PV descriptor expects); this thread writes
@@ -945,12 +903,10 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, 
       }
     }
     l = l * alpha + rs;
-    TRACE(x * 8192 + it * 16 + 8, lead);
     tmem_wait_st();
     tc_fence_before();
     __syncwarp();  // the warp's P stores are ordered before lane 0's arrive
     if (lane == 0) mbar_arrive(smem_addr(&misc->p_full[x]));
-    TRACE(x * 8192 + it * 16 + 9, lead);
     ++it;
   }
 

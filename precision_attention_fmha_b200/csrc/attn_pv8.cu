@@ -1,13 +1,6 @@
 // QK-BF16 / PV-E4M3 instantiations of the attention kernel (D = 128).
 #include "attn_kernel.cuh"
 
-
-#ifdef FMHA_TRACE
-extern "C" int fmha_trace_read_pv8(void* host, size_t bytes) {
-  return (int)cudaMemcpyFromSymbol(host, g_fmha_trace, bytes);
-}
-#endif
-
 namespace fmha {
 cudaError_t launch_attention_pv8(int, bool paged, const AttnParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
                                  const CUtensorMap& tv, const CUtensorMap& to, cudaStream_t s) {

@@ -24,6 +24,7 @@
 // element, before the amax). The shift is normally the token mean per channel,
 // which channel_mean_* computes: fp64 partial sums per CTA, then a fixed-order
 // sum over the CTAs, one fp64 division by S and one rounding to fp32.
+#include <algorithm>
 #include <mutex>
 
 #include "fmha_internal.h"
@@ -263,6 +264,13 @@ __global__ void __launch_bounds__(kThreads) quant_apply_kernel(const QuantParams
   }
 }
 
+// S == 0 for a grid-wide kind: every group's amax is 0, so every scale is 1.
+__global__ void __launch_bounds__(kThreads) fill_unit_scales_kernel(float* sf, int64_t n) {
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * kThreads)
+    sf[i] = 1.f;
+}
+
 template <bool kE4M3>
 cudaError_t launch_quantize_t(const QuantParams& p, cudaStream_t stream) {
   if (p.kind == FMHA_SF_PER_TOKEN_BLOCK) {
@@ -276,6 +284,11 @@ cudaError_t launch_quantize_t(const QuantParams& p, cudaStream_t stream) {
   const size_t groups = p.kind == FMHA_SF_PER_CHANNEL ? static_cast<size_t>(p.B) * p.H * p.D
                         : p.kind == FMHA_SF_PER_HEAD  ? static_cast<size_t>(p.B) * p.H
                                                       : 1;
+  if (p.S == 0) {  // no token: no amax pass (its grid would be empty), unit scales
+    const unsigned blocks = static_cast<unsigned>(std::min<size_t>((groups + kThreads - 1) / kThreads, 1024));
+    fill_unit_scales_kernel<<<blocks, kThreads, 0, stream>>>(p.sf, static_cast<int64_t>(groups));
+    return cudaGetLastError();
+  }
   cudaError_t e = cudaMemsetAsync(p.ws, 0, groups * sizeof(uint32_t), stream);
   if (e != cudaSuccess) return e;
   dim3 grid((p.S + p.rows_per_cta - 1) / p.rows_per_cta, p.H, p.B);

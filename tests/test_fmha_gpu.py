@@ -64,7 +64,7 @@ def check(mode, o, ref):
         assert_close_q8(o, ref)
 
 
-def run_dense(mode, B, Hq, Hkv, Sq, Skv, D, causal, seed, with_lse=False):
+def run_dense(mode, B, Hq, Hkv, Sq, Skv, D, causal, seed, with_lse=False, p_terms=None):
     if mode == "fp8":
         q, k, v = workloads.outlier_qkv(seed, B, max(Sq, Skv), Hq, D)
         q, k, v = q[:, :Sq], k[:, :Skv, :Hkv], v[:, :Skv, :Hkv]
@@ -79,7 +79,8 @@ def run_dense(mode, B, Hq, Hkv, Sq, Skv, D, causal, seed, with_lse=False):
     sf_p = None
     if mode == "sage":  # per-row-block P scale: P is stored as 16 p (lazy-rescale bound 2^4 * 16 <= 448)
         sf_p = Scale(torch.full((B, Hq, math.ceil(Sq / 128)), 1 / 16, device=DEV), "per_token_block", 128)
-    p_terms = 2 if mode == "sage" else 1  # Sage: P as two E4M3 terms (its sharp softmax needs the precision)
+    if p_terms is None:
+        p_terms = 1
     o = fmha.fmha_fwd(g["q"], g["k"], g["v"], sf_q=g["sf_q"], sf_k=g["sf_k"], sf_v=g["sf_v"], sf_p=sf_p,
                       softmax_scale=scale, causal=causal, lse=lse, p_terms=p_terms)
     fmha.get_device_error()
@@ -91,7 +92,7 @@ def run_dense(mode, B, Hq, Hkv, Sq, Skv, D, causal, seed, with_lse=False):
         assert np.array_equal(np.isfinite(got), fin)
         # BF16 P and two-term E4M3 P: exact sum of p; one-term E4M3 P: the sum of the
         # stored rounded P (|err| <= ln(1 + 2^-4))
-        bound = 2e-2 if mode in ("bf16", "sage") else math.log1p(2.0 ** -4) + 2e-3
+        bound = 2e-2 if mode == "bf16" or p_terms == 2 else math.log1p(2.0 ** -4) + 2e-3
         assert np.abs(got[fin] - ref_lse[fin]).max() < bound
     return o
 
@@ -123,7 +124,22 @@ def test_bf16(B, Hq, Hkv, Sq, Skv, D, causal):
 @pytest.mark.parametrize("Sq,Skv,causal,Hq,Hkv", [(300, 300, False, 2, 2), (1024, 1024, True, 2, 2),
                                                   (700, 1500, False, 4, 2), (129, 129, True, 1, 1)])
 def test_8bit_modes(mode, Sq, Skv, causal, Hq, Hkv):
+    """One E4M3 term of P (the precision every 8-bit workload states), whole heads."""
     run_dense(mode, 1, Hq, Hkv, Sq, Skv, 128, causal, seed=7 * Sq + Skv, with_lse=True)
+
+
+@pytest.mark.parametrize("Sq,Skv,causal", [(2048, 2048, False), (4096, 4096, False), (4096, 4096, True)])
+def test_sage_one_term_p_longer(Sq, Skv, causal):
+    """One-term Sage on longer rows: its biased scores sharpen the softmax as Skv grows."""
+    run_dense("sage", 1, 2, 2, Sq, Skv, 128, causal, seed=3 * Sq + 11, with_lse=True, p_terms=1)
+
+
+@pytest.mark.parametrize("Sq,Skv,causal,Hq,Hkv", [(300, 300, False, 2, 2), (1024, 1024, True, 2, 2),
+                                                  (700, 1500, False, 4, 2), (2048, 2048, False, 2, 2),
+                                                  (2048, 2048, True, 2, 2)])
+def test_sage_two_term_p(Sq, Skv, causal, Hq, Hkv):
+    """Sage with P split into two E4M3 terms (the more precise option)."""
+    run_dense("sage", 1, Hq, Hkv, Sq, Skv, 128, causal, seed=7 * Sq + Skv + 1, with_lse=True, p_terms=2)
 
 
 def test_empty_kv_gives_zero_and_minus_inf():

@@ -72,3 +72,22 @@ def test_quantizer_workload_sizes(name):
         _, _, x = workloads.normal_qkv(workloads.SEED_BASE + 2 + 16384, 1, 16384, 16384, 40, 40, 128)
         out, kind, rpb = "e4m3", "per_tensor", None
     _check(x, out, kind, rpb)
+
+
+@pytest.mark.parametrize("out", ["int8", "e4m3"])
+@pytest.mark.parametrize("kind,rpb", [("per_token_block", 64), ("per_head", None), ("per_tensor", None),
+                                      ("per_channel", None)])
+def test_quantizer_empty_sequence(out, kind, rpb):
+    """S == 0: no code is written; the grid-wide kinds write scale 1.0 (amax 0) into every group."""
+    B, H, D = 2, 3, 128
+    x = torch.zeros((B, 0, H, D), dtype=torch.bfloat16)
+    ref_c, ref_s = oq.quantize_blockwise(f32(x), out, kind, rpb)
+    dev = torch.device("cuda")
+    scales = torch.full(fmha.scale_shape(kind, B, 0, H, D, rpb), float("nan"), device=dev)
+    codes, scales = fmha.fmha_quantize_blockwise(x.to(dev), DT[out], kind, rpb, scales=scales)
+    torch.cuda.synchronize()
+    assert codes.numel() == 0
+    got_s = scales.cpu().numpy().reshape(ref_s.shape)
+    assert np.array_equal(got_s, ref_s)
+    if kind != "per_token_block":
+        assert np.all(got_s == 1.0)

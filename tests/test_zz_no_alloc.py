@@ -77,3 +77,18 @@ def test_noalloc_rejects_more_groups_than_the_builtin_scratch():
                                             None)
     assert st == 1
     assert "65536" in lib.fmha_last_error_message().decode()
+
+
+@pytest.mark.parametrize("kind", ["per_tensor", "per_head", "per_channel", "per_token_block"])
+def test_noalloc_empty_sequence(kind):
+    """S == 0 through the no-allocation entry point: no code, unit scales for the grid-wide kinds,
+    the same as the workspace entry point."""
+    x = torch.zeros((2, 0, 3, 128), dtype=torch.bfloat16, device=DEV)
+    st, codes, scales = _noalloc(x, torch.int8, kind, 64 if kind == "per_token_block" else 0)
+    assert st == 0, _lib().fmha_last_error_message().decode()
+    _, ref_scales = fmha.fmha_quantize_blockwise(x, torch.int8, kind, 64 if kind == "per_token_block" else None)
+    torch.cuda.synchronize()
+    assert codes.numel() == 0
+    assert np.array_equal(scales.cpu().numpy(), ref_scales.cpu().numpy())
+    if kind != "per_token_block":
+        assert np.all(scales.cpu().numpy() == 1.0)
