@@ -17,7 +17,7 @@ from oracle import attention as oa
 from oracle import quant as oq
 from precision_attention_fmha_b200 import fmha, workloads
 from precision_attention_fmha_b200.fmha import Scale
-from tests.helpers import assert_close_bf16, assert_close_q8, codes_np, f32, f64
+from tests.helpers import Q8_ATOL, Q8_ONE_TERM_ATOL, assert_close_bf16, assert_close_q8, codes_np, f32, f64
 
 pytestmark = pytest.mark.gpu
 DEV = torch.device("cuda")
@@ -56,15 +56,15 @@ def prepare(mode, q, k, v):
     return g, ref["q"], ref["k"], ref["v"]
 
 
-def check(mode, o, ref):
+def check(mode, o, ref, atol=Q8_ATOL):
     o = f64(o)
     if mode == "bf16":
         assert_close_bf16(o, ref)
     else:
-        assert_close_q8(o, ref)
+        assert_close_q8(o, ref, atol=atol)
 
 
-def run_dense(mode, B, Hq, Hkv, Sq, Skv, D, causal, seed, with_lse=False, p_terms=None):
+def run_dense(mode, B, Hq, Hkv, Sq, Skv, D, causal, seed, with_lse=False, p_terms=None, atol=Q8_ATOL):
     if mode == "fp8":
         q, k, v = workloads.outlier_qkv(seed, B, max(Sq, Skv), Hq, D)
         q, k, v = q[:, :Sq], k[:, :Skv, :Hkv], v[:, :Skv, :Hkv]
@@ -85,7 +85,7 @@ def run_dense(mode, B, Hq, Hkv, Sq, Skv, D, causal, seed, with_lse=False, p_term
                       softmax_scale=scale, causal=causal, lse=lse, p_terms=p_terms)
     fmha.get_device_error()
     ref_o, ref_lse = oa.attention(rq, rk, rv, scale, causal)
-    check(mode, o, ref_o)
+    check(mode, o, ref_o, atol)
     if with_lse:
         got = lse.cpu().numpy().astype(np.float64)
         fin = np.isfinite(ref_lse)
@@ -125,13 +125,16 @@ def test_bf16(B, Hq, Hkv, Sq, Skv, D, causal):
                                                   (700, 1500, False, 4, 2), (129, 129, True, 1, 1)])
 def test_8bit_modes(mode, Sq, Skv, causal, Hq, Hkv):
     """One E4M3 term of P (the precision every 8-bit workload states), whole heads."""
-    run_dense(mode, 1, Hq, Hkv, Sq, Skv, 128, causal, seed=7 * Sq + Skv, with_lse=True)
+    run_dense(mode, 1, Hq, Hkv, Sq, Skv, 128, causal, seed=7 * Sq + Skv, with_lse=True,
+              atol=Q8_ONE_TERM_ATOL if mode == "sage" else Q8_ATOL)
 
 
 @pytest.mark.parametrize("Sq,Skv,causal", [(2048, 2048, False), (4096, 4096, False), (4096, 4096, True)])
 def test_sage_one_term_p_longer(Sq, Skv, causal):
-    """One-term Sage on longer rows: its biased scores sharpen the softmax as Skv grows."""
-    run_dense("sage", 1, 2, 2, Sq, Skv, 128, causal, seed=3 * Sq + 11, with_lse=True, p_terms=1)
+    """One-term Sage on longer rows: its biased scores sharpen the softmax as Skv grows, and
+    the E4M3 rounding of a few dominant weights shows in max-abs (cosine stays binding)."""
+    run_dense("sage", 1, 2, 2, Sq, Skv, 128, causal, seed=3 * Sq + 11, with_lse=True, p_terms=1,
+              atol=Q8_ONE_TERM_ATOL)
 
 
 @pytest.mark.parametrize("Sq,Skv,causal,Hq,Hkv", [(300, 300, False, 2, 2), (1024, 1024, True, 2, 2),
