@@ -114,10 +114,12 @@ typedef struct {
  *   causal != 0: key j is visible to query i iff j <= i + (Skv - Sq)
  *   (bottom-right aligned).
  *   lse (nullable): fp32 [B, Hq, Sq], natural-log log-sum-exp of the scaled
- *   scores; -inf for a row with no visible key (whose O row is 0). When P is
- *   cast to E4M3 (8-bit V) the sum runs over the stored, rounded P values --
- *   the same normaliser O uses, so partial results merge exactly -- and lse
- *   then differs from the exact value by at most ln(1 + 2^-4) ~ 0.061.
+ *   scores; -inf for a row with no visible key (whose O row is 0). The sum
+ *   runs over the exponentials before P is rounded to its BF16 or E4M3
+ *   format (with one E4M3 term, plus the rounding error of each 128-key
+ *   tile's largest weight, so that a dominant key's weight is exact, which
+ *   moves lse by at most ln(1 + 2^-4) ~ 0.061); it is the normaliser O uses,
+ *   so partial results merge exactly.
  * Supported (q, k, v, o) dtype tuples: (BF16, BF16, BF16, BF16),
  * (BF16, BF16, E4M3, BF16) ("QK-BF16/PV-FP8", [BW-FP8]),
  * (E4M3, E4M3, E4M3, BF16) ("all-FP8", [BW-FP8]), (INT8, INT8, E4M3, BF16)
@@ -237,7 +239,9 @@ fmha_status fmha_fwd(const fmha_args* args, struct CUstream_st* stream);
  *   mask: uint8, element (b, h_kv, i, j) at mask[b*mask_stride_b +
  *   h_kv*mask_stride_h + i*ceil(Skv/128) + j], nonzero = the 128x128 block of
  *   query rows [128i, 128i+128) x keys [128j, 128j+128) is visible (ANDed with
- *   causal). Strides may be 0 to broadcast. Fully hidden rows give O = 0.    */
+ *   causal). Strides may be 0 to broadcast. Fully hidden rows give O = 0.
+ *   Skv <= 131072 (1024 key blocks) when a mask is given: each CTA keeps its
+ *   rows' kept key blocks as a 1024-bit set in shared memory.               */
 fmha_status fmha_fwd_block_sparse(const fmha_args* args, const uint8_t* mask, int64_t mask_stride_b,
                                   int64_t mask_stride_h, struct CUstream_st* stream);
 

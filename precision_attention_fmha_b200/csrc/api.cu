@@ -328,6 +328,8 @@ fmha_status run_attention(const fmha_args* a, const uint8_t* mask, int64_t msb, 
   if (a->lse != nullptr && (reinterpret_cast<uintptr_t>(a->lse) & 3u) != 0)
     return fail(FMHA_ERR_INVALID_ARG, "lse misaligned");
   if (mask != nullptr && (msb < 0 || msh < 0)) return fail(FMHA_ERR_INVALID_ARG, "mask strides must be >= 0");
+  if (mask != nullptr && ceil_div(Skv, 128) > 1024)
+    return fail(FMHA_ERR_UNSUPPORTED, "block mask: Skv %d > 131072 (1024 KV blocks)", Skv);
 
   // TMA descriptors
   const int eqk = qk == QK_BF16 ? 2 : 1, ev = pv == PV_BF16 ? 2 : 1;

@@ -41,6 +41,8 @@
 #include "fmha_internal.h"
 #include "ptx_sm100.cuh"
 
+#include <type_traits>
+
 namespace fmha {
 
 template <int D_, int QK_, int PV_, bool PAGED_, bool P2_ = false, bool PACKED_ = false, bool O8_ = false>
@@ -93,20 +95,16 @@ struct AttnCfg {
                                                        : ptx::make_idesc(2, 1, 1, 0, 0, BN, BM);
   static constexpr uint32_t IDESC_PV =
       PV == PV_BF16 ? ptx::make_idesc(1, 1, 1, 0, 1, D, BM) : ptx::make_idesc(1, 0, 0, 0, 1, D, BM);
-  // Threads per query row in the softmax. 2 splits every row's 128 scores
-  // between two warps of the same TMEM lane quadrant (64 columns each, 640
-  // threads, a row-max exchange per tile); it is correct but measured 10-15 %
-  // slower than one thread per row (more warps per scheduler, 104 registers).
-  static constexpr int NH = 1;
-  static constexpr int THREADS = 128 + 256 * NH;
+  static constexpr int THREADS = 384;
   // Warp roles: warpgroup 0 = control (MMA issue, TMA loads, two idle warps),
-  // warpgroups 1 and 2 = softmax of query tiles 0 and 1. The control warps
-  // come first: the issue scheduler favours older warps, and the MMA warp's
-  // short serial steps sit on the critical path of both softmax pipelines.
+  // warpgroups 1 and 2 = softmax of query tiles 0 and 1 (one thread per row).
+  // The control warps come first: the issue scheduler favours older warps, and
+  // the MMA warp's short serial steps sit on the critical path of both softmax
+  // pipelines.
   static constexpr int MMA_WARP = 0, LOAD_WARP = 1, SOFTMAX_WARP0 = 4;
-  // setmaxnreg split of the launch's registers (THREADS x 168 or x 96):
-  // 384 threads: 2*128*216 + 128*72; 640 threads: 4*128*104 + 128*64.
-  static constexpr uint32_t SOFTMAX_REGS = NH == 2 ? 104 : 216, CONTROL_REGS = NH == 2 ? 64 : 72;
+  // setmaxnreg split of the launch's registers (384 threads x 168):
+  // 2 * 128 * 216 + 128 * 72.
+  static constexpr uint32_t SOFTMAX_REGS = 216, CONTROL_REGS = 72;
   static_assert(2 * 128 * SOFTMAX_REGS + 128 * CONTROL_REGS <= THREADS * 168, "register split exceeds launch");
 };
 
@@ -124,12 +122,12 @@ struct alignas(8) AttnMisc {
   uint32_t tmem_base;
   volatile uint32_t abort;
   float sf_v[128];
-  // Packed (decode) CTAs: the KV tiles each query tile processes, as a bit set
-  // over KV tiles (at most 1024), and its [first, last + 1) range.
+  // The KV tiles each query tile processes, as a bit set over KV tiles (at
+  // most 1024), for packed (decode) CTAs and for every launch with a block
+  // mask: built once in the prologue, so no role reads the mask per tile.
   uint32_t keep_bits[2][32];
-  int32_t range[2][2];
-  // Two threads per row: one exchange slot per row of each query tile.
-  float xchg[2][128];
+  int32_t range[2][2];  // packed: [first, last + 1) of each query tile's kept tiles
+  int32_t same_kept;    // masked: both query tiles keep the same KV tiles (count), else 0
 };
 
 static_assert(sizeof(AttnMisc) <= 2048, "AttnMisc must fit the 2 KB misc area");
@@ -205,14 +203,32 @@ struct Waiter {
 // Tile info and waiters are passed by value everywhere: a runtime-indexed
 // array or a by-reference argument would live in local memory, and with the
 // shared-memory carve-out near its maximum every such load goes to L2.
+// Whether the CTA's KV tiles are listed in the keep-bit set (packed CTAs: the
+// split's tiles; masked launches: the block mask's kept tiles).
 template <class C>
-__device__ __forceinline__ bool keep_tile(const AttnParams& p, const TileInfo t, int b, int hkv, int u,
-                                          const AttnMisc* misc) {
-  if constexpr (C::PACKED)  // the split's tiles were chosen up front (mask, split, query-tile share)
-    return u >= t.u0 && u < t.n_kv && ((misc->keep_bits[t.x][u >> 5] >> (u & 31)) & 1u);
-  if (u >= t.n_kv) return false;
-  if (p.mask == nullptr) return true;
-  return p.mask[b * p.mask_sb + hkv * p.mask_sh + static_cast<int64_t>(t.mrow) * p.n_kv_blocks + u] != 0;
+__device__ __forceinline__ bool uses_keep_bits(const AttnParams& p) {
+  return C::PACKED || p.mask != nullptr;
+}
+
+template <class C>
+__device__ __forceinline__ bool keep_tile(const AttnParams& p, const TileInfo t, int u, const AttnMisc* misc) {
+  if (u < t.u0 || u >= t.n_kv) return false;
+  if (!uses_keep_bits<C>(p)) return true;
+  return (misc->keep_bits[t.x][u >> 5] >> (u & 31)) & 1u;
+}
+
+// First KV tile at or after `from` (and below n) kept by the query tiles whose
+// bits `sel` selects (1: tile 0, 2: tile 1, 3: either); n when none.
+template <class C>
+__device__ __forceinline__ int next_kept_tile(const AttnParams& p, const AttnMisc* misc, int sel, int from, int n) {
+  if (from >= n) return n;
+  if (!uses_keep_bits<C>(p)) return from;
+  for (int wd = from >> 5; (wd << 5) < n; ++wd) {
+    uint32_t bits = ((sel & 1) ? misc->keep_bits[0][wd] : 0u) | ((sel & 2) ? misc->keep_bits[1][wd] : 0u);
+    if (wd == (from >> 5)) bits &= ~0u << (from & 31);
+    if (bits) return min(n, (wd << 5) + __ffs(bits) - 1);
+  }
+  return n;
 }
 
 __device__ __forceinline__ float sf_lookup(const float* sf, int kind, int64_t bh, int nblk, int idx_in_seq,
@@ -266,20 +282,7 @@ __device__ void attn_load_role(const AttnParams& p, const TileInfo t0, const Til
   const int n_u = max(t0.n_kv, t1.n_kv);
   bool ok = true;
   // Next KV tile at or after `from` that either query tile keeps.
-  auto next_kept = [&](int from) {
-    if constexpr (C::PACKED) {  // scan the keep-bit words (at most 32)
-      for (int wd = from >> 5; wd < 32 && (wd << 5) < n_u; ++wd) {
-        uint32_t bits = misc->keep_bits[0][wd] | misc->keep_bits[1][wd];
-        if (wd == (from >> 5)) bits &= ~0u << (from & 31);
-        if (bits) return min(n_u, (wd << 5) + __ffs(bits) - 1);
-      }
-      return n_u;
-    } else {
-      int v = from;
-      while (v < n_u && !keep_tile<C>(p, t0, b, hkv, v, misc) && !keep_tile<C>(p, t1, b, hkv, v, misc)) ++v;
-      return v;
-    }
-  };
+  auto next_kept = [&](int from) { return next_kept_tile<C>(p, misc, 3, from, n_u); };
   // Paged K/V: lane l reads the page-table entry of page l of a tile (BN /
   // page_size <= 8 pages) once for its K and V copies, one kept tile ahead.
   const int per = C::PAGED ? C::BN / p.page_size : 1;
@@ -423,9 +426,9 @@ __device__ void attn_mma_role(const AttnParams& p, const TileInfo t0, const Tile
   const int n_u = max(t0.n_kv, t1.n_kv);
   bool ok = __all_sync(FULL, w.wait(smem_addr(&misc->q_full), 0));
   tc_fence_after();
-  for (int u = min(t0.u0, t1.u0); u < n_u && ok; ++u) {
-    const bool kx[2] = {keep_tile<C>(p, t0, b, hkv, u, misc), keep_tile<C>(p, t1, b, hkv, u, misc)};
-    if (!kx[0] && !kx[1]) continue;
+  for (int u = next_kept_tile<C>(p, misc, 3, min(t0.u0, t1.u0), n_u); u < n_u && ok;
+       u = next_kept_tile<C>(p, misc, 3, u + 1, n_u)) {
+    const bool kx[2] = {keep_tile<C>(p, t0, u, misc), keep_tile<C>(p, t1, u, misc)};
     const int ks = slot_it % C::STAGES;
     const uint32_t kph = (slot_it / C::STAGES) & 1;
     ++slot_it;
@@ -536,27 +539,39 @@ __device__ void attn_mma_role_psmem(const AttnParams& p, const TileInfo t0, cons
   int slot_it = 0;
   bool ok = __all_sync(FULL, w.wait(smem_addr(&misc->q_full), 0));
   tc_fence_after();
-  auto next_kept = [&](int from) {
-    int u = from;
-    while (u < n_u && !keep_tile<C>(p, t0, b, hkv, u, misc) && !keep_tile<C>(p, t1, b, hkv, u, misc)) ++u;
-    return u;
-  };
-  // Issues S_x(u) for every query tile keeping u; K_u lives in slot ks.
-  auto issue_s = [&](int u, int ks) {
-#pragma unroll
-    for (int x = 0; x < 2; ++x) {
-      if (!keep_tile<C>(p, x ? t1 : t0, b, hkv, u, misc)) continue;
-      if (s_cnt[x] > 0) {  // the softmax must have loaded this tile's previous S
-        if (!(ok = __all_sync(FULL, w.wait(smem_addr(&misc->s_free[x]), (s_cnt[x] - 1) & 1)))) return;
-        tc_fence_after();
-      }
-      if (leader) {
-        issue_qk<C>(tmem + s_col[x], x ? q_lo1 : q_lo0, k_lo0 + ks * (C::SLOT >> 4), hi);
-        tc_commit(smem_addr(&misc->s_full[x]));
-      }
-      __syncwarp();
-      ++s_cnt[x];
+  auto next_kept = [&](int from) { return next_kept_tile<C>(p, misc, 3, from, n_u); };
+  // S_x(u) = Q_x K_u^T into tile x's S columns; K_u lives in slot ks.
+  auto issue_s = [&](int x, int u, int ks) {
+    if (!keep_tile<C>(p, x ? t1 : t0, u, misc)) return;
+    if (s_cnt[x] > 0) {  // the softmax must have loaded this tile's previous S
+      if (!(ok = __all_sync(FULL, w.wait(smem_addr(&misc->s_free[x]), (s_cnt[x] - 1) & 1)))) return;
+      tc_fence_after();
     }
+    if (leader) {
+      issue_qk<C>(tmem + s_col[x], x ? q_lo1 : q_lo0, k_lo0 + ks * (C::SLOT >> 4), hi);
+      tc_commit(smem_addr(&misc->s_full[x]));
+    }
+    __syncwarp();
+    ++s_cnt[x];
+  };
+  // O_x += P_x V (V in slot vsl), once the softmax has written P_x; committed
+  // to pv_done[x].
+  auto issue_pv = [&](int x, int vsl) {
+    if (!(ok = __all_sync(FULL, w.wait(smem_addr(&misc->p_full[x]), pv_cnt[x] & 1)))) return;
+    tc_fence_after();
+    if (leader) {
+      const uint32_t plo = x ? p_lo1 : p_lo0;
+      const uint32_t vlo = v_lo0 + vsl * (C::SLOT >> 4);
+      issue_pv_ss<C>(tmem + o_col[x], plo, vlo, hi, pv_cnt[x] > 0);
+      if constexpr (C::P2) issue_pv_ss<C>(tmem + o_col[x], plo + (C::P_TILE >> 4), vlo, hi, 1u);
+      tc_commit(smem_addr(&misc->pv_done[x]));
+    }
+    __syncwarp();
+    ++pv_cnt[x];
+  };
+  auto release = [&](int slot) {
+    if (leader) tc_commit(smem_addr(&misc->kv_empty[slot]));  // arrives when the MMAs issued so far finish
+    __syncwarp();
   };
   int u = next_kept(min(t0.u0, t1.u0));
   int vs = 0;
@@ -568,49 +583,43 @@ __device__ void attn_mma_role_psmem(const AttnParams& p, const TileInfo t0, cons
     ++slot_it;
     if ((ok = __all_sync(FULL, w.wait(smem_addr(&misc->kv_full[ks]), kph)))) {
       tc_fence_after();
-      issue_s(u, ks);
-      if (leader) tc_commit(smem_addr(&misc->kv_empty[ks]));
-      __syncwarp();
+      issue_s(0, u, ks);
+      if (ok) issue_s(1, u, ks);
+      if (ok) release(ks);
     }
   }
+  // Per kept KV tile u: QK^T of the next kept tile for both query tiles (as
+  // soon as each softmax has loaded its current S), then PV of tile u for
+  // both. (Issuing in the order the two softmax warpgroups release -- tile 1's
+  // PV one tile behind -- was measured 7 % slower with a BF16 QK^T.)
   while (u < n_u && ok) {
-    const int vph_it = slot_it - 1;  // ring position of V_u
-    const uint32_t vph = (vph_it / C::STAGES) & 1;
+    const uint32_t vph = ((slot_it - 1) / C::STAGES) & 1;  // ring phase of V_u (slot vs)
     const int nu = next_kept(u + 1);
-    int nvs = 0;
-    if (nu < n_u) {  // QK^T of the next kept tile, overlapping this tile's softmax
-      const int nks = slot_it % C::STAGES;
+    int nks = 0, nvs = 0;
+    if (nu < n_u) {
+      nks = slot_it % C::STAGES;
       const uint32_t nkph = (slot_it / C::STAGES) & 1;
       ++slot_it;
       nvs = slot_it % C::STAGES;
       ++slot_it;
       if (!(ok = __all_sync(FULL, w.wait(smem_addr(&misc->kv_full[nks]), nkph)))) break;
       tc_fence_after();
-      issue_s(nu, nks);
+      issue_s(0, nu, nks);
+      if (ok) issue_s(1, nu, nks);
       if (!ok) break;
-      if (leader) tc_commit(smem_addr(&misc->kv_empty[nks]));
-      __syncwarp();
+      release(nks);  // K_nu: both S MMAs issued
     }
     if (!(ok = __all_sync(FULL, w.wait(smem_addr(&misc->kv_full[vs]), vph)))) break;
     tc_fence_after();
-#pragma unroll
-    for (int x = 0; x < 2; ++x) {
-      if (!keep_tile<C>(p, x ? t1 : t0, b, hkv, u, misc)) continue;
-      if (!(ok = __all_sync(FULL, w.wait(smem_addr(&misc->p_full[x]), pv_cnt[x] & 1)))) break;
-      tc_fence_after();
-      if (leader) {
-        const uint32_t plo = x ? p_lo1 : p_lo0;
-        const uint32_t vlo = v_lo0 + vs * (C::SLOT >> 4);
-        issue_pv_ss<C>(tmem + o_col[x], plo, vlo, hi, pv_cnt[x] > 0);
-        if constexpr (C::P2) issue_pv_ss<C>(tmem + o_col[x], plo + (C::P_TILE >> 4), vlo, hi, 1u);
-        tc_commit(smem_addr(&misc->pv_done[x]));
-      }
-      __syncwarp();
-      ++pv_cnt[x];
+    if (keep_tile<C>(p, t0, u, misc)) {
+      issue_pv(0, vs);
+      if (!ok) break;
     }
-    if (!ok) break;
-    if (leader) tc_commit(smem_addr(&misc->kv_empty[vs]));
-    __syncwarp();
+    if (keep_tile<C>(p, t1, u, misc)) {
+      issue_pv(1, vs);
+      if (!ok) break;
+    }
+    release(vs);  // V_u: both PV MMAs issued
     u = nu;
     vs = nvs;
   }
@@ -619,20 +628,64 @@ __device__ void attn_mma_role_psmem(const AttnParams& p, const TileInfo t0, cons
   w.drain(smem_addr(&misc->drain), 0);
 }
 
+// 2^x on the FMA pipe, for two values at once ("FlashInfer FP8/BF16
+// mixed-precision attention for Blackwell", section 3: part of the exp2 work
+// moved from MUFU to FMA). x is clamped to [-125, +inf) (results below 2^-125
+// are zero to every P format); n = rint(x) comes from adding 1.5 * 2^23 (the
+// integer lands in the low mantissa bits), f = x - n lies in [-1/2, 1/2],
+// 2^f is a polynomial in f fitted to minimise the relative error on that
+// interval (degree 2: 1.7e-3, degree 3: 7.5e-5), and 2^n is added to the
+// exponent field as an integer (n << 23). Valid for x < 128.
+// Share of a tile's exponentials taken by the polynomial: one group of four
+// scores in kExpPolyEvery (0: none). A standalone exp + pack pass ran 16 %
+// faster with one in four, but in the kernel every such setting measured
+// slower (3-6 % for the E4M3-P modes): the softmax chain, not MUFU, bounds the
+// kernel, and with one E4M3 term the polynomial's rounding differs from MUFU's
+// for the weight the row-sum correction below relies on. Kept selectable.
+constexpr int kExpPolyEvery = 0;
+
+template <int DEG>
+__device__ __forceinline__ void exp2_poly_x2(float& a, float& b) {
+  using namespace ptx;
+  a = fmaxf(a, -125.f);
+  b = fmaxf(b, -125.f);
+  float ja, jb, na, nb, fa, fb, pa, pb;
+  fadd2(ja, jb, a, b, 12582912.f, 12582912.f);
+  fadd2(na, nb, ja, jb, -12582912.f, -12582912.f);
+  fadd2(fa, fb, a, b, -na, -nb);
+  if constexpr (DEG == 3) {
+    ffma2(pa, pb, fa, fb, 0.05517098f, 0.05517098f, 0.24260971f, 0.24260971f);
+    ffma2(pa, pb, pa, pb, fa, fb, 0.69326097f, 0.69326097f);
+    ffma2(pa, pb, pa, pb, fa, fb, 0.99992818f, 0.99992818f);
+  } else {
+    ffma2(pa, pb, fa, fb, 0.23842251f, 0.23842251f, 0.70343643f, 0.70343643f);
+    ffma2(pa, pb, pa, pb, fa, fb, 1.00044274f, 1.00044274f);
+  }
+  a = __int_as_float(__float_as_int(pa) + (__float_as_int(ja) << 23));
+  b = __int_as_float(__float_as_int(pb) + (__float_as_int(jb) << 23));
+}
+
 // --------------------------------------------------------------- softmax ----
-// Per kept KV tile: load S (128 fp32 per row) from TMEM, scale and mask,
-// reduce the row max with three-input max, lazily correct O, exponentiate
-// with packed fp32x2 FMAs feeding MUFU ex2, pack P (BF16 or E4M3) over the
-// first S columns and release it to the MMA warp with one arrive per warp.
+// One thread per query row (TMEM lane = row). Per kept KV tile: load S (128
+// fp32 or s32 per row) from TMEM, scale and mask, exponentiate with packed
+// fp32x2 FMAs feeding MUFU ex2, pack P (BF16 into TMEM over S, or E4M3 into
+// shared memory) and release it to the MMA warp with one arrive per warp.
+//
+// The running row max m is lazy ("FlashInfer FP8/BF16 mixed-precision
+// attention for Blackwell", section 3): it only moves, and O and l are only
+// rescaled, when a tile's max exceeds m by more than tau (log2 units). So for
+// every tile after the first, the exponentials are computed speculatively with
+// the current m while the tile's max is reduced in the same pass; only when
+// some row of the warp crosses m + tau does the warp redo the tile with the
+// new max. The row max is then off the critical chain of a tile.
 template <class C>
-__device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, int h, int b, int hkv,
-                                  uint8_t* sQx, uint8_t* sPx, int n_turns, AttnMisc* misc, uint32_t tmem,
-                                  const CUtensorMap* tmO, const Waiter w) {
+__device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, int b, int hkv, uint8_t* sQx,
+                                  uint8_t* sPx, int n_turns, AttnMisc* misc, uint32_t tmem, const CUtensorMap* tmO,
+                                  const Waiter w) {
   using namespace ptx;
   constexpr uint32_t FULL = 0xffffffffu;
-  // h: which part of each row this thread owns when NH threads share a row:
-  // S columns [32 * NC * h, 32 * NC * (h + 1)), O columns likewise over D.
-  constexpr int NH = C::NH, NC = 4 / NH, OB = C::D / 32 / NH;
+  constexpr int NCH = C::BN / 32;  // 32-key chunks per tile (one TMEM load each)
+  constexpr int OB = C::D / 32;    // 32-column blocks of O
   const int warp = (threadIdx.x >> 5) & 3;  // TMEM lane quadrant of this warp
   const int lane = threadIdx.x & 31;
   const int r = warp * 32 + lane;  // row within the tile
@@ -642,31 +695,7 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, 
   const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
   const uint32_t tS = tmem + lane_off + (x ? 128u : 0u);
   const uint32_t tO = tmem + lane_off + (x ? 256u + C::D : 256u);
-  const int wg_tid = threadIdx.x & 127;
-  const bool lead = wg_tid == 0 && h == 0;  // one thread of the query tile
-  // The two threads of a row meet through one shared-memory slot and the
-  // named barrier of their lane quadrant's two warps (ids 3..10).
-  const uint32_t pair_bar = 3u + 4u * x + warp;
-  // ok_io: in, this thread's wait results; out, the AND over both threads, so
-  // that the two warps of a pair always leave the tile loop together (named
-  // barriers have no time limit: a warp must not wait for a partner that left).
-  auto pair_combine = [&](float v, bool is_max, bool& ok_io) {
-    if constexpr (NH == 1) {
-      return v;
-    } else {
-      float* slot = &misc->xchg[x][r];
-      if (h == 1) *slot = v;
-      ok_io = named_bar_and(pair_bar, 64, ok_io);
-      float res = v;
-      if (h == 0) {
-        res = is_max ? fmaxf(v, *slot) : v + *slot;
-        *slot = res;
-      }
-      named_bar_sync(pair_bar, 64);
-      if (h == 1) res = *slot;
-      return res;
-    }
-  };
+  const bool lead = (threadIdx.x & 127) == 0;  // one thread of the query tile
   const int64_t bhq = static_cast<int64_t>(b) * p.Hq + head;
   const int64_t bhk = static_cast<int64_t>(b) * p.Hkv + hkv;
 
@@ -675,6 +704,7 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, 
   if (C::QK != QK_BF16) cq *= sf_lookup(p.sf_q, p.sf_q_kind, bhq, p.sf_q_nblk, min(row, p.Sq - 1), p.sf_q_rpb);
   const float ck_uniform =
       p.sf_k_kind == FMHA_SF_PER_TOKEN_BLOCK ? 1.f : sf_lookup(p.sf_k, p.sf_k_kind, bhk, 1, 0, 1);
+  const bool ck_blocked = C::QK != QK_BF16 && p.sf_k_kind == FMHA_SF_PER_TOKEN_BLOCK;
 
   // P encoding: E4M3 P holds p * g with g = 1 / sf_p; the lazy-rescale
   // threshold tau keeps the stale-max bound 2^tau * g <= 448. BF16 P: g = 1, tau = 8.
@@ -688,76 +718,76 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, 
     tau = fminf(8.f, fmaxf(0.f, floorf(__log2f(448.f * sfp))));
   }
 
+  // K scale of each 32-key chunk of tile u (token-block K scales).
+  auto load_ck = [&](int u, float (&dst)[NCH]) {
+#pragma unroll
+    for (int c = 0; c < NCH; ++c)
+      dst[c] = (ck_blocked ? __ldg(p.sf_k + bhk * p.sf_k_nblk + min(u * C::BN + 32 * c, p.Skv - 1) / p.sf_k_rpb)
+                           : ck_uniform) * cq;
+  };
+
   float m = -INFINITY;  // running row max (log2 units, scaled)
-  float l = 0.f;        // running row sum of the stored P (times g)
+  float l = 0.f;        // running row sum of P (times g)
   int it = 0;
   bool ok = true;
-  for (int u = t.u0; u < t.n_kv; ++u) {
-    if (!keep_tile<C>(p, t, b, hkv, u, misc)) continue;
-    // A failed wait does not leave the loop here: the exchange below does, for
-    // both threads of the row at once (the work in between is harmless).
+  for (int u = next_kept_tile<C>(p, misc, 1 << t.x, t.u0, t.n_kv); u < t.n_kv;
+       u = next_kept_tile<C>(p, misc, 1 << t.x, u + 1, t.n_kv)) {
+    float ck[NCH];
+    load_ck(u, ck);  // issued before the wait: the loads overlap it
     ok = __all_sync(FULL, w.wait(smem_addr(&misc->s_full[x]), it & 1)) && ok;
+    if (!ok) break;
     tc_fence_after();
+    int lim = p.Skv - u * C::BN;  // keys at or past `lim` in this tile are hidden
+    if (p.causal) lim = min(lim, row + 1 + (p.Skv - p.Sq) - u * C::BN);
 
-    // Column factors: K scale per 32-key chunk (token-block K scales), times cq.
-    const int kv0 = u * C::BN;
-    float ck[NC];
+    // S of this tile into f (fp32 scores; hidden keys -inf).
+    float f[NCH][32];
+    {
+      uint32_t s[NCH][32];
 #pragma unroll
-    for (int c = 0; c < NC; ++c) {
-      float f = ck_uniform;
-      if (C::QK != QK_BF16 && p.sf_k_kind == FMHA_SF_PER_TOKEN_BLOCK)
-        f = p.sf_k[bhk * p.sf_k_nblk + min(kv0 + 32 * (NC * h + c), p.Skv - 1) / p.sf_k_rpb];
-      ck[c] = f * cq;
-    }
-    int lim = p.Skv - kv0;  // keys at or past `lim` in this tile are hidden
-    if (p.causal) lim = min(lim, row + 1 + (p.Skv - p.Sq) - kv0);
-
-    uint32_t s[NC][32];
+      for (int c = 0; c < NCH; ++c) tmem_ld32(tS + 32 * c, s[c]);
+      tmem_wait_ld();
 #pragma unroll
-    for (int c = 0; c < NC; ++c) tmem_ld32(tS + 32 * (NC * h + c), s[c]);
-    tmem_wait_ld();
-#pragma unroll
-    for (int c = 0; c < NC; ++c) reg_fence(s[c]);
-    if constexpr (C::PSMEM) {  // S is in registers: the MMA warp may issue the next QK^T into this tile
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_addr(&misc->s_free[x]));
-    }
-    float f[NC][32];
-#pragma unroll
-    for (int c = 0; c < NC; ++c)
-#pragma unroll
-      for (int j = 0; j < 32; ++j) {
-        if constexpr (C::QK == QK_INT8)
-          f[c][j] = __int_as_float(static_cast<int>(s[c][j]) + 0x4B400000) - 12582912.f;
-        else
-          f[c][j] = __uint_as_float(s[c][j]);
+      for (int c = 0; c < NCH; ++c) reg_fence(s[c]);
+      if constexpr (C::PSMEM) {  // S is in registers: the MMA warp may issue the next QK^T into this tile
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_addr(&misc->s_free[x]));
       }
+      // INT8 scores: s32 s is exact in fp32 (|s| <= 127 * 127 * D < 2^22): one
+      // integer add makes the bits of 1.5 * 2^23 + s, one exact subtraction
+      // (two per packed instruction) removes the offset.
+#pragma unroll
+      for (int c = 0; c < NCH; ++c)
+#pragma unroll
+        for (int j = 0; j < 32; j += 2) {
+          if constexpr (C::QK == QK_INT8)
+            fadd2(f[c][j], f[c][j + 1], __int_as_float(static_cast<int>(s[c][j]) + 0x4B400000),
+                  __int_as_float(static_cast<int>(s[c][j + 1]) + 0x4B400000), -12582912.f, -12582912.f);
+          else
+            f[c][j] = __uint_as_float(s[c][j]), f[c][j + 1] = __uint_as_float(s[c][j + 1]);
+        }
+    }
     if (lim < C::BN) {
 #pragma unroll
-      for (int c = 0; c < NC; ++c)
+      for (int c = 0; c < NCH; ++c)
 #pragma unroll
         for (int j = 0; j < 32; ++j)
-          if (32 * (NC * h + c) + j >= lim) f[c][j] = -INFINITY;
+          if (32 * c + j >= lim) f[c][j] = -INFINITY;
     }
-    float mc[NC];
+
+    // Row max of the tile (ck > 0: the scaled max is the raw max times ck).
+    float m_tile = -INFINITY;
 #pragma unroll
-    for (int c = 0; c < NC; ++c) {
+    for (int c = 0; c < NCH; ++c) {
       float a0 = fmax3(f[c][0], f[c][1], f[c][2]), a1 = fmax3(f[c][3], f[c][4], f[c][5]);
 #pragma unroll
       for (int j = 6; j < 30; j += 4) {
         a0 = fmax3(a0, f[c][j], f[c][j + 1]);
         a1 = fmax3(a1, f[c][j + 2], f[c][j + 3]);
       }
-      mc[c] = fmax3(a0, a1, fmaxf(f[c][30], f[c][31])) * ck[c];
+      m_tile = fmaxf(m_tile, fmax3(a0, a1, fmaxf(f[c][30], f[c][31])) * ck[c]);
     }
-    float m_part = mc[0];
-#pragma unroll
-    for (int c = 1; c < NC; ++c) m_part = fmaxf(m_part, mc[c]);
-    // Both threads of the row have loaded their S columns once they meet here,
-    // so P may overwrite S columns of either part from now on.
-    const float m_tile = pair_combine(m_part, true, ok);
-    if (!ok) break;
     const float m_new = fmaxf(m, m_tile);
     float alpha = 1.f;
     bool resc = false;
@@ -774,133 +804,146 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, 
     auto rescale_o = [&]() {
       if (__any_sync(FULL, resc)) {
 #pragma unroll 1
-        for (int c = 0; c < OB; ++c) {  // this thread's O columns
+        for (int c = 0; c < OB; ++c) {
           uint32_t o[32];
-          tmem_ld32(tO + 32 * (OB * h + c), o);
+          tmem_ld32(tO + 32 * c, o);
           tmem_wait_ld();
           reg_fence(o);
 #pragma unroll
           for (int j = 0; j < 32; ++j) o[j] = __float_as_uint(__uint_as_float(o[j]) * alpha);
-          tmem_st32(tO + 32 * (OB * h + c), o);
+          tmem_st32(tO + 32 * c, o);
         }
       }
     };
     if constexpr (!C::PSMEM) rescale_o();
+    // Row r of the 128 x 128-byte E4M3 P tile in shared memory, 16-byte chunks
+    // XOR-swizzled by r % 8 (the 128-byte swizzle the PV descriptor expects).
+    // (Storing each chunk inside the exp pass was measured 15 % slower: the
+    // stores then compete with the turn's exponentials.)
+    [[maybe_unused]] const uint32_t prow = smem_addr(sPx) + r * 128;
+    [[maybe_unused]] auto store_p = [&](int k, uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3, uint32_t plane) {
+      const uint32_t addr = prow + plane + ((k ^ (r & 7)) << 4);
+      asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(w0), "r"(w1), "r"(w2), "r"(w3)
+                   : "memory");
+    };
+
     // Turn-taking on the exp2 unit: for the first n_turns tiles (both tiles
     // walk the same KV tiles) the warpgroups alternate their exponential
     // phases, so that one exponentiates while the other loads, reduces and
-    // packs. Tile 0 goes first.
-    if (x == 0 ? (it >= 1 && it < n_turns) : (it < n_turns)) {
+    // stores. Tile 0 goes first.
+    if (C::TURNS && (x == 0 ? (it >= 1 && it < n_turns) : (it < n_turns))) {
       ok = __all_sync(FULL, w.wait(smem_addr(&misc->exp_done[x ^ 1]), (x == 0 ? it - 1 : it) & 1)) && ok;
 #pragma unroll
-      for (int c = 0; c < NC; ++c) reg_fence(f[c]);
+      for (int c = 0; c < NCH; ++c) reg_fence(f[c]);
     }
-    const float mb = (m == -INFINITY ? 0.f : m) - log2g;
+
+    // Exponentials, P and its row sum in one pass: per group of scores
+    // 2^(f * ck - mb) (packed FMAs feeding MUFU ex2), packed to BF16 (TMEM)
+    // or E4M3 (registers, for shared memory) as soon as a group is done, so
+    // the conversions and additions fill the issue slots between ex2s.
+    const float nmb = -((m == -INFINITY ? 0.f : m) - log2g);
+    float rs = 0.f;
+    [[maybe_unused]] uint32_t pk[C::PV == PV_E4M3 ? 8 * NCH : 1];
+    [[maybe_unused]] uint32_t pl[C::P2 ? 8 * NCH : 1];
+    if constexpr (C::PV == PV_BF16) {
+      // BF16 P of keys 64q..64q+63 goes over TMEM columns [32q, 32q + 32) of S.
+      float r0 = 0.f, r1 = 0.f, r2 = 0.f, r3 = 0.f;
 #pragma unroll
-    for (int c = 0; c < NC; ++c)
+      for (int q = 0; q < NCH / 2; ++q) {
+        uint32_t p32[32];
 #pragma unroll
-      for (int j = 0; j < 32; j += 2) ffma2(f[c][j], f[c][j + 1], f[c][j], f[c][j + 1], ck[c], ck[c], -mb, -mb);
+        for (int h = 0; h < 2; ++h) {
+          const int c = 2 * q + h;
 #pragma unroll
-    for (int c = 0; c < NC; ++c)
+          for (int j = 0; j < 32; j += 4) {
+            float e0, e1, e2, e3;
+            ffma2(e0, e1, f[c][j], f[c][j + 1], ck[c], ck[c], nmb, nmb);
+            ffma2(e2, e3, f[c][j + 2], f[c][j + 3], ck[c], ck[c], nmb, nmb);
+            e0 = ex2(e0); e1 = ex2(e1); e2 = ex2(e2); e3 = ex2(e3);
+            p32[16 * h + j / 2] = pack_bf16x2(e0, e1);
+            p32[16 * h + j / 2 + 1] = pack_bf16x2(e2, e3);
+            fadd2(r0, r1, r0, r1, e0, e1);
+            fadd2(r2, r3, r2, r3, e2, e3);
+          }
+        }
+        tmem_st32(tS + 32 * q, p32);
+      }
+      rs = (r0 + r1) + (r2 + r3);
+    } else if constexpr (C::P2) {
+      // Two-term E4M3 P: hi = E4M3(p g), lo = E4M3(p g - hi) (the residual taken
+      // in f16), ~7 significant bits between them; both feed their own PV
+      // product. The row sum adds the unrounded values (as precise as BF16 P).
+      // With kExpPolyEvery set, the degree-3 polynomial (well inside the two
+      // terms' precision) takes that share of the exponentials.
+      float r0 = 0.f, r1 = 0.f, r2 = 0.f, r3 = 0.f;
 #pragma unroll
-      for (int j = 0; j < 32; ++j) f[c][j] = ex2(f[c][j]);
-    if (x == 0 ? (it < n_turns) : (it + 1 < n_turns)) {
+      for (int c = 0; c < NCH; ++c)
 #pragma unroll
-      for (int c = 0; c < NC; ++c) reg_fence(f[c]);
+        for (int j = 0; j < 8; ++j) {
+          float e[4];
+          ffma2(e[0], e[1], f[c][4 * j], f[c][4 * j + 1], ck[c], ck[c], nmb, nmb);
+          ffma2(e[2], e[3], f[c][4 * j + 2], f[c][4 * j + 3], ck[c], ck[c], nmb, nmb);
+          if (kExpPolyEvery > 0 && j % kExpPolyEvery == kExpPolyEvery - 1) {
+            exp2_poly_x2<3>(e[0], e[1]);
+            exp2_poly_x2<3>(e[2], e[3]);
+          } else {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) e[q] = ex2(e[q]);
+          }
+          const uint32_t h01 = pack_e4m3x2(e[0], e[1]), h23 = pack_e4m3x2(e[2], e[3]);
+          pk[c * 8 + j] = h01 | (h23 << 16);
+          const uint32_t d01 = hsub2(pack_f16x2(e[0], e[1]), e4m3x2_to_f16x2(h01));
+          const uint32_t d23 = hsub2(pack_f16x2(e[2], e[3]), e4m3x2_to_f16x2(h23));
+          pl[c * 8 + j] = f16x2_to_e4m3x2(d01) | (f16x2_to_e4m3x2(d23) << 16);
+          fadd2(r0, r1, r0, r1, e[0], e[1]);
+          fadd2(r2, r3, r2, r3, e[2], e[3]);
+        }
+      rs = (r0 + r1) + (r2 + r3);
+    } else {
+      // One E4M3 term. The row sum adds the unrounded values (packed adds; the
+      // conversions back from E4M3 cost 3-5 % of the kernel) plus, below, the
+      // rounding error of the tile's largest weight: a dominant key's
+      // normalised weight is then exact, as with a sum of the stored values
+      // (an outlier value otherwise comes back off by up to 2^-4 of itself).
+      // The correction recomputes that weight with the same MUFU ex2, so it is
+      // bit-identical to the stored one; a polynomial exponential would break
+      // that, so this mode always uses MUFU.
+      float r0 = 0.f, r1 = 0.f, r2 = 0.f, r3 = 0.f;
+#pragma unroll
+      for (int c = 0; c < NCH; ++c)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          float e0, e1, e2, e3;
+          ffma2(e0, e1, f[c][4 * j], f[c][4 * j + 1], ck[c], ck[c], nmb, nmb);
+          ffma2(e2, e3, f[c][4 * j + 2], f[c][4 * j + 3], ck[c], ck[c], nmb, nmb);
+          e0 = ex2(e0); e1 = ex2(e1); e2 = ex2(e2); e3 = ex2(e3);
+          pk[c * 8 + j] = pack_e4m3x2(e0, e1) | (pack_e4m3x2(e2, e3) << 16);
+          fadd2(r0, r1, r0, r1, e0, e1);
+          fadd2(r2, r3, r2, r3, e2, e3);
+        }
+      rs = (r0 + r1) + (r2 + r3);
+      if (m_tile != -INFINITY) {
+        const float emax = ex2(m_tile + nmb);
+        rs += e4m3_round(emax) - emax;
+      }
+    }
+    if (C::TURNS && (x == 0 ? (it < n_turns) : (it + 1 < n_turns))) {
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_addr(&misc->exp_done[x]));
     }
-    float rs = 0.f;
-    if constexpr (C::PV == PV_BF16) {
-      // BF16 P of this thread's columns goes over TMEM columns [32 * NC/2 * h, ...)
-      // of S (two values per column); the pair exchange above ordered it after
-      // both threads' S loads.
-      uint32_t pk[NC / 2][32];
-      float r0 = 0.f, r1 = 0.f, r2 = 0.f, r3 = 0.f;
-#pragma unroll
-      for (int c = 0; c < NC; ++c)
-#pragma unroll
-        for (int j = 0; j < 16; ++j) pk[c >> 1][(c & 1) * 16 + j] = pack_bf16x2(f[c][2 * j], f[c][2 * j + 1]);
-#pragma unroll
-      for (int c = 0; c < NC; ++c)
-#pragma unroll
-        for (int j = 0; j < 32; j += 4) {
-          fadd2(r0, r1, r0, r1, f[c][j], f[c][j + 1]);
-          fadd2(r2, r3, r2, r3, f[c][j + 2], f[c][j + 3]);
-        }
-      rs = (r0 + r1) + (r2 + r3);
-#pragma unroll
-      for (int q = 0; q < NC / 2; ++q) tmem_st32(tS + 32 * (NC / 2 * h + q), pk[q]);
-    } else {
-      uint32_t pk[8 * NC];
-      [[maybe_unused]] uint32_t pl[8 * NC];
-      if constexpr (C::P2) {
-        // Two-term E4M3 P: hi = E4M3(p g), lo = E4M3(p g - hi) (the residual taken
-        // in f16), ~7 significant bits between them; both feed their own PV
-        // product. The row sum adds the unrounded values (as precise as BF16 P).
-        float r0 = 0.f, r1 = 0.f, r2 = 0.f, r3 = 0.f;
-#pragma unroll
-        for (int c = 0; c < NC; ++c)
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const float* e = &f[c][4 * j];
-            const uint32_t h01 = pack_e4m3x2(e[0], e[1]), h23 = pack_e4m3x2(e[2], e[3]);
-            pk[c * 8 + j] = h01 | (h23 << 16);
-            const uint32_t d01 = hsub2(pack_f16x2(e[0], e[1]), e4m3x2_to_f16x2(h01));
-            const uint32_t d23 = hsub2(pack_f16x2(e[2], e[3]), e4m3x2_to_f16x2(h23));
-            pl[c * 8 + j] = f16x2_to_e4m3x2(d01) | (f16x2_to_e4m3x2(d23) << 16);
-            fadd2(r0, r1, r0, r1, e[0], e[1]);
-            fadd2(r2, r3, r2, r3, e[2], e[3]);
-          }
-        rs = (r0 + r1) + (r2 + r3);
-      } else {
-        // The row sum adds the E4M3-rounded values actually stored, so the
-        // normalised weights sum to one and a dominant key returns its value.
-        float racc[NC];
-#pragma unroll
-        for (int c = 0; c < NC; ++c) {
-          uint32_t acc[2] = {0u, 0u};
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const uint32_t lo = pack_e4m3x2(f[c][4 * j], f[c][4 * j + 1]);
-            const uint32_t hi = pack_e4m3x2(f[c][4 * j + 2], f[c][4 * j + 3]);
-            pk[c * 8 + j] = lo | (hi << 16);
-            acc[j & 1] = hadd2(acc[j & 1], hadd2(e4m3x2_to_f16x2(lo), e4m3x2_to_f16x2(hi)));
-          }
-          racc[c] = f16x2_sum(acc[0]) + f16x2_sum(acc[1]);
-        }
-        rs = racc[0];
-#pragma unroll
-        for (int c = 1; c < NC; ++c) rs += racc[c];
+    if constexpr (C::PSMEM) {
+      // The previous PV must be done before P (single buffer) or O is rewritten.
+      if (it > 0) {
+        ok = __all_sync(FULL, w.wait(smem_addr(&misc->pv_done[x]), (it - 1) & 1)) && ok;
+        tc_fence_after();
       }
-      if constexpr (C::PSMEM) {
-        // The previous PV must be done before P (single buffer) or O is rewritten.
-        if (it > 0) {
-          ok = __all_sync(FULL, w.wait(smem_addr(&misc->pv_done[x]), (it - 1) & 1)) && ok;
-          tc_fence_after();
-        }
-        rescale_o();
-        // Row r of the 128 x 128-byte P tile, 16-byte chunks XOR-swizzled by r % 8
-        // (the 128-byte swizzle the PV descriptor expects); this thread writes
-        // the chunks of its columns.
-        const uint32_t prow = smem_addr(sPx) + r * 128;
+      rescale_o();
 #pragma unroll
-        for (int kk = 0; kk < 2 * NC; ++kk) {
-          const int k = 2 * NC * h + kk;
-          const uint32_t addr = prow + ((k ^ (r & 7)) << 4);
-          asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[4 * kk]), "r"(pk[4 * kk + 1]),
-                       "r"(pk[4 * kk + 2]), "r"(pk[4 * kk + 3])
-                       : "memory");
-          if constexpr (C::P2)
-            asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr + C::P_TILE), "r"(pl[4 * kk]),
-                         "r"(pl[4 * kk + 1]), "r"(pl[4 * kk + 2]), "r"(pl[4 * kk + 3])
-                         : "memory");
-        }
-        fence_proxy_async_smem();  // generic-proxy P writes -> tensor-core reads
-      } else if constexpr (NH == 1) {  // E4M3 P in TMEM (unused while E4M3 P goes through shared memory)
-        tmem_st32(tS, pk);
-        if constexpr (C::P2) tmem_st32(tS + 32, pl);
+      for (int k = 0; k < 2 * NCH; ++k) {
+        store_p(k, pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3], 0);
+        if constexpr (C::P2) store_p(k, pl[4 * k], pl[4 * k + 1], pl[4 * k + 2], pl[4 * k + 3], C::P_TILE);
       }
+      fence_proxy_async_smem();  // generic-proxy P writes -> tensor-core reads
     }
     l = l * alpha + rs;
     tmem_wait_st();
@@ -921,16 +964,11 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, 
     tc_fence_after();
     have_o = ok;
   }
-  // The row sum of the stored P: the threads of a row add their parts.
-  {
-    bool ok_pair = ok;
-    l = pair_combine(l, false, ok_pair);
-  }
   float sfv = 1.f;
   if (C::PV == PV_E4M3 && p.sf_v_kind != FMHA_SF_PER_CHANNEL) sfv = sf_lookup(p.sf_v, p.sf_v_kind, bhk, 1, 0, 1);
   const float inv_l = l > 0.f ? sfv / l : 0.f;
   const uint32_t stage0 = smem_addr(sQx);
-  constexpr uint32_t TILE_THREADS = 128 * NH;
+  constexpr uint32_t TILE_THREADS = 128;
   if constexpr (C::O8) {
     // E4M3 output: the whole 128-column row is 128 bytes, one swizzled
     // 128 x 128-byte chunk (the size and layout of a 64-column BF16 chunk),
@@ -939,7 +977,6 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, 
     const uint32_t base = stage0 + r * 128;
 #pragma unroll 1
     for (int sc = 0; sc < C::D / 32; ++sc) {
-      if (sc / OB != h) continue;  // warp-uniform: another thread of this row owns these columns
       uint32_t o[32];
       if (have_o) {
         tmem_ld32(tO + 32 * sc, o);
@@ -975,13 +1012,10 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, 
   }
 #pragma unroll 1
   for (int c64 = 0; c64 < (C::O8 ? 0 : C::D / 64); ++c64) {
-    // 32-column blocks of this 64-column chunk held by this thread (its O
-    // columns are [32 * OB * h, 32 * OB * (h + 1))); warp-uniform.
-    const bool mine[2] = {(2 * c64) / OB == h, (2 * c64 + 1) / OB == h};
     uint32_t o[2][32];
     if (have_o) {
-      if (mine[0]) tmem_ld32(tO + 64 * c64, o[0]);
-      if (mine[1]) tmem_ld32(tO + 64 * c64 + 32, o[1]);
+      tmem_ld32(tO + 64 * c64, o[0]);
+      tmem_ld32(tO + 64 * c64 + 32, o[1]);
       tmem_wait_ld();
       reg_fence(o[0]);
       reg_fence(o[1]);
@@ -997,7 +1031,6 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, 
           float* dst = p.o_part + ((((int64_t)t.part * p.B + b) * p.Sq + row) * p.Hq + head) * C::D + 64 * c64;
 #pragma unroll
           for (int j = 0; j < 64; j += 4) {
-            if (!mine[j >> 5]) continue;
             asm volatile("st.global.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst + j), "f"(out_val(j)),
                          "f"(out_val(j + 1)), "f"(out_val(j + 2)), "f"(out_val(j + 3))
                          : "memory");
@@ -1014,7 +1047,6 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, 
     const uint32_t base = stage0 + buf * C::CHUNK_BYTES + r * 128;
 #pragma unroll
     for (int sc = 0; sc < 2; ++sc) {
-      if (!mine[sc]) continue;
       uint32_t pk[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) pk[j] = pack_bf16x2(out_val(32 * sc + 2 * j), out_val(32 * sc + 2 * j + 1));
@@ -1038,15 +1070,14 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, 
     }
   }
   const float lse = l > 0.f ? (m + __log2f(l) - log2g) * 0.69314718055994531f : -INFINITY;
-  if (h == 0) {
-    if (C::PACKED && p.n_parts > 1) {
-      if (row < p.Sq && ok) p.lse_part[(((int64_t)t.part * p.B + b) * p.Hq + head) * p.Sq + row] = lse;
-    } else if (p.lse != nullptr && row < p.Sq && ok) {
-      p.lse[bhq * p.Sq + row] = lse;
-    }
+  if (C::PACKED && p.n_parts > 1) {
+    if (row < p.Sq && ok) p.lse_part[(((int64_t)t.part * p.B + b) * p.Hq + head) * p.Sq + row] = lse;
+  } else if (p.lse != nullptr && row < p.Sq && ok) {
+    p.lse[bhq * p.Sq + row] = lse;
   }
   if (lead) bulk_wait0();
 }
+
 
 // ------------------------------------------------------------------ kernel --
 template <class C>
@@ -1184,20 +1215,41 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       }
       t[x].n_kv = t[x].valid ? n : 0;
     }
+    // Masked launch: warp 2 (otherwise idle) turns each query tile's block-mask
+    // row into the keep-bit set (one coalesced 32-byte read per word), and
+    // records whether both tiles keep the same KV tiles.
+    if (p.mask != nullptr && warp == 2) {
+      const int n_words = (max(t[0].n_kv, t[1].n_kv) + 31) >> 5;
+      bool same = t[0].n_kv == t[1].n_kv;
+      int count = 0;
+      for (int wd = 0; wd < n_words; ++wd) {
+        uint32_t bits[2];
+        for (int x = 0; x < 2; ++x) {
+          const uint8_t* mrow =
+              p.mask + b * p.mask_sb + hkv * p.mask_sh + static_cast<int64_t>(t[x].mrow) * p.n_kv_blocks;
+          const int u = (wd << 5) + lane;
+          bits[x] = __ballot_sync(0xffffffffu, u < t[x].n_kv && mrow[u] != 0);
+          if (lane == 0) misc->keep_bits[x][wd] = bits[x];
+        }
+        same = same && bits[0] == bits[1];
+        count += __popc(bits[0]);
+      }
+      if (lane == 0) misc->same_kept = same ? count : 0;
+    }
   }
 
   if (threadIdx.x == 0) {
     mbar_init(smem_addr(&misc->q_full), 1);
     for (int x = 0; x < 2; ++x) {
       mbar_init(smem_addr(&misc->s_full[x]), 1);
-      mbar_init(smem_addr(&misc->p_full[x]), 4 * C::NH);  // one arrive per softmax warp
+      mbar_init(smem_addr(&misc->p_full[x]), 4);  // one arrive per softmax warp
     }
     mbar_init(smem_addr(&misc->o_full), 1);
     mbar_init(smem_addr(&misc->drain), 1);
     for (int x = 0; x < 2; ++x) {
-      mbar_init(smem_addr(&misc->s_free[x]), 4 * C::NH);  // one arrive per softmax warp
+      mbar_init(smem_addr(&misc->s_free[x]), 4);  // one arrive per softmax warp
       mbar_init(smem_addr(&misc->pv_done[x]), 1);
-      mbar_init(smem_addr(&misc->exp_done[x]), 4 * C::NH);  // one arrive per softmax warp
+      mbar_init(smem_addr(&misc->exp_done[x]), 4);  // one arrive per softmax warp
     }
     for (int s = 0; s < C::STAGES; ++s) {
       mbar_init(smem_addr(&misc->kv_full[s]), 1);
@@ -1235,17 +1287,17 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     }
   }
 
-  if (warp >= C::SOFTMAX_WARP0 && warp < C::SOFTMAX_WARP0 + 8 * C::NH) {
+  if (warp >= C::SOFTMAX_WARP0) {
     regs_inc<C::SOFTMAX_REGS>();
-    const int x = (warp - C::SOFTMAX_WARP0) / (4 * C::NH);     // query tile
-    const int h = ((warp - C::SOFTMAX_WARP0) >> 2) % C::NH;   // part of each row
+    const int x = (warp - C::SOFTMAX_WARP0) >> 2;  // query tile
     const TileInfo tx = x ? t[1] : t[0];  // select by value (no runtime-indexed array)
-    // Exp turn-taking needs both tiles to walk the same KV tiles (dense masks:
-    // prefixes [0, n_kv)); with a block mask the lists differ, so it is off.
+    // Exp turn-taking needs both tiles to walk the same KV tiles: without a
+    // mask their common prefix [0, min n_kv); with a block mask only when both
+    // tiles keep the same tiles (e.g. two query heads of one KV head).
     int n_turns = 0;
-    if (C::TURNS && !C::PACKED && p.mask == nullptr) n_turns = min(t[0].n_kv, t[1].n_kv);
+    if (C::TURNS && !C::PACKED) n_turns = p.mask == nullptr ? min(t[0].n_kv, t[1].n_kv) : misc->same_kept;
     if (tx.valid)
-      attn_softmax_role<C>(p, tx, x, h, b, hkv, x ? sQ[1] : sQ[0], x ? sP[1] : sP[0], n_turns, misc, tmem, &tmO,
+      attn_softmax_role<C>(p, tx, x, b, hkv, x ? sQ[1] : sQ[0], x ? sP[1] : sP[0], n_turns, misc, tmem, &tmO,
                            w);
   } else {
     regs_dec<C::CONTROL_REGS>();

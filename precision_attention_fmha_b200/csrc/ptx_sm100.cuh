@@ -349,7 +349,7 @@ __device__ __forceinline__ void fadd2(float& d0, float& d1, float a0, float a1, 
       : "f"(a0), "f"(a1), "f"(b0), "f"(b1));
 }
 // Register-fence helpers for the smaller TMEM loads / stores.
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
   asm volatile(
       "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
       "%15, %16};" ::"r"(taddr),
@@ -357,7 +357,7 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
       "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
       : "memory");
 }
-__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t* r) {
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8]) {
   asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
                "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
                : "memory");
@@ -385,6 +385,13 @@ __device__ __forceinline__ uint32_t f16x2_to_e4m3x2(uint32_t v) {
 __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t v) {
   uint32_t r;
   asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(r) : "h"(static_cast<uint16_t>(v)));
+  return r;
+}
+// x rounded to E4M3 (nearest even, saturating) and back to fp32, exact.
+__device__ __forceinline__ float e4m3_round(float x) {
+  const uint32_t h = e4m3x2_to_f16x2(pack_e4m3x2(x, 0.f));
+  float r;
+  asm("{\n\t.reg .f16 a, b;\n\tmov.b32 {a, b}, %1;\n\tcvt.f32.f16 %0, a;\n\t}" : "=f"(r) : "r"(h));
   return r;
 }
 __device__ __forceinline__ uint32_t hadd2(uint32_t a, uint32_t b) {

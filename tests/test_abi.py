@@ -174,3 +174,21 @@ def test_k_smoothing_entry_points_on_host(lib):
     assert g(ctypes.byref(src), None, ctypes.byref(dst), ctypes.byref(sf), 2, 300, 3, 128, None, 0, None) == 1
     assert g(ctypes.byref(src), 0x40004, ctypes.byref(dst), ctypes.byref(sf), 2, 300, 3, 128, None, 0, None) == 1
     assert g(ctypes.byref(src), 0x40000, ctypes.byref(dst), ctypes.byref(sf), 0, 300, 3, 128, None, 0, None) == 0
+
+
+def test_masked_launch_limits_key_blocks(lib):
+    """A block mask needs Skv <= 131072 (the CTA's 1024-bit keep set); without a mask there is no limit."""
+    a = _args()
+    a.Skv = 131072 + 1
+    for t in (a.k, a.v):
+        t.stride_b = a.Skv * a.Hkv * a.D
+    assert lib.fmha_fwd_block_sparse(ctypes.byref(a), 0x40000, 0, 0, None) == 2
+    assert "131072" in lib.fmha_last_error_message().decode()
+
+
+def test_quantizer_grid_limit_on_host(lib):
+    x = fmha._Tensor(0x10000, fmha.BF16, 0, 70000 * 8 * 128, 70000 * 128, 128)
+    y = fmha._Tensor(0x20000, fmha.INT8, 0, 70000 * 8 * 128, 70000 * 128, 128)
+    sf = fmha._Sf(0x30000, 3, 64)
+    assert lib.fmha_quantize_blockwise(ctypes.byref(x), ctypes.byref(y), ctypes.byref(sf), 1, 8, 70000, 128,
+                                       None, 0, None) == 2
