@@ -117,6 +117,13 @@ def all_fp8(S=8192, B=2, H=32, D=128):
     return dict(q=q, k=k, v=v, scale=1.0 / math.sqrt(D))
 
 
+# P scale of the Sage workload's one-term E4M3 P, per 128-row query block: P is
+# stored as 224 p. With the lazy-rescale threshold it implies (tau = 1: the row
+# max may grow by 2x before O is rescaled) a stored P stays <= 448, and small
+# weights keep 3.8 more binades above E4M3's subnormal range than with 1/16.
+SAGE_SF_P = 1.0 / 224
+
+
 def sage(S=16384, B=1, H=24, D=128):
     q, k, v = biased_qk_v(SEED_BASE + 4 + S, B, S, H, D)
     return dict(q=q, k=k, v=v, scale=1.0 / math.sqrt(D))

@@ -16,13 +16,6 @@ import torch
 BF16_ATOL = 1e-2
 Q8_ATOL = 3e-2
 Q8_COS = 0.999
-# One E4M3 term of P on a sharp softmax (the Sage workload's biased scores):
-# each weight keeps a relative rounding error of up to 2^-4 that a few
-# dominant keys do not average out. Measured on the full-size Sage workload:
-# max-abs 0.066 at max|O| 1.57 (4.2 %), cos >= 0.99969 per head. Such a case
-# is held to the binding cosine and to max-abs <= 2^-4 x max(1, max|O_ref|);
-# two E4M3 terms meet the 3e-2 bound.
-Q8_ONE_TERM_ATOL = 2.0 ** -4
 
 
 def f64(t):

@@ -22,7 +22,7 @@ from oracle import e4m3 as oe
 from oracle import quant as oq
 from precision_attention_fmha_b200 import fmha, workloads
 from precision_attention_fmha_b200.fmha import Scale
-from tests.helpers import BF16_ATOL, Q8_ATOL, Q8_COS, Q8_ONE_TERM_ATOL, codes_np, cos_per_head, f32, f64
+from tests.helpers import BF16_ATOL, Q8_ATOL, Q8_COS, codes_np, cos_per_head, f32, f64
 
 pytestmark = [pytest.mark.gpu, pytest.mark.big]
 DEV = torch.device("cuda")
@@ -156,9 +156,8 @@ def test_sage_full_size(p_terms):
     B, S, H, D = w["q"].shape
     spec = {"q": ("int8", "per_token_block", 128), "k": ("int8", "per_token_block", 64),
             "v": ("e4m3", "per_channel", None)}
-    sf_p = Scale(torch.full((B, H, math.ceil(S / 128)), 1.0 / 16, device=DEV), "per_token_block", 128)
-    run_case("sage", w["q"], w["k"], w["v"], spec, heads=[(0, 0), (0, 11), (0, 23)], sf_p=sf_p, p_terms=p_terms,
-             atol=Q8_ONE_TERM_ATOL if p_terms == 1 else Q8_ATOL)
+    sf_p = Scale(torch.full((B, H, math.ceil(S / 128)), workloads.SAGE_SF_P, device=DEV), "per_token_block", 128)
+    run_case("sage", w["q"], w["k"], w["v"], spec, heads=[(0, 0), (0, 11), (0, 23)], sf_p=sf_p, p_terms=p_terms)
 
 
 def test_sparse_paged_full_size():

@@ -17,7 +17,7 @@ from oracle import attention as oa
 from oracle import quant as oq
 from precision_attention_fmha_b200 import fmha, workloads
 from precision_attention_fmha_b200.fmha import Scale
-from tests.helpers import Q8_ATOL, Q8_ONE_TERM_ATOL, assert_close_bf16, assert_close_q8, codes_np, f32, f64
+from tests.helpers import Q8_ATOL, assert_close_bf16, assert_close_q8, codes_np, f32, f64
 
 pytestmark = pytest.mark.gpu
 DEV = torch.device("cuda")
@@ -77,8 +77,8 @@ def run_dense(mode, B, Hq, Hkv, Sq, Skv, D, causal, seed, with_lse=False, p_term
     scale = 1 / math.sqrt(D)
     lse = torch.full((B, Hq, Sq), float("nan"), device=DEV) if with_lse else None
     sf_p = None
-    if mode == "sage":  # per-row-block P scale: P is stored as 16 p (lazy-rescale bound 2^4 * 16 <= 448)
-        sf_p = Scale(torch.full((B, Hq, math.ceil(Sq / 128)), 1 / 16, device=DEV), "per_token_block", 128)
+    if mode == "sage":  # per-row-block P scale: P is stored as 224 p (lazy-rescale bound 2^1 * 224 <= 448)
+        sf_p = Scale(torch.full((B, Hq, math.ceil(Sq / 128)), workloads.SAGE_SF_P, device=DEV), "per_token_block", 128)
     if p_terms is None:
         p_terms = 1
     o = fmha.fmha_fwd(g["q"], g["k"], g["v"], sf_q=g["sf_q"], sf_k=g["sf_k"], sf_v=g["sf_v"], sf_p=sf_p,
@@ -126,16 +126,13 @@ def test_bf16(B, Hq, Hkv, Sq, Skv, D, causal):
                                                   (700, 1500, False, 4, 2), (129, 129, True, 1, 1)])
 def test_8bit_modes(mode, Sq, Skv, causal, Hq, Hkv):
     """One E4M3 term of P (the precision every 8-bit workload states), whole heads."""
-    run_dense(mode, 1, Hq, Hkv, Sq, Skv, 128, causal, seed=7 * Sq + Skv, with_lse=True,
-              atol=Q8_ONE_TERM_ATOL if mode == "sage" else Q8_ATOL)
+    run_dense(mode, 1, Hq, Hkv, Sq, Skv, 128, causal, seed=7 * Sq + Skv, with_lse=True)
 
 
 @pytest.mark.parametrize("Sq,Skv,causal", [(2048, 2048, False), (4096, 4096, False), (4096, 4096, True)])
 def test_sage_one_term_p_longer(Sq, Skv, causal):
-    """One-term Sage on longer rows: its biased scores sharpen the softmax as Skv grows, and
-    the E4M3 rounding of a few dominant weights shows in max-abs (cosine stays binding)."""
-    run_dense("sage", 1, 2, 2, Sq, Skv, 128, causal, seed=3 * Sq + 11, with_lse=True, p_terms=1,
-              atol=Q8_ONE_TERM_ATOL)
+    """One-term Sage on longer rows: its biased scores sharpen the softmax as Skv grows."""
+    run_dense("sage", 1, 2, 2, Sq, Skv, 128, causal, seed=3 * Sq + 11, with_lse=True, p_terms=1)
 
 
 @pytest.mark.parametrize("Sq,Skv,causal,Hq,Hkv", [(300, 300, False, 2, 2), (1024, 1024, True, 2, 2),

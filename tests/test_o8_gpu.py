@@ -45,8 +45,8 @@ def _inputs(mode, B, Hq, Hkv, Sq, Skv, D, seed):
 def _extra(mode, B, Hq, Sq):
     if mode != "sage":
         return {}
-    sf_p = Scale(torch.full((B, Hq, math.ceil(Sq / 128)), 1 / 16, device=DEV), "per_token_block", 128)
-    return {"sf_p": sf_p, "p_terms": 2}
+    sf_p = Scale(torch.full((B, Hq, math.ceil(Sq / 128)), workloads.SAGE_SF_P, device=DEV), "per_token_block", 128)
+    return {"sf_p": sf_p, "p_terms": 1}
 
 
 def check_o8(codes, sf_o, ref, mode):

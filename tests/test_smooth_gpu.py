@@ -97,7 +97,9 @@ def test_quantize_smoothed_matches_oracle_pipeline():
 
 
 def _sage_attention(q, k, v, smooth, causal):
-    """GPU Sage path (INT8 Q/K, E4M3 per-channel V, two-term P) and its oracle operands."""
+    """GPU Sage path (INT8 Q/K, E4M3 per-channel V) and its oracle operands. P is split
+    into two E4M3 terms here: the comparison with and without smoothing measures the INT8
+    K error, so the P rounding noise is kept well below it."""
     qc, qs = fmha.fmha_quantize_blockwise(q.to(DEV), torch.int8, "per_token_block", 128)
     if smooth:
         shift = oq.channel_mean(f32(k))
@@ -108,7 +110,7 @@ def _sage_attention(q, k, v, smooth, causal):
         kc, ks = fmha.fmha_quantize_blockwise(k.to(DEV), torch.int8, "per_token_block", 64)
     vc, vs = fmha.fmha_quantize_blockwise(v.to(DEV), torch.float8_e4m3fn, "per_channel")
     B, Sq, Hq, D = q.shape
-    sf_p = Scale(torch.full((B, Hq, math.ceil(Sq / 128)), 1 / 16, device=DEV), "per_token_block", 128)
+    sf_p = Scale(torch.full((B, Hq, math.ceil(Sq / 128)), workloads.SAGE_SF_P, device=DEV), "per_token_block", 128)
     o = fmha.fmha_fwd(qc, kc, vc, sf_q=Scale(qs, "per_token_block", 128), sf_k=Scale(ks, "per_token_block", 64),
                       sf_v=Scale(vs, "per_channel", 0), sf_p=sf_p, softmax_scale=1 / math.sqrt(D),
                       causal=causal, p_terms=2)
