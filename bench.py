@@ -282,9 +282,12 @@ def roofline(W, args, attn_ms, achieved_tflops):
                 "frac": round(gbs / hbm, 4), "traffic": TRAFFIC.get(args.workload),
                 "peak_note": f"{src}: HBM copy bandwidth", "algorithmic_bytes": int(W.hbm_bytes),
                 "kernel": "attn_fwd_kernel (packed, split-KV) + split_merge_kernel", "kernel_ms": round(attn_ms, 4)}
-    return {"bound": "tensor", "achieved": round(achieved_tflops, 2), "peak": round(W.peak, 1), "unit": "TFLOP/s",
-            "frac": round(achieved_tflops / W.peak, 4), "traffic": TRAFFIC.get(args.workload),
+    r = {"bound": "tensor", "achieved": round(achieved_tflops, 2), "peak": round(W.peak, 1), "unit": "TFLOP/s",
+         "frac": round(achieved_tflops / W.peak, 4), "traffic": TRAFFIC.get(args.workload),
             "peak_note": f"{W.peak_src}: {W.peak_note}", "kernel": "attn_fwd_kernel", "kernel_ms": round(attn_ms, 4)}
+    if args.workload == "dense_pv8_s32768":
+        r["traffic_note"] = "ncu DRAM bytes of the S = 16384 launch times two (all tensors scale with S)"
+    return r
 
 
 def run_nvfp4(args):
@@ -470,15 +473,17 @@ def run_ours(args):
 
 
 # DRAM bytes (read + write) of one attention launch from an ncu capture of the
-# same kernel build, per workload (None until captured for the current kernel):
-#   ncu --metrics dram__bytes_read.sum,dram__bytes_write.sum,gpu__time_duration.sum
-#       --clock-control none -k regex:attn_fwd -s 1 -c 1
-#       python bench.py [--workload W] --steps 1 --warmup 1 --no-cpu-baseline
-# (one pass; summary in profiles/attn_fwd_pv8_dram_traffic.md).
+# current kernel, per workload (None when not captured for it):
+#   ncu --set full --clock-control none -k regex:attn_fwd -s 3 -c 1
+#       python bench.py --workload W --steps 1 --warmup 3 --no-cpu-baseline
+# The default S = 32768 launch is the S = 16384 capture times two (every tensor the
+# launch moves doubles with S); profiles/attn_fwd_pv8_dram_traffic.md has the numbers.
 TRAFFIC = {
-    "dense_pv8_s32768": 847.74e6 + 315.64e6,  # compulsory: Q,K 335.5 MB + V 167.8 MB read, O 335.5 MB written
-    "dense_pv8_s16384": 420.76e6 + 145.64e6,
-    "decode_paged_s16384": 69.25e6 + 0.89e6 + 1.08e6,  # attention (kept K/V read once) + split merge
+    "dense_pv8_s32768": 2 * (421.13e6 + 151.15e6),  # scaled from the S = 16384 capture
+    "dense_pv8_s16384": 421.13e6 + 151.15e6,
+    "all_fp8_s8192": 201.48e6 + 106.56e6,
+    "sage_s16384": 151.20e6 + 71.45e6,
+    "sparse_paged_s16384": 1344.55e6 + 1042.80e6,
 }
 
 
