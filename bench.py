@@ -48,6 +48,10 @@ WORKLOADS = {
     "sage_s16384": ("sage", 1, 24, 24, 16384, 128, False),
     # the same with P split into two E4M3 terms (about 7 significant bits, twice the PV work)
     "sage_p2_s16384": ("sage_p2", 1, 24, 24, 16384, 128, False),
+    # a 192-wide Q/K head dim with a 128-wide V / O (flops 2·B·H·Sq·Skv·(192 + 128))
+    "wide_qk_bf16_s16384": ("wide_bf16", 1, 40, 40, 16384, 192, False),
+    "wide_qk_pv8_s16384": ("wide_pv8", 1, 40, 40, 16384, 192, False),
+    "wide_qk_fp8_s16384": ("wide_fp8", 1, 40, 40, 16384, 192, False),
     "sparse_paged_s16384": ("sparse_paged", 4, 64, 8, 16384, 128, False),
     # the same mask, Q and K/V values with K/V contiguous [B, S, Hkv, D] (the paged-overhead control)
     "sparse_contig_s16384": ("sparse_contig", 4, 64, 8, 16384, 128, False),
@@ -183,6 +187,21 @@ class Work:
                          "mask": w["mask"]}
             self.peak, self.peak_note, self.dtype = bf16_peak, "bf16 burst", "bf16"
             self.quant = []
+        elif kind in ("wide_bf16", "wide_pv8", "wide_fp8"):
+            w = workloads.wide_qk(S=S, B=B, H=Hq, D=D, outliers=kind == "wide_fp8")
+            self.host = {n: w[n] for n in ("q", "k", "v")}
+            if kind == "wide_bf16":
+                self.peak, self.peak_note, self.dtype = bf16_peak, "bf16 burst", "bf16"
+                self.quant = []
+            elif kind == "wide_pv8":  # QK^T carries 192 / 320 of the flops
+                self.peak = 1.0 / (0.6 / bf16_peak + 0.4 / (2.0 * bf16_peak))
+                self.peak_note = (f"bf16 burst {bf16_peak} for QK^T, 2x (nominal E4M3 ratio) for PV, "
+                                  "flop-weighted 192:128")
+                self.dtype = "bf16,e4m3"
+                self.quant = [("v", E4, "per_tensor", None)]
+            else:
+                self.peak, self.peak_note, self.dtype = 2.0 * bf16_peak, f"2 x bf16 burst {bf16_peak} (nominal E4M3 ratio)", "e4m3"
+                self.quant = [("q", E4, "per_head", None), ("k", E4, "per_head", None), ("v", E4, "per_head", None)]
         elif kind == "sparse_contig":
             w = workloads.sparse_paged(S=S, B=B, Hq=Hq, Hkv=Hkv, D=D)
             self.host = {"q": w["q"], "k": w["k"], "v": w["v"], "mask": w["mask"]}
@@ -193,7 +212,8 @@ class Work:
         self.dev_in = {n: t.to(dev) for n, t in self.host.items()}
         self.Sq = self.host["q"].shape[1]
         self.o8 = kind == "pv8_o8"
-        self.o = torch.empty((B, self.Sq, Hq, D), dtype=E4 if self.o8 else torch.bfloat16, device=dev)
+        self.Dv = self.host["v_pool" if "v_pool" in self.host else "v"].shape[3]
+        self.o = torch.empty((B, self.Sq, Hq, self.Dv), dtype=E4 if self.o8 else torch.bfloat16, device=dev)
         # density = kept score elements / (Sq * Skv)
         self.ws = None
         if kind in ("sparse_paged", "sparse_contig"):
@@ -213,13 +233,14 @@ class Work:
             self.n_parts = fmha.decode_num_parts(self.q_dev, self.dev_in["k_pool"], S)
         else:
             self.density = (S + 1) / (2 * S) if causal else 1.0
-            self.flop = 4.0 * B * Hq * S * S * D * self.density
+            self.flop = 2.0 * B * Hq * S * S * (D + self.Dv) * self.density
         self.qbuf = {}
         for name, dt, gran, rpb in self.quant:
             x = self.dev_in[name]
-            shp = fmha.scale_shape(gran, B, S, x.shape[2], D, rpb)
+            xd = x.shape[3]
+            shp = fmha.scale_shape(gran, B, S, x.shape[2], xd, rpb)
             self.qbuf[name] = (torch.empty(x.shape, dtype=dt, device=dev), torch.empty(shp, dtype=torch.float32,
-                               device=dev), torch.empty(max(4, fmha.quantize_workspace_bytes(gran, B, S, x.shape[2], D)),
+                               device=dev), torch.empty(max(4, fmha.quantize_workspace_bytes(gran, B, S, x.shape[2], xd)),
                                                         dtype=torch.uint8, device=dev), gran, rpb, dt)
         # bytes one step reads: all inputs, or for decode the kept K/V blocks
         touched = (self.hbm_bytes if kind == "decode_paged"
@@ -265,12 +286,14 @@ class Work:
     def config(self, world):
         c = {"workload": self.name, "B": self.B,
              "Hq": self.Hq,
-             "Hkv": self.Hkv, "Sq": self.Sq, "Skv": self.S, "D": self.D, "causal": self.causal,
+             "Hkv": self.Hkv, "Sq": self.Sq, "Skv": self.S, "D": self.D, "Dv": self.Dv, "causal": self.causal,
              "density": round(self.density, 6),
              "quantized_in_step": [f"{n}:{g}" for n, _, g, _ in self.quant], "p_terms": self.p_terms,
              "l2": "inputs fit in L2: flushed before each step (512 MiB write, outside the timed events)"
                    if self.fits_l2 else "inputs larger than L2",
              "parallelism": f"replicas{world}"}
+        if self.Dv != self.D:
+            c["flops"] = "2·B·H·Sq·Skv·(D + Dv)·density (the metric's 4·…·D when D = Dv)"
         return c
 
 
@@ -284,7 +307,7 @@ def roofline(W, args, attn_ms, achieved_tflops):
                 "kernel": "attn_fwd_kernel (packed, split-KV) + split_merge_kernel", "kernel_ms": round(attn_ms, 4)}
     r = {"bound": "tensor", "achieved": round(achieved_tflops, 2), "peak": round(W.peak, 1), "unit": "TFLOP/s",
          "frac": round(achieved_tflops / W.peak, 4), "traffic": TRAFFIC.get(args.workload),
-            "peak_note": f"{W.peak_src}: {W.peak_note}", "kernel": "attn_fwd_kernel", "kernel_ms": round(attn_ms, 4)}
+         "peak_note": f"{W.peak_src}: {W.peak_note}", "kernel": "attn_fwd_kernel", "kernel_ms": round(attn_ms, 4)}
     if args.workload == "dense_pv8_s32768":
         r["traffic_note"] = "ncu DRAM bytes of the S = 16384 launch times two (all tensors scale with S)"
     return r
@@ -528,7 +551,9 @@ def oracle_sample(host, kind, B, Hq, Hkv, S, D, causal, rows):
         spec = {"bf16": {}, "pv8": {"v": ("e4m3", "per_tensor", None)}, "pv8_o8": {"v": ("e4m3", "per_tensor", None)},
                 "fp8": {n: ("e4m3", "per_head", None) for n in "qkv"},
                 "sage": {"q": ("int8", "per_token_block", 128), "k": ("int8", "per_token_block", 64),
-                         "v": ("e4m3", "per_channel", None)}}[kind if kind != "sage_p2" else "sage"]
+                         "v": ("e4m3", "per_channel", None)}}
+        spec["wide_bf16"], spec["wide_pv8"], spec["wide_fp8"] = spec["bf16"], spec["pv8"], spec["fp8"]
+        spec = spec[kind if kind != "sage_p2" else "sage"]
         ops = {"q": q32, "k": k32, "v": v32}
         for n, (dt, g, rpb) in spec.items():
             c, sc = oq.quantize_blockwise(ops[n], dt, g, rpb)
@@ -542,7 +567,7 @@ def oracle_sample(host, kind, B, Hq, Hkv, S, D, causal, rows):
     dt = time.perf_counter() - t
     dens = ((Sq + 1) / (2 * Sq)) if causal else (float(mask.sum()) * 128 * 128 / (Sq * S) if mask is not None else 1.0)
     keys = Sq if causal else S
-    return dt, 4.0 * Sq * keys * D * min(1.0, dens)
+    return dt, 2.0 * Sq * keys * (D + v.shape[3]) * min(1.0, dens)
 
 
 def cpu_cores():
@@ -575,7 +600,10 @@ def run_reference(args):
            "sage_p2": lambda: workloads.sage(S=S, B=B, H=Hq, D=D),
            "sparse_paged": lambda: workloads.sparse_paged(S=S, B=B, Hq=Hq, Hkv=Hkv, D=D),
            "sparse_contig": lambda: workloads.sparse_paged(S=S, B=B, Hq=Hq, Hkv=Hkv, D=D),
-           "decode_paged": lambda: workloads.decode_paged(S=S, B=B, Hq=Hq, Hkv=Hkv, D=D)}[kind]
+           "decode_paged": lambda: workloads.decode_paged(S=S, B=B, Hq=Hq, Hkv=Hkv, D=D),
+           "wide_bf16": lambda: workloads.wide_qk(S=S, B=B, H=Hq, D=D),
+           "wide_pv8": lambda: workloads.wide_qk(S=S, B=B, H=Hq, D=D),
+           "wide_fp8": lambda: workloads.wide_qk(S=S, B=B, H=Hq, D=D, outliers=True)}[kind]
     host = gen()
     rows = 256
     for _ in range(args.warmup):

@@ -140,7 +140,8 @@ typedef struct {
                       bits); 2 = P split into two E4M3 terms hi + lo, each fed to
                       its own PV product (about 7 significant bits, twice the PV
                       tensor work). Must be 0 or 1 when V is BF16. */
-  int32_t reserved; /* must be 0 */
+  int32_t Dv;       /* head dim of V and O; 0 = D. Differs from D only for
+                       D = 192 (QK) with Dv = 128 (V, O). */
   fmha_sf sf_o;     /* o of dtype E4M3 only: PER_TENSOR dequantization multiplier
                        of the output, O ~= code * sf_o[0], or NONE (= 1.0). Must
                        be NONE for a BF16 o. */

@@ -32,6 +32,8 @@ cudaError_t launch_attention_fp8(int, bool, const AttnParams&, const CUtensorMap
                                  const CUtensorMap&, const CUtensorMap&, cudaStream_t);
 cudaError_t launch_attention_sage(int, bool, const AttnParams&, const CUtensorMap&, const CUtensorMap&,
                                   const CUtensorMap&, const CUtensorMap&, cudaStream_t);
+cudaError_t launch_attention_d192(int qk, int pv, bool paged, const AttnParams&, const CUtensorMap&,
+                                  const CUtensorMap&, const CUtensorMap&, const CUtensorMap&, cudaStream_t);
 
 cudaError_t launch_attention(int qk_kind, int pv_kind, int D, bool paged, const AttnParams& p,
                              const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
@@ -262,7 +264,10 @@ fmha_status run_attention(const fmha_args* a, const uint8_t* mask, int64_t msb, 
   if (B < 0 || Hq < 0 || Hkv < 0 || Sq < 0 || Skv < 0) return fail(FMHA_ERR_INVALID_ARG, "negative size");
   if (B == 0 || Hq == 0 || Sq == 0) return ok_status();  // nothing to compute
   if (Hkv == 0 || Hq % Hkv != 0) return fail(FMHA_ERR_INVALID_ARG, "Hq (%d) must be a multiple of Hkv (%d)", Hq, Hkv);
-  if (D != 64 && D != 128) return fail(FMHA_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128)", D);
+  if (D != 64 && D != 128 && D != 192) return fail(FMHA_ERR_UNSUPPORTED, "head dim %d (supported: 64, 128, 192)", D);
+  const int Dv = a->Dv == 0 ? D : a->Dv;  // head dim of V and O
+  if (D == 192 ? Dv != 128 : Dv != D)
+    return fail(FMHA_ERR_UNSUPPORTED, "V / O head dim %d with QK head dim %d (supported: equal, or 192 / 128)", Dv, D);
 
   // dtype tuple
   int qk, pv;
@@ -278,9 +283,11 @@ fmha_status run_attention(const fmha_args* a, const uint8_t* mask, int64_t msb, 
   if (!tuple_ok || (dout != FMHA_BF16 && dout != FMHA_E4M3))
     return fail(FMHA_ERR_UNSUPPORTED, "dtype tuple (q %d, k %d, v %d, o %d) unsupported", dq, dk, dv, dout);
   if (D == 64 && !(qk == QK_BF16 && pv == PV_BF16)) return fail(FMHA_ERR_UNSUPPORTED, "D=64 needs BF16 Q/K/V");
+  if (D == 192 && (qk == QK_INT8 || dout != FMHA_BF16 || a->p_terms == 2 || dec != nullptr))
+    return fail(FMHA_ERR_UNSUPPORTED, "D=192: BF16 or E4M3 Q/K, one-term P, BF16 O, not decode");
   const bool packed = dec != nullptr;
   const bool o8 = dout == FMHA_E4M3;
-  if (o8 && D != 128) return fail(FMHA_ERR_UNSUPPORTED, "E4M3 O needs D = 128");
+  if (o8 && Dv != 128) return fail(FMHA_ERR_UNSUPPORTED, "E4M3 O needs D = 128");
   if (o8 && packed) return fail(FMHA_ERR_UNSUPPORTED, "decode: O must be BF16");
   const int group = Hq / Hkv;
   int group_shift = 0;
@@ -302,14 +309,13 @@ fmha_status run_attention(const fmha_args* a, const uint8_t* mask, int64_t msb, 
   if ((st = check_sf(a->sf_v, "sf_v", v8, v8, false, 1, v8)) != FMHA_OK) return st;
   if ((st = check_sf(a->sf_p, "sf_p", false, v8, v8, 128, false)) != FMHA_OK) return st;
   if ((st = check_sf(a->sf_o, "sf_o", false, o8, false, 1, false)) != FMHA_OK) return st;
-  if (a->reserved != 0) return fail(FMHA_ERR_INVALID_ARG, "args.reserved must be 0");
   if (a->p_terms < 0 || a->p_terms > 2) return fail(FMHA_ERR_INVALID_ARG, "p_terms must be 0, 1 or 2");
   if (a->p_terms == 2 && !v8) return fail(FMHA_ERR_INVALID_ARG, "p_terms = 2 needs an E4M3 V");
 
   // tensors
   const bool paged = pg != nullptr;
   if ((st = check_tensor(a->q, "q", B, Sq, Hq, D)) != FMHA_OK) return st;
-  if ((st = check_tensor(a->o, "o", B, Sq, Hq, D)) != FMHA_OK) return st;
+  if ((st = check_tensor(a->o, "o", B, Sq, Hq, Dv)) != FMHA_OK) return st;
   if (paged) {
     if (pg->page_size != 16 && pg->page_size != 32 && pg->page_size != 64 && pg->page_size != 128)
       return fail(FMHA_ERR_UNSUPPORTED, "page_size %d (supported: 16, 32, 64, 128)", pg->page_size);
@@ -320,10 +326,10 @@ fmha_status run_attention(const fmha_args* a, const uint8_t* mask, int64_t msb, 
     if (pg->max_pages_per_seq < ceil_div(Skv, pg->page_size))
       return fail(FMHA_ERR_INVALID_ARG, "max_pages_per_seq %d < ceil(Skv / page_size)", pg->max_pages_per_seq);
     if ((st = check_tensor(a->k, "k", pg->num_pages, pg->page_size, Hkv, D)) != FMHA_OK) return st;
-    if ((st = check_tensor(a->v, "v", pg->num_pages, pg->page_size, Hkv, D)) != FMHA_OK) return st;
+    if ((st = check_tensor(a->v, "v", pg->num_pages, pg->page_size, Hkv, Dv)) != FMHA_OK) return st;
   } else if (Skv > 0) {
     if ((st = check_tensor(a->k, "k", B, Skv, Hkv, D)) != FMHA_OK) return st;
-    if ((st = check_tensor(a->v, "v", B, Skv, Hkv, D)) != FMHA_OK) return st;
+    if ((st = check_tensor(a->v, "v", B, Skv, Hkv, Dv)) != FMHA_OK) return st;
   }
   if (a->lse != nullptr && (reinterpret_cast<uintptr_t>(a->lse) & 3u) != 0)
     return fail(FMHA_ERR_INVALID_ARG, "lse misaligned");
@@ -347,10 +353,11 @@ fmha_status run_attention(const fmha_args* a, const uint8_t* mask, int64_t msb, 
     const int64_t strides[3] = {a->q.stride_h, a->q.stride_s, a->q.stride_b};
     const uint32_t box[4] = {uint32_t(128 / eqk), 1, 128, 1};
     if ((st = make_map(&tq, a->q.ptr, eqk, dims, strides, box, "q")) != FMHA_OK) return st;
+    const uint64_t odims[4] = {uint64_t(Dv), uint64_t(Hq), uint64_t(Sq), uint64_t(B)};
     const int64_t ostr[3] = {a->o.stride_h, a->o.stride_s, a->o.stride_b};
     // BF16 O: 64-column (128-byte) boxes; E4M3 O: the whole 128-byte row.
     const uint32_t obox[4] = {o8 ? 128u : 64u, 1, 128, 1};
-    if ((st = make_map(&to, a->o.ptr, o8 ? 1 : 2, dims, ostr, obox, "o")) != FMHA_OK) return st;
+    if ((st = make_map(&to, a->o.ptr, o8 ? 1 : 2, odims, ostr, obox, "o")) != FMHA_OK) return st;
   }
   if (Skv == 0) {  // no key is ever loaded; any valid descriptor will do
     tk = tq;
@@ -360,13 +367,14 @@ fmha_status run_attention(const fmha_args* a, const uint8_t* mask, int64_t msb, 
     CUtensorMap* out[2] = {&tk, &tv};
     for (int i = 0; i < 2; ++i) {
       const int eb = i == 0 ? eqk : ev;
+      const int dd = i == 0 ? D : Dv;
       const int64_t strides[3] = {kv[i]->stride_h, kv[i]->stride_s, kv[i]->stride_b};
       if (paged) {
-        const uint64_t dims[4] = {uint64_t(D), uint64_t(Hkv), uint64_t(pg->page_size), uint64_t(pg->num_pages)};
+        const uint64_t dims[4] = {uint64_t(dd), uint64_t(Hkv), uint64_t(pg->page_size), uint64_t(pg->num_pages)};
         const uint32_t box[4] = {uint32_t(128 / eb), 1, uint32_t(pg->page_size), 1};
         st = make_map(out[i], kv[i]->ptr, eb, dims, strides, box, i == 0 ? "k pool" : "v pool");
       } else {
-        const uint64_t dims[4] = {uint64_t(D), uint64_t(Hkv), uint64_t(Skv), uint64_t(B)};
+        const uint64_t dims[4] = {uint64_t(dd), uint64_t(Hkv), uint64_t(Skv), uint64_t(B)};
         const uint32_t box[4] = {uint32_t(128 / eb), 1, 128, 1};
         st = make_map(out[i], kv[i]->ptr, eb, dims, strides, box, i == 0 ? "k" : "v");
       }
@@ -379,7 +387,7 @@ fmha_status run_attention(const fmha_args* a, const uint8_t* mask, int64_t msb, 
   p.B = B; p.Hq = Hq; p.Hkv = Hkv; p.Sq = Sq; p.Skv = Skv; p.group = Hq / Hkv;
   p.n_q_blocks = ceil_div(Sq, 128);
   p.n_kv_blocks = ceil_div(Skv, 128);
-  p.pair_mode = (p.group % 2 == 0) ? PAIR_HEADS : PAIR_ROWS;
+  p.pair_mode = query_tiles_per_cta(qk, D) == 1 ? SINGLE : (p.group % 2 == 0) ? PAIR_HEADS : PAIR_ROWS;
   p.n_units = p.pair_mode == PAIR_ROWS ? ceil_div(p.n_q_blocks, 2) : p.n_q_blocks;
   p.causal = a->causal != 0;
   const float scale = a->softmax_scale > 0.f ? a->softmax_scale : 1.0f / std::sqrt(float(D));
@@ -444,10 +452,11 @@ fmha_status run_attention(const fmha_args* a, const uint8_t* mask, int64_t msb, 
     }
     return ok_status();
   }
-  const long long head_units = p.pair_mode == PAIR_ROWS ? Hq : Hq / 2;
+  const long long head_units = p.pair_mode == PAIR_HEADS ? Hq / 2 : Hq;
   if (static_cast<long long>(p.n_units) * head_units * B >= (1ll << 31))
     return fail(FMHA_ERR_UNSUPPORTED, "grid too large");
-  e = launch_attention(qk, pv, D, paged, p, tq, tk, tv, to, stream);
+  e = D == 192 ? launch_attention_d192(qk, pv, paged, p, tq, tk, tv, to, stream)
+               : launch_attention(qk, pv, D, paged, p, tq, tk, tv, to, stream);
   if (e != cudaSuccess) return fail(FMHA_ERR_CUDA, "attention launch: %s", cudaGetErrorString(e));
   return ok_status();
 }

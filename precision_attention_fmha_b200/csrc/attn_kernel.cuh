@@ -45,9 +45,11 @@
 
 namespace fmha {
 
-template <int D_, int QK_, int PV_, bool PAGED_, bool P2_ = false, bool PACKED_ = false, bool O8_ = false>
+// D: head dim of Q and K; DV: head dim of V and O (192 / 128 for a wide QK).
+template <int D_, int QK_, int PV_, bool PAGED_, bool P2_ = false, bool PACKED_ = false, bool O8_ = false,
+          int DV_ = D_>
 struct AttnCfg {
-  static constexpr int D = D_, QK = QK_, PV = PV_;
+  static constexpr int D = D_, DV = DV_, QK = QK_, PV = PV_;
   static constexpr bool PAGED = PAGED_;
   // GQA-packed query tiles and split-KV ranges (decode shapes).
   static constexpr bool PACKED = PACKED_;
@@ -55,20 +57,24 @@ struct AttnCfg {
   static_assert(!P2 || PV == PV_E4M3, "two-term P needs an E4M3 V");
   // E4M3 output: O / sf_o rounded to E4M3 (one 128-byte row per query row).
   static constexpr bool O8 = O8_;
-  static_assert(!O8 || (D == 128 && !PACKED), "E4M3 O is built for D = 128 tiles");
+  static_assert(!O8 || (DV == 128 && !PACKED), "E4M3 O is built for 128-wide O tiles");
+  static_assert(DV == 64 || DV == 128, "V / O head dim 64 or 128");
   static constexpr int BM = 128, BN = 128;
   static constexpr int QK_ELEM = QK == QK_BF16 ? 2 : 1;
   static constexpr int V_ELEM = PV == PV_BF16 ? 2 : 1;
   static constexpr int QK_ROW_BYTES = D * QK_ELEM;
-  static constexpr int QK_CHUNKS = QK_ROW_BYTES / 128;  // 128-byte swizzle columns along D
+  // 128-byte swizzle columns along D. A 192-byte E4M3 row takes two: the copy
+  // of the second reads 64 bytes past the row's end, which TMA fills with
+  // zeros (they count in the transaction bytes; no MMA step reads them).
+  static constexpr int QK_CHUNKS = (QK_ROW_BYTES + 127) / 128;
   static constexpr int QK_CHUNK_ELEMS = 128 / QK_ELEM;
-  static constexpr int V_CHUNKS = D * V_ELEM / 128;
+  static constexpr int V_CHUNKS = DV * V_ELEM / 128;
   static constexpr int V_CHUNK_ELEMS = 128 / V_ELEM;
-  static_assert(QK_ROW_BYTES % 128 == 0 && (D * V_ELEM) % 128 == 0, "rows must be whole 128-byte atoms");
+  static_assert(QK_ROW_BYTES % 64 == 0 && (DV * V_ELEM) % 128 == 0, "rows must be whole swizzle atoms");
   static constexpr int CHUNK_BYTES = 128 * 128;  // one 128-row x 128-byte swizzled column block
-  static constexpr int Q_TILE = BM * QK_ROW_BYTES;
-  static constexpr int K_TILE = BN * QK_ROW_BYTES;
-  static constexpr int V_TILE = BN * D * V_ELEM;
+  static constexpr int Q_TILE = BM * QK_CHUNKS * 128;
+  static constexpr int K_TILE = BN * QK_CHUNKS * 128;
+  static constexpr int V_TILE = BN * DV * V_ELEM;
   static constexpr int SLOT = K_TILE > V_TILE ? K_TILE : V_TILE;
   // E4M3 P is staged in shared memory (one 128 x 128 byte tile per query tile
   // and term) so that a tile's S buffer in TMEM is free as soon as the softmax
@@ -78,13 +84,16 @@ struct AttnCfg {
   static constexpr bool PSMEM = PV == PV_E4M3;
   static constexpr bool TURNS = PSMEM;  // exp-phase turn-taking between the softmax warpgroups
   static constexpr int P_TILE = BM * BN;  // bytes per E4M3 P tile
-  static constexpr int P_BYTES = PSMEM ? 2 * P_TILE * (P2 ? 2 : 1) : 0;
+  // Query tiles per CTA (1 when two 48 KB BF16 Q tiles would starve the K/V ring).
+  static constexpr int NQ = query_tiles_per_cta(QK, D);
+  static_assert(NQ == 2 || !PACKED, "decode tiles come in pairs");
+  static constexpr int P_BYTES = PSMEM ? NQ * P_TILE * (P2 ? 2 : 1) : 0;
   static constexpr int MISC_BYTES = 2048;
   static constexpr int SMEM_CAP = 232448;  // 227 KB opt-in maximum per CTA
-  static constexpr int STAGES_FIT = (SMEM_CAP - 1024 - MISC_BYTES - 2 * Q_TILE - P_BYTES) / SLOT;
+  static constexpr int STAGES_FIT = (SMEM_CAP - 1024 - MISC_BYTES - NQ * Q_TILE - P_BYTES) / SLOT;
   static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
   static_assert(STAGES >= 3, "the K/V ring needs at least three slots");
-  static constexpr int SMEM_BYTES = 1024 + 2 * Q_TILE + P_BYTES + STAGES * SLOT + MISC_BYTES;
+  static constexpr int SMEM_BYTES = 1024 + NQ * Q_TILE + P_BYTES + STAGES * SLOT + MISC_BYTES;
   static constexpr int QK_STEPS = QK_ROW_BYTES / 32;  // one MMA covers 32 bytes of K (16 bf16 / 32 8-bit)
   static constexpr int PV_K = PV == PV_BF16 ? 16 : 32;
   static constexpr int PV_STEPS = BN / PV_K;
@@ -94,7 +103,7 @@ struct AttnCfg {
                                        : QK == QK_E4M3 ? ptx::make_idesc(1, 0, 0, 0, 0, BN, BM)
                                                        : ptx::make_idesc(2, 1, 1, 0, 0, BN, BM);
   static constexpr uint32_t IDESC_PV =
-      PV == PV_BF16 ? ptx::make_idesc(1, 1, 1, 0, 1, D, BM) : ptx::make_idesc(1, 0, 0, 0, 1, D, BM);
+      PV == PV_BF16 ? ptx::make_idesc(1, 1, 1, 0, 1, DV, BM) : ptx::make_idesc(1, 0, 0, 0, 1, DV, BM);
   static constexpr int THREADS = 384;
   // Warp roles: warpgroup 0 = control (MMA issue, TMA loads, two idle warps),
   // warpgroups 1 and 2 = softmax of query tiles 0 and 1 (one thread per row).
@@ -418,7 +427,7 @@ __device__ void attn_mma_role(const AttnParams& p, const TileInfo t0, const Tile
   const uint32_t q_lo0 = desc_lo(smem_addr(sQ0), 16), q_lo1 = desc_lo(smem_addr(sQ1), 16);
   const uint32_t k_lo0 = desc_lo(smem_addr(sSlots), 16);
   const uint32_t v_lo0 = desc_lo(smem_addr(sSlots), C::CHUNK_BYTES);
-  const uint32_t o_col[2] = {256u, 256u + C::D};
+  const uint32_t o_col[2] = {256u, 256u + C::DV};
   int pend[2] = {-1, -1};
   int pv_cnt[2] = {0, 0};
   int prev_v = -1;
@@ -533,7 +542,7 @@ __device__ void attn_mma_role_psmem(const AttnParams& p, const TileInfo t0, cons
   const uint32_t k_lo0 = desc_lo(smem_addr(sSlots), 16);
   const uint32_t v_lo0 = desc_lo(smem_addr(sSlots), C::CHUNK_BYTES);
   const uint32_t s_col[2] = {0u, 128u};
-  const uint32_t o_col[2] = {256u, 256u + C::D};
+  const uint32_t o_col[2] = {256u, 256u + C::DV};
   const int n_u = max(t0.n_kv, t1.n_kv);
   int s_cnt[2] = {0, 0}, pv_cnt[2] = {0, 0};
   int slot_it = 0;
@@ -685,7 +694,7 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, 
   using namespace ptx;
   constexpr uint32_t FULL = 0xffffffffu;
   constexpr int NCH = C::BN / 32;  // 32-key chunks per tile (one TMEM load each)
-  constexpr int OB = C::D / 32;    // 32-column blocks of O
+  constexpr int OB = C::DV / 32;   // 32-column blocks of O
   const int warp = (threadIdx.x >> 5) & 3;  // TMEM lane quadrant of this warp
   const int lane = threadIdx.x & 31;
   const int r = warp * 32 + lane;  // row within the tile
@@ -694,7 +703,7 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, 
   const int head = C::PACKED ? t.h + (r & ((1 << p.group_shift) - 1)) : t.h;
   const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
   const uint32_t tS = tmem + lane_off + (x ? 128u : 0u);
-  const uint32_t tO = tmem + lane_off + (x ? 256u + C::D : 256u);
+  const uint32_t tO = tmem + lane_off + (x ? 256u + C::DV : 256u);
   const bool lead = (threadIdx.x & 127) == 0;  // one thread of the query tile
   const int64_t bhq = static_cast<int64_t>(b) * p.Hq + head;
   const int64_t bhk = static_cast<int64_t>(b) * p.Hkv + hkv;
@@ -976,7 +985,7 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, 
     const float inv_lo = inv_l / (p.sf_o != nullptr ? __ldg(p.sf_o) : 1.f);
     const uint32_t base = stage0 + r * 128;
 #pragma unroll 1
-    for (int sc = 0; sc < C::D / 32; ++sc) {
+    for (int sc = 0; sc < C::DV / 32; ++sc) {
       uint32_t o[32];
       if (have_o) {
         tmem_ld32(tO + 32 * sc, o);
@@ -1011,7 +1020,7 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, 
     }
   }
 #pragma unroll 1
-  for (int c64 = 0; c64 < (C::O8 ? 0 : C::D / 64); ++c64) {
+  for (int c64 = 0; c64 < (C::O8 ? 0 : C::DV / 64); ++c64) {
     uint32_t o[2][32];
     if (have_o) {
       tmem_ld32(tO + 64 * c64, o[0]);
@@ -1028,7 +1037,7 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, 
     if constexpr (C::PACKED) {
       if (p.n_parts > 1) {  // one partial: O / l in fp32 for the merge kernel (no staging)
         if (row < p.Sq && ok) {
-          float* dst = p.o_part + ((((int64_t)t.part * p.B + b) * p.Sq + row) * p.Hq + head) * C::D + 64 * c64;
+          float* dst = p.o_part + ((((int64_t)t.part * p.B + b) * p.Sq + row) * p.Hq + head) * C::DV + 64 * c64;
 #pragma unroll
           for (int j = 0; j < 64; j += 4) {
             asm volatile("st.global.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst + j), "f"(out_val(j)),
@@ -1088,9 +1097,11 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   using namespace ptx;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* const sQ[2] = {smem, smem + C::Q_TILE};
-  uint8_t* const sP[2] = {smem + 2 * C::Q_TILE, smem + 2 * C::Q_TILE + C::P_BYTES / 2};  // E4M3 P (shared-memory P)
-  uint8_t* sSlots = smem + 2 * C::Q_TILE + C::P_BYTES;
+  // Q buffers, then E4M3 P buffers (shared-memory P), then the K/V ring. With one
+  // query tile per CTA the second tile's pointers alias the first (never used).
+  uint8_t* const sQ[2] = {smem, smem + (C::NQ - 1) * C::Q_TILE};
+  uint8_t* const sP[2] = {smem + C::NQ * C::Q_TILE, smem + C::NQ * C::Q_TILE + (C::NQ - 1) * (C::P_BYTES / C::NQ)};
+  uint8_t* sSlots = smem + C::NQ * C::Q_TILE + C::P_BYTES;
   AttnMisc* misc = reinterpret_cast<AttnMisc*>(sSlots + C::STAGES * C::SLOT);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -1178,7 +1189,16 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     }
   } else {
     int item = blockIdx.x;
-    if (p.pair_mode == PAIR_ROWS) {
+    if (C::NQ == 1) {  // SINGLE: one query block of one head; tile 1 stays empty
+      int qb = item % p.n_units;
+      item /= p.n_units;
+      const int h = item % p.Hq;
+      b = item / p.Hq;
+      if (p.causal) qb = p.n_units - 1 - qb;  // heaviest causal tiles first
+      t[0].h = t[1].h = h;
+      t[0].qblk = qb;
+      t[1].qblk = p.n_q_blocks;  // past the end: not valid
+    } else if (p.pair_mode == PAIR_ROWS) {
       int pr = item % p.n_units;
       item /= p.n_units;
       const int h = item % p.Hq;
@@ -1258,8 +1278,8 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     misc->abort = 0u;
     fence_barrier_init();
   }
-  if (C::PV == PV_E4M3 && p.sf_v_kind == FMHA_SF_PER_CHANNEL && threadIdx.x < C::D)
-    misc->sf_v[threadIdx.x] = p.sf_v[(static_cast<int64_t>(b) * p.Hkv + hkv) * C::D + threadIdx.x];
+  if (C::PV == PV_E4M3 && p.sf_v_kind == FMHA_SF_PER_CHANNEL && threadIdx.x < C::DV)
+    misc->sf_v[threadIdx.x] = p.sf_v[(static_cast<int64_t>(b) * p.Hkv + hkv) * C::DV + threadIdx.x];
   if (warp == C::MMA_WARP) {
     tmem_alloc(smem_addr(&misc->tmem_base), C::TMEM_COLS);
     tmem_relinquish();
@@ -1325,7 +1345,7 @@ cudaError_t launch_attention_t(const AttnParams& p, const CUtensorMap& tq, const
   auto kern = attn_fwd_kernel<C>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  const int head_units = C::PACKED ? p.Hkv * p.n_splits : (p.pair_mode == PAIR_ROWS ? p.Hq : p.Hq / 2);
+  const int head_units = C::PACKED ? p.Hkv * p.n_splits : (p.pair_mode == PAIR_HEADS ? p.Hq / 2 : p.Hq);
   const long long blocks = static_cast<long long>(p.n_units) * head_units * p.B;
   kern<<<static_cast<unsigned>(blocks), C::THREADS, C::SMEM_BYTES, stream>>>(p, tq, tk, tv, to);
   return cudaGetLastError();
@@ -1335,6 +1355,7 @@ cudaError_t launch_attention_t(const AttnParams& p, const CUtensorMap& tq, const
 template <int D, int QK, int PV, bool PAGED>
 cudaError_t launch_attention_variants(const AttnParams& p, const CUtensorMap& tq, const CUtensorMap& tk,
                                       const CUtensorMap& tv, const CUtensorMap& to, cudaStream_t s) {
+  static_assert(D == 64 || D == 128, "the 192-wide QK kernels have their own instantiation unit");
   if constexpr (PV == PV_E4M3) {
     if (p.p_terms == 2)
       return p.o8 ? launch_attention_t<AttnCfg<D, QK, PV, PAGED, true, false, true>>(p, tq, tk, tv, to, s)

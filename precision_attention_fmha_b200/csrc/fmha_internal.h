@@ -28,13 +28,19 @@ enum PvKind : int { PV_BF16 = 0, PV_E4M3 = 1 };
 enum PairMode : int {
   PAIR_ROWS = 0,   // query blocks 2i and 2i+1 of one head
   PAIR_HEADS = 1,  // one query block of heads 2j and 2j+1 (same KV head)
+  SINGLE = 2,      // one query block of one head (one query tile per CTA)
 };
+
+// Query tiles per attention CTA. Two share every K/V tile, except when the QK
+// head dim makes a BF16 Q tile 48 KB (D = 192): two of them would leave room
+// for only two 48 KB K/V slots, so such a CTA takes one query tile.
+constexpr int query_tiles_per_cta(int qk_kind, int d_qk) { return (qk_kind == QK_BF16 && d_qk > 128) ? 1 : 2; }
 
 struct AttnParams {
   int32_t B, Hq, Hkv, Sq, Skv, group;
   int32_t n_q_blocks;   // ceil(Sq / 128)
   int32_t n_kv_blocks;  // ceil(Skv / 128)
-  int32_t pair_mode;
+  int32_t pair_mode;  // PAIR_ROWS / PAIR_HEADS / SINGLE
   int32_t n_units;      // work items per (b, head unit): pairs of q blocks (PAIR_ROWS) or q blocks (PAIR_HEADS)
   int32_t causal;
   float scale_log2;     // softmax_scale * log2(e)

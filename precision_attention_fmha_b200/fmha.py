@@ -51,7 +51,7 @@ class _Args(ctypes.Structure):
                 ("B", ctypes.c_int32), ("Hq", ctypes.c_int32), ("Hkv", ctypes.c_int32),
                 ("Sq", ctypes.c_int32), ("Skv", ctypes.c_int32), ("D", ctypes.c_int32),
                 ("softmax_scale", ctypes.c_float), ("causal", ctypes.c_int32), ("lse", ctypes.c_void_p),
-                ("p_terms", ctypes.c_int32), ("reserved", ctypes.c_int32), ("sf_o", _Sf)]
+                ("p_terms", ctypes.c_int32), ("Dv", ctypes.c_int32), ("sf_o", _Sf)]
 
 
 _lib = None
@@ -225,24 +225,28 @@ def _args(q, k, v, out, sf_q, sf_k, sf_v, sf_p, softmax_scale, causal, lse, Skv=
     a.causal = 1 if causal else 0
     a.lse = lse.data_ptr() if lse is not None else None
     a.p_terms = int(p_terms)
+    a.Dv = v.shape[3]
     a.sf_o = _sf(sf_o)
     return a
 
 
-def _out_like(q, out):
+def _out_like(q, v, out):
+    """O is [B, Sq, Hq, Dv]: Dv, the head dim of V, differs from q's for D = 192 / 128."""
     if out is None:
-        out = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device)
+        out = torch.empty(q.shape[:3] + v.shape[3:], dtype=torch.bfloat16, device=q.device)
     return out
 
 
 def fmha_fwd(q, k, v, out=None, sf_q=None, sf_k=None, sf_v=None, sf_p=None, softmax_scale=None, causal=False,
              lse=None, stream=None, p_terms=1, sf_o=None):
-    """Dense attention. Returns O (BF16 [B, Sq, Hq, D]). p_terms=2 splits an E4M3 P into two terms.
+    """Dense attention. Returns O (BF16 [B, Sq, Hq, Dv]). p_terms=2 splits an E4M3 P into two terms.
+
+    Head dims: q / k D and v / out Dv, equal (64 or 128), or D = 192 with Dv = 128.
 
     An E4M3 ``out`` (torch.float8_e4m3fn, D = 128) receives E4M3(O / sf_o),
     with sf_o an optional per-tensor Scale (1.0 when None)."""
     lib = load_library()
-    out = _out_like(q, out)
+    out = _out_like(q, v, out)
     a = _args(q, k, v, out, sf_q, sf_k, sf_v, sf_p, softmax_scale, causal, lse, p_terms=p_terms, sf_o=sf_o)
     _check(lib.fmha_fwd(ctypes.byref(a), _stream(stream)))
     return out
@@ -252,7 +256,7 @@ def fmha_fwd_block_sparse(q, k, v, mask, out=None, sf_q=None, sf_k=None, sf_v=No
                           softmax_scale=None, causal=False, lse=None, stream=None, p_terms=1, sf_o=None):
     """Attention restricted by a uint8 128x128 block mask [B or 1, Hkv or 1, ceil(Sq/128), ceil(Skv/128)]."""
     lib = load_library()
-    out = _out_like(q, out)
+    out = _out_like(q, v, out)
     a = _args(q, k, v, out, sf_q, sf_k, sf_v, sf_p, softmax_scale, causal, lse, p_terms=p_terms, sf_o=sf_o)
     msb, msh = _mask_strides(mask, q.shape[1], k.shape[1])
     _check(lib.fmha_fwd_block_sparse(ctypes.byref(a), mask.data_ptr(), msb, msh, _stream(stream)))
@@ -272,7 +276,7 @@ def fmha_fwd_paged(q, k_pool, v_pool, page_table, Skv, mask=None, out=None, sf_q
                    sf_p=None, softmax_scale=None, causal=False, lse=None, stream=None, p_terms=1, sf_o=None):
     """Attention over a paged K/V pool [num_pages, page_size, Hkv, D] through page_table int32 [B, max_pages]."""
     lib = load_library()
-    out = _out_like(q, out)
+    out = _out_like(q, v_pool, out)
     if page_table.dtype != torch.int32 or page_table.dim() != 2 or not page_table.is_contiguous():
         raise ValueError("page_table must be contiguous int32 [B, max_pages_per_seq]")
     a = _args(q, k_pool, v_pool, out, sf_q, sf_k, sf_v, sf_p, softmax_scale, causal, lse, Skv=Skv, p_terms=p_terms,
@@ -295,7 +299,7 @@ def fmha_fwd_decode(q, k, v, page_table=None, Skv=None, mask=None, num_splits=0,
     with page_table int32 [B, max_pages] and Skv. The workspace (uint8 CUDA tensor)
     is allocated here when not given. Returns O (BF16 [B, Sq, Hq, D])."""
     lib = load_library()
-    out = _out_like(q, out)
+    out = _out_like(q, v, out)
     if page_table is not None:
         if page_table.dtype != torch.int32 or page_table.dim() != 2 or not page_table.is_contiguous():
             raise ValueError("page_table must be contiguous int32 [B, max_pages_per_seq]")

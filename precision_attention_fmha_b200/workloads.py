@@ -22,6 +22,9 @@ Workloads (B, heads, sequence lengths, head dim, distributions):
                   pool of 64-token pages addressed through a seeded random
                   page-table permutation; 128x128 block mask per (b, kv head)
                   drawn Bernoulli(0.25) with the diagonal block forced on.
+* ``wide_qk``     the dense workload with a 192-wide Q/K head dim and a
+                  128-wide V: B=1 H=40 Sq=Skv=16384, BF16 N(0,1) (with the
+                  all_fp8 outliers when ``outliers``), scale 1/sqrt(192).
 
 Every generator takes the sizes as arguments so tests can draw small cases
 with the same recipe.
@@ -83,15 +86,16 @@ def block_mask(seed, B, Hkv, Sq, Skv, density=0.25, block=128):
 
 def paged_pool(seed, k, v, page_size=64, extra_pages=0):
     """Scatter contiguous K/V [B,S,H,D] into a pool of pages through a seeded
-    random permutation. Returns (k_pool, v_pool [P,page,H,D], page_table int32
-    [B, pages_per_seq]). Unused pool pages (``extra_pages``) hold N(0,1) noise."""
+    random permutation. Returns (k_pool [P,page,H,D], v_pool [P,page,H,Dv],
+    page_table int32 [B, pages_per_seq]). Unused pool pages (``extra_pages``)
+    hold N(0,1) noise."""
     B, S, H, D = k.shape
     per_seq = -(-S // page_size)
     P = B * per_seq + extra_pages
     rng = np.random.default_rng(seed)
     perm = rng.permutation(P)[: B * per_seq].reshape(B, per_seq).astype(np.int32)
     kp = _normal_bf16(rng, (P, page_size, H, D))
-    vp = _normal_bf16(rng, (P, page_size, H, D))
+    vp = _normal_bf16(rng, (P, page_size, H, v.shape[3]))
     for b in range(B):
         for i in range(per_seq):
             t0, t1 = i * page_size, min(S, (i + 1) * page_size)
@@ -114,6 +118,18 @@ def dense_pv8(S=16384, B=1, H=40, D=128):
 
 def all_fp8(S=8192, B=2, H=32, D=128):
     q, k, v = outlier_qkv(SEED_BASE + 3 + S, B, S, H, D)
+    return dict(q=q, k=k, v=v, scale=1.0 / math.sqrt(D))
+
+
+def wide_qk(S=16384, B=1, H=40, D=192, Dv=128, outliers=False):
+    """Q, K [B,S,H,D] and V [B,S,H,Dv] (D != Dv): N(0,1), or with 1% x20 outliers."""
+    seed = SEED_BASE + 6 + S
+    if outliers:
+        q, k, _ = outlier_qkv(seed, B, S, H, D)
+        _, _, v = outlier_qkv(seed + 1, B, S, H, Dv)
+    else:
+        q, k, _ = normal_qkv(seed, B, S, S, H, H, D)
+        _, _, v = normal_qkv(seed + 1, B, S, S, H, H, Dv)
     return dict(q=q, k=k, v=v, scale=1.0 / math.sqrt(D))
 
 

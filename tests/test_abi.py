@@ -97,6 +97,32 @@ def test_eight_bit_scale_rules(lib):
     assert lib.fmha_fwd(ctypes.byref(a), None) == 2
 
 
+def _wide_args(dq=fmha.BF16, dv=fmha.BF16, Dv=128):
+    """D = 192 Q/K with a Dv-wide V / O (strides sized per operand)."""
+    a = _args(D=192, dq=dq, dv=dv)
+    for t in (a.v, a.o):
+        t.stride_b, t.stride_s, t.stride_h = 256 * 4 * Dv, 4 * Dv, Dv
+    a.Dv = Dv
+    return a
+
+
+@pytest.mark.parametrize("mutate", [
+    lambda a: setattr(a, "Dv", 0),                                    # Dv = D = 192
+    lambda a: setattr(a, "Dv", 192),
+    lambda a: (setattr(a, "D", 128), setattr(a, "Dv", 64)),           # Dv != D below 192
+    lambda a: (setattr(a.q, "dtype", fmha.INT8), setattr(a.k, "dtype", fmha.INT8),
+               setattr(a.v, "dtype", fmha.E4M3)),                     # INT8 Q/K
+    lambda a: setattr(a.o, "dtype", fmha.E4M3),                       # E4M3 O
+    lambda a: (setattr(a.v, "dtype", fmha.E4M3), setattr(a, "p_terms", 2)),  # two-term P
+])
+def test_wide_qk_head_dim_rules(lib, mutate):
+    """D = 192 takes Dv = 128, BF16 or E4M3 Q/K, one-term P and a BF16 O."""
+    a = _wide_args()
+    mutate(a)
+    assert lib.fmha_fwd(ctypes.byref(a), None) == 2
+    assert lib.fmha_last_error_message().decode()
+
+
 def test_paged_argument_checks(lib):
     a = _args()
     assert lib.fmha_fwd_paged(ctypes.byref(a), 0x30000, 8, 48, 4, None, 0, 0, None) == 2  # page size
