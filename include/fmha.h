@@ -94,7 +94,8 @@ typedef struct {
 } fmha_sf;
 
 /* Arguments of one attention call.
- *   q [B, Sq, Hq, D], k [B, Skv, Hkv, D], v [B, Skv, Hkv, D], o [B, Sq, Hq, D].
+ *   q [B, Sq, Hq, D], k [B, Skv, Hkv, D], v [B, Skv, Hkv, Dv], o [B, Sq, Hq, Dv]
+ *   (Dv = D except for the 192 / 128 head dims below).
  *   Query head h attends to KV head h / (Hq / Hkv) (grouped-query attention).
  *   O_i = sum_j softmax_j(softmax_scale * q_i . k_j) v_j over the visible keys
  *   j, where q, k, v are the DEQUANTIZED operands (code * scale).
@@ -123,7 +124,11 @@ typedef struct {
  * Supported (q, k, v, o) dtype tuples: (BF16, BF16, BF16, BF16),
  * (BF16, BF16, E4M3, BF16) ("QK-BF16/PV-FP8", [BW-FP8]),
  * (E4M3, E4M3, E4M3, BF16) ("all-FP8", [BW-FP8]), (INT8, INT8, E4M3, BF16)
- * ("SageAttention", [DiT-Sage]). D must be 64 or 128 (128 for 8-bit Q/K).
+ * ("SageAttention", [DiT-Sage]). D must be 64 or 128 (128 for 8-bit Q/K),
+ * or D = 192 with Dv = 128 for the BF16, QK-BF16/PV-FP8 and all-FP8 tuples
+ * with one-term P and a BF16 o, not through fmha_fwd_decode: the QK head dim
+ * that [BW-FP8]'s reviewer notes name as the case their shared-memory-P
+ * schedule was gated off for (shared-memory capacity).
  * Any of these may instead write an E4M3 o (D = 128, not fmha_fwd_decode):
  * o = E4M3(O / sf_o) rounded to nearest even and saturated to +-448. This is
  * the FP8 output that [BW-FP8]'s reviewer notes mention, where their shared-

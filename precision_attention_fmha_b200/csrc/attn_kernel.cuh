@@ -682,11 +682,10 @@ __device__ __forceinline__ void exp2_poly_x2(float& a, float& b) {
 //
 // The running row max m is lazy ("FlashInfer FP8/BF16 mixed-precision
 // attention for Blackwell", section 3): it only moves, and O and l are only
-// rescaled, when a tile's max exceeds m by more than tau (log2 units). So for
-// every tile after the first, the exponentials are computed speculatively with
-// the current m while the tile's max is reduced in the same pass; only when
-// some row of the warp crosses m + tau does the warp redo the tile with the
-// new max. The row max is then off the critical chain of a tile.
+// rescaled, when a tile's max exceeds m by more than tau (log2 units). Each
+// tile takes its row max first, then one pass computes the exponentials,
+// packs P and adds the row sum. (Loading the next tile's S from TMEM while
+// this tile's E4M3 P is stored was measured 10 % slower.)
 template <class C>
 __device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, int b, int hkv, uint8_t* sQx,
                                   uint8_t* sPx, int n_turns, AttnMisc* misc, uint32_t tmem, const CUtensorMap* tmO,
