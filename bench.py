@@ -61,6 +61,8 @@ WORKLOADS = {
     "nvfp4_t16384_k4096": ("nvfp4", 1, 1, 1, 16384, 4096, False),
     # SageAttention K smoothing of the Sage workload's K: token mean per channel + shifted INT8 quantizer
     "sage_k_smooth_s16384": ("smooth_k", 1, 24, 24, 16384, 128, False),
+    # the token-block quantizer alone on the same K: INT8 codes with one scale per 64 tokens of a head
+    "sage_k_quant_s16384": ("quant_k", 1, 24, 24, 16384, 128, False),
 }
 DEFAULT_WORKLOAD = "dense_pv8_s32768"
 L2_BYTES = 126 * 2**20          # B200 L2
@@ -628,14 +630,21 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+SMOOTH_METRIC = ("K smoothing GB/s (token mean per channel + INT8 quantization of K - mean: 4 B read + 1 B written "
+                 "per element)")
+QUANT_METRIC = "token-block quantization GB/s (INT8 codes of K, one scale per 64-token block: 2 B read + 1 B written per element)"
+
+
 def run_smooth(args):
-    """SageAttention K smoothing of the Sage workload's K: channel mean + shifted INT8 quantizer. HBM-bound."""
+    """SageAttention K smoothing of the Sage workload's K (channel mean + shifted INT8
+    quantizer), or the token-block quantizer alone (workload kind quant_k). HBM-bound."""
     from precision_attention_fmha_b200 import fmha, workloads
 
     world, rank, local = dist_setup(args.gpus)
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
-    _, B, H, _, S, D, _ = WORKLOADS[args.workload]
+    kind, B, H, _, S, D, _ = WORKLOADS[args.workload]
+    smooth = kind == "smooth_k"
     kh = workloads.sage(S=S, B=B, H=H, D=D)["k"].contiguous().pin_memory()
     k = kh.to(dev)
     mean = torch.empty((B, H, D), dtype=torch.float32, device=dev)
@@ -644,8 +653,10 @@ def run_smooth(args):
     scales = torch.empty(fmha.scale_shape("per_token_block", B, S, H, D, 64), dtype=torch.float32, device=dev)
 
     def step(inp):
-        fmha.channel_mean(inp, out=mean, workspace=mws)
-        fmha.fmha_quantize_blockwise(inp, torch.int8, "per_token_block", 64, out=codes, scales=scales, shift=mean)
+        if smooth:
+            fmha.channel_mean(inp, out=mean, workspace=mws)
+        fmha.fmha_quantize_blockwise(inp, torch.int8, "per_token_block", 64, out=codes, scales=scales,
+                                     shift=mean if smooth else None)
 
     for _ in range(args.warmup):
         step(k)
@@ -671,11 +682,12 @@ def run_smooth(args):
     clk = clocks.stop()
     ms = max_over_ranks(statistics.mean(a.elapsed_time(b) for a, b in evs), world)
     # mean: K read once; quantizer: K read once, codes + scales written; mean written once
-    out_bytes = codes.numel() + scales.numel() * 4 + mean.numel() * 4
-    algo = 2 * k.numel() * 2 + out_bytes
+    outs = (codes, scales, mean) if smooth else (codes, scales)
+    out_bytes = sum(t.numel() * t.element_size() for t in outs)
+    algo = (2 if smooth else 1) * k.numel() * 2 + out_bytes
     _, hbm, src = load_peaks()
     gbs = algo / (ms * 1e-3) / 1e9
-    oh = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (codes, scales, mean)]
+    oh = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
     Ke = max(1, min(K_, 10))
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier(world)
@@ -683,15 +695,14 @@ def run_smooth(args):
     e0.record(stream)
     for _ in range(Ke):
         step(kh.to(dev, non_blocking=True))
-        for h, d in zip(oh, (codes, scales, mean)):
+        for h, d in zip(oh, outs):
             h.copy_(d, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / Ke, world)
     fmha.get_device_error()
     line = {
-        "metric": "K smoothing GB/s (token mean per channel + INT8 quantization of K - mean: 4 B read + 1 B written "
-                  "per element)",
+        "metric": SMOOTH_METRIC if smooth else QUANT_METRIC,
         "value": round(world * gbs, 1), "unit": "GB/s", "n_gpus": world, "steps": K_, "warmup": args.warmup,
         "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16->int8", "data": "synthetic (seeded; the Sage workload's K, N(0,1) + per-channel N(0,2) bias)",
@@ -702,15 +713,16 @@ def run_smooth(args):
         "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": round(hbm, 1), "unit": "GB/s",
                      "frac": round(gbs / hbm, 4), "traffic": None, "peak_note": f"{src}: HBM copy bandwidth",
                      "algorithmic_bytes": int(algo),
-                     "kernel": "channel_mean_partial_kernel + channel_mean_final_kernel + quant_token_block_kernel",
+                     "kernel": ("channel_mean_partial_kernel + channel_mean_final_kernel + quant_token_block_kernel"
+                                if smooth else "quant_token_block_kernel"),
                      "kernel_ms": round(ms, 5)},
         "e2e": {"value": round(world * algo / (e2e_ms * 1e-3) / 1e9, 1), "unit": "GB/s",
                 "h2d_bytes_per_step": k.numel() * 2, "d2h_bytes_per_step": out_bytes, "steps": Ke},
-        "gpu_launches": 3 * K_,
+        "gpu_launches": (3 if smooth else 1) * K_,
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        dt, nbytes = smooth_oracle_sample(kh, heads=2)
+        dt, nbytes = smooth_oracle_sample(kh, heads=2, smooth=smooth)
         line["cpu_baseline"] = {"value": round(nbytes / dt / 1e9, 6), "unit": "GB/s", "cores": cpu_cores(),
                                 "kind": "oracle", "sample": f"heads 0..1 of {H}, NumPy oracle, {dt:.2f} s"}
     if rank == 0:
@@ -718,16 +730,17 @@ def run_smooth(args):
     teardown(world)
 
 
-def smooth_oracle_sample(kh, heads):
-    """The oracle's channel mean + shifted quantizer on the first `heads` heads: (seconds, algorithmic bytes)."""
+def smooth_oracle_sample(kh, heads, smooth=True):
+    """The oracle's channel mean + shifted quantizer (or the quantizer alone) on the
+    first `heads` heads: (seconds, algorithmic bytes)."""
     from oracle import quant as oq
 
     x = kh[:, :, :heads].to(torch.float32).numpy()
     t = time.perf_counter()
-    mu = oq.channel_mean(x)
+    mu = oq.channel_mean(x) if smooth else None
     oq.quantize_blockwise(x, "int8", "per_token_block", 64, shift=mu)
     dt = time.perf_counter() - t
-    return dt, x.size * 5
+    return dt, x.size * (5 if smooth else 3)
 
 
 def run_reference_smooth(args):
@@ -735,20 +748,20 @@ def run_reference_smooth(args):
         return
     from precision_attention_fmha_b200 import workloads
 
-    _, B, H, _, S, D, _ = WORKLOADS[args.workload]
+    kind, B, H, _, S, D, _ = WORKLOADS[args.workload]
+    smooth = kind == "smooth_k"
     kh = workloads.sage(S=S, B=B, H=H, D=D)["k"].contiguous()
     heads = 2  # a bounded sample of the H heads per step
     for _ in range(args.warmup):
-        smooth_oracle_sample(kh, heads)
+        smooth_oracle_sample(kh, heads, smooth)
     times, nbytes = [], 0
     for _ in range(args.steps):
-        dt, nbytes = smooth_oracle_sample(kh, heads)
+        dt, nbytes = smooth_oracle_sample(kh, heads, smooth)
         times.append(dt)
     ms = 1e3 * sum(times) / len(times)
     val = nbytes / (ms * 1e-3) / 1e9
     print(json.dumps({
-        "impl": "reference", "metric": "K smoothing GB/s (token mean per channel + INT8 quantization of K - mean: "
-                                       "4 B read + 1 B written per element)",
+        "impl": "reference", "metric": SMOOTH_METRIC if smooth else QUANT_METRIC,
         "value": round(val, 6), "unit": "GB/s", "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 3), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f32", "data": "synthetic (seeded; the Sage workload's K)",
@@ -799,9 +812,10 @@ def main():
         args.warmup = 3
     kind = WORKLOADS[args.workload][0]
     if args.impl == "reference":
-        {"nvfp4": run_reference_nvfp4, "smooth_k": run_reference_smooth}.get(kind, run_reference)(args)
+        {"nvfp4": run_reference_nvfp4, "smooth_k": run_reference_smooth,
+         "quant_k": run_reference_smooth}.get(kind, run_reference)(args)
     else:
-        {"nvfp4": run_nvfp4, "smooth_k": run_smooth}.get(kind, run_ours)(args)
+        {"nvfp4": run_nvfp4, "smooth_k": run_smooth, "quant_k": run_smooth}.get(kind, run_ours)(args)
 
 
 if __name__ == "__main__":

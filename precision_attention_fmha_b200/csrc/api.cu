@@ -115,7 +115,8 @@ EncodeTiledFn encode_fn(cudaError_t* err) {
 // the descriptor stays valid whatever the caller's stride.
 template <int RANK>
 fmha_status make_map_n(CUtensorMap* map, void* base, int elem_bytes, const uint64_t (&dims)[RANK],
-                       const int64_t (&strides_elems)[RANK - 1], const uint32_t (&box)[RANK], const char* what) {
+                       const int64_t (&strides_elems)[RANK - 1], const uint32_t (&box)[RANK], const char* what,
+                       CUtensorMapSwizzle swizzle = CU_TENSOR_MAP_SWIZZLE_128B) {
   cudaError_t e;
   EncodeTiledFn fn = encode_fn(&e);
   if (fn == nullptr) return fail(FMHA_ERR_CUDA, "cuTensorMapEncodeTiled unavailable: %s", cudaGetErrorString(e));
@@ -137,7 +138,7 @@ fmha_status make_map_n(CUtensorMap* map, void* base, int elem_bytes, const uint6
   }
   const CUtensorMapDataType dt = elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
   CUresult r = fn(map, dt, RANK, base, gdim, gstride, bdim, ebox, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                  swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(FMHA_ERR_INVALID_ARG, "TMA descriptor for %s rejected (CUresult %d)", what, (int)r);
   return FMHA_OK;
 }
@@ -588,7 +589,27 @@ fmha_status quantize_impl(const fmha_tensor* src, const float* shift, const fmha
   p.ws = static_cast<uint32_t*>(workspace);
   p.rows_per_cta = 2048 / (D / 8) > 0 ? 2048 / (D / 8) : 1;
   p.shift = shift;
-  cudaError_t e = launch_quantize(dst->dtype == FMHA_E4M3, p, stream);
+  cudaError_t e;
+  p.err = device_error_word(&e);
+  if (p.err == nullptr) return fail(FMHA_ERR_CUDA, "device error word: %s", cudaGetErrorString(e));
+  const uint64_t wc = g_wait_cycles.load();
+  p.wait_cycles = wc ? wc : kDefaultWaitCycles;
+  // Token blocks of at most 32 KB whose rows TMA can address (16-byte strides,
+  // D <= 256 elements per box row, D / 8 a power of two) are staged whole in
+  // shared memory by TMA.
+  CUtensorMap tm;
+  const CUtensorMap* tm_src = nullptr;
+  auto stride_ok = [](int64_t st, int n) { return n <= 1 || (st > 0 && st % 8 == 0); };
+  if (kind == FMHA_SF_PER_TOKEN_BLOCK && S > 0 && D <= 256 && ((D / 8) & (D / 8 - 1)) == 0 && p.rpb <= 256 &&
+      static_cast<int64_t>(p.rpb) * D * 2 <= 32768 && stride_ok(p.s_sh, H) && stride_ok(p.s_ss, S) &&
+      stride_ok(p.s_sb, B)) {
+    const uint64_t dims[4] = {uint64_t(D), uint64_t(H), uint64_t(S), uint64_t(B)};
+    const int64_t strides[3] = {p.s_sh, p.s_ss, p.s_sb};
+    const uint32_t box[4] = {uint32_t(D), 1u, uint32_t(p.rpb), 1u};
+    if (make_map_n<4>(&tm, src->ptr, 2, dims, strides, box, "src", CU_TENSOR_MAP_SWIZZLE_NONE) == FMHA_OK)
+      tm_src = &tm;
+  }
+  e = launch_quantize(dst->dtype == FMHA_E4M3, p, tm_src, stream);
   if (e != cudaSuccess) return fail(FMHA_ERR_CUDA, "quantizer launch: %s", cudaGetErrorString(e));
   return ok_status();
 }

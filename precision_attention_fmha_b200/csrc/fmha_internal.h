@@ -86,13 +86,17 @@ struct QuantParams {
   double* partial;       // [B, H, n_chunks, D]
   float* mean;           // [B, H, D]
   int32_t n_chunks;
+  uint32_t* err;         // device error word (a timed-out wait sets kErrTimeout)
+  uint64_t wait_cycles;  // limit of one wait
 };
 
 // Launchers (defined in the .cu files). They return cudaSuccess or the launch error.
 cudaError_t launch_attention(int qk_kind, int pv_kind, int D, bool paged, const AttnParams& p,
                              const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                              const CUtensorMap& to, cudaStream_t stream);
-cudaError_t launch_quantize(bool to_e4m3, const QuantParams& p, cudaStream_t stream);
+// tm_src (nullable): TMA map of the source as [D, H, S, B] with box [D, 1, rows_per_block, 1];
+// token-block quantization then stages whole blocks in shared memory.
+cudaError_t launch_quantize(bool to_e4m3, const QuantParams& p, const CUtensorMap* tm_src, cudaStream_t stream);
 cudaError_t launch_channel_mean(const QuantParams& p, cudaStream_t stream);
 // Decode path: attention over GQA-packed tiles (p.packed = 1), then, for
 // n_splits > 1, the split merge into o (bf16, element strides) and lse.
