@@ -286,6 +286,10 @@ fmha_status run_attention(const fmha_args* a, const uint8_t* mask, int64_t msb, 
   if (D == 64 && !(qk == QK_BF16 && pv == PV_BF16)) return fail(FMHA_ERR_UNSUPPORTED, "D=64 needs BF16 Q/K/V");
   if (D == 192 && (qk == QK_INT8 || dout != FMHA_BF16 || a->p_terms == 2 || dec != nullptr))
     return fail(FMHA_ERR_UNSUPPORTED, "D=192: BF16 or E4M3 Q/K, one-term P, BF16 O, not decode");
+  // One query tile per CTA: its kept KV tiles are dealt to the two softmax
+  // warpgroups through a 1024-bit keep set.
+  if (query_tiles_per_cta(qk, D) == 1 && ceil_div(Skv, 128) > 1024)
+    return fail(FMHA_ERR_UNSUPPORTED, "D=192 with BF16 Q/K: Skv %d > 131072", Skv);
   const bool packed = dec != nullptr;
   const bool o8 = dout == FMHA_E4M3;
   if (o8 && Dv != 128) return fail(FMHA_ERR_UNSUPPORTED, "E4M3 O needs D = 128");

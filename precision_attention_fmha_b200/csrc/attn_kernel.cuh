@@ -87,13 +87,22 @@ struct AttnCfg {
   // Query tiles per CTA (1 when two 48 KB BF16 Q tiles would starve the K/V ring).
   static constexpr int NQ = query_tiles_per_cta(QK, D);
   static_assert(NQ == 2 || !PACKED, "decode tiles come in pairs");
-  static constexpr int P_BYTES = PSMEM ? NQ * P_TILE * (P2 ? 2 : 1) : 0;
+  // One query tile: the two softmax warpgroups take alternate kept KV tiles of
+  // it (an intra-CTA split of the keys), each with its own S, P and O, and the
+  // epilogue merges the two partial results. K and V then have rings of their
+  // own (2 slots each: a 48 KB K slot and a 32 KB V slot are not interchangeable).
+  static constexpr bool SPLIT = NQ == 1;
+  static_assert(!SPLIT || (!O8 && !P2), "split tiles: BF16 O, one-term P");
+  static constexpr int P_BYTES = PSMEM ? 2 * P_TILE * (P2 ? 2 : 1) : 0;
   static constexpr int MISC_BYTES = 2048;
   static constexpr int SMEM_CAP = 232448;  // 227 KB opt-in maximum per CTA
   static constexpr int STAGES_FIT = (SMEM_CAP - 1024 - MISC_BYTES - NQ * Q_TILE - P_BYTES) / SLOT;
   static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
-  static_assert(STAGES >= 3, "the K/V ring needs at least three slots");
-  static constexpr int SMEM_BYTES = 1024 + NQ * Q_TILE + P_BYTES + STAGES * SLOT + MISC_BYTES;
+  static_assert(SPLIT || STAGES >= 3, "the K/V ring needs at least three slots");
+  static constexpr int K_STAGES = 2, V_STAGES = 2;  // split rings
+  static constexpr int RING_BYTES = SPLIT ? K_STAGES * K_TILE + V_STAGES * V_TILE : STAGES * SLOT;
+  static constexpr int SMEM_BYTES = 1024 + NQ * Q_TILE + P_BYTES + RING_BYTES + MISC_BYTES;
+  static_assert(SMEM_BYTES <= SMEM_CAP, "shared memory");
   static constexpr int QK_STEPS = QK_ROW_BYTES / 32;  // one MMA covers 32 bytes of K (16 bf16 / 32 8-bit)
   static constexpr int PV_K = PV == PV_BF16 ? 16 : 32;
   static constexpr int PV_STEPS = BN / PV_K;
@@ -136,7 +145,8 @@ struct alignas(8) AttnMisc {
   // mask: built once in the prologue, so no role reads the mask per tile.
   uint32_t keep_bits[2][32];
   int32_t range[2][2];  // packed: [first, last + 1) of each query tile's kept tiles
-  int32_t same_kept;    // masked: both query tiles keep the same KV tiles (count), else 0
+  int32_t same_kept;    // masked: both query tiles keep the same KV tiles (count), else 0;
+                        // split tiles: the kept tiles each warpgroup has at least
 };
 
 static_assert(sizeof(AttnMisc) <= 2048, "AttnMisc must fit the 2 KB misc area");
@@ -216,7 +226,7 @@ struct Waiter {
 // split's tiles; masked launches: the block mask's kept tiles).
 template <class C>
 __device__ __forceinline__ bool uses_keep_bits(const AttnParams& p) {
-  return C::PACKED || p.mask != nullptr;
+  return C::PACKED || C::SPLIT || p.mask != nullptr;
 }
 
 template <class C>
@@ -357,6 +367,80 @@ __device__ void attn_load_role(const AttnParams& p, const TileInfo t0, const Til
   if (lane == 0) {
     w.drain(q_full, 0);
     for (int s = 0; s < C::STAGES; ++s)
+      if (issued & (1u << s)) w.drain(smem_addr(&misc->kv_full[s]), (issued_phase >> s) & 1u);
+  }
+  __syncwarp();
+}
+
+// TMA producer for split tiles (one query tile, two softmax warpgroups taking
+// alternate kept KV tiles): Q once, then per pair of kept tiles (a, b) their K
+// tiles into the K ring and then their V tiles into the V ring, so the next
+// pair's K is in flight while this pair's V waits for a free slot. Barriers:
+// kv_full/kv_empty [0, K_STAGES) for K, [K_STAGES, K_STAGES + V_STAGES) for V.
+template <class C>
+__device__ void attn_load_role_split(const AttnParams& p, const TileInfo t0, int b, int hkv, uint8_t* sQ,
+                                     uint8_t* sK, uint8_t* sV, AttnMisc* misc, const CUtensorMap* tmQ,
+                                     const CUtensorMap* tmK, const CUtensorMap* tmV, const Waiter w) {
+  using namespace ptx;
+  constexpr uint32_t FULL = 0xffffffffu;
+  const int lane = threadIdx.x & 31;
+  const uint32_t q_full = smem_addr(&misc->q_full);
+  if (lane == 0) mbar_arrive_expect_tx(q_full, C::Q_TILE);
+  __syncwarp();
+  if (lane < C::QK_CHUNKS)
+    tma_load_4d(smem_addr(sQ) + lane * C::CHUNK_BYTES, tmQ, q_full, lane * C::QK_CHUNK_ELEMS, t0.h, t0.q0, b);
+  const uint64_t pol = policy_evict_last();  // K/V tiles are re-read by every CTA of this head
+  uint32_t issued = 0u, issued_phase = 0u;    // per barrier: a load was issued / parity of its last phase
+  int it[2] = {0, 0};                         // K and V ring positions
+  bool ok = true;
+  const int n = t0.n_kv;
+  const int per = C::PAGED ? C::BN / p.page_size : 1;
+  // One K (kv = 0) or V (kv = 1) tile u into its ring: lane l issues copy l
+  // (page l / chunks, chunk l % chunks), the page entry read here.
+  auto load = [&](int kv, int u) {
+    const int ring = kv ? C::K_STAGES : 0, stages = kv ? C::V_STAGES : C::K_STAGES;
+    const int s = it[kv] % stages;
+    const uint32_t ph = (it[kv] / stages) & 1;
+    ++it[kv];
+    if (!(ok = __all_sync(FULL, w.wait(smem_addr(&misc->kv_empty[ring + s]), ph ^ 1)))) return;
+    const uint32_t full = smem_addr(&misc->kv_full[ring + s]);
+    const int chunks = kv == 0 ? C::QK_CHUNKS : C::V_CHUNKS;
+    const int chunk_elems = kv == 0 ? C::QK_CHUNK_ELEMS : C::V_CHUNK_ELEMS;
+    const CUtensorMap* tm = kv == 0 ? tmK : tmV;
+    const uint32_t dst = kv == 0 ? smem_addr(sK + s * C::K_TILE) : smem_addr(sV + s * C::V_TILE);
+    if (lane == 0) mbar_arrive_expect_tx(full, kv == 0 ? C::K_TILE : C::V_TILE);
+    __syncwarp();
+    issued |= 1u << (ring + s);
+    issued_phase = (issued_phase & ~(1u << (ring + s))) | (ph << (ring + s));
+    if constexpr (!C::PAGED) {
+      if (lane < chunks)
+        tma_load_4d_hint(dst + lane * C::CHUNK_BYTES, tm, full, lane * chunk_elems, hkv, u * C::BN, b, pol);
+    } else {
+      const int pp = lane / chunks, c = lane - pp * chunks;
+      const int lp = u * per + pp;  // logical page of this sequence
+      int pg = p.num_pages;         // out of range: TMA reads zeros
+      if (pp < per && lp * p.page_size < p.Skv) {
+        const int e = __ldg(p.page_table + static_cast<int64_t>(b) * p.max_pages_per_seq + lp);
+        if (e < 0 || e >= p.num_pages) atomicOr(p.err, kErrPageIndex);
+        else pg = e;
+      }
+      if (pp < per)
+        tma_load_4d_hint(dst + c * C::CHUNK_BYTES + pp * p.page_size * 128, tm, full, c * chunk_elems, hkv, 0, pg,
+                         pol);
+    }
+  };
+  for (int ua = next_kept_tile<C>(p, misc, 3, t0.u0, n); ua < n && ok;) {
+    const int ub = next_kept_tile<C>(p, misc, 3, ua + 1, n);
+    load(0, ua);
+    if (ok && ub < n) load(0, ub);
+    if (ok) load(1, ua);
+    if (ok && ub < n) load(1, ub);
+    ua = ub < n ? next_kept_tile<C>(p, misc, 3, ub + 1, n) : n;
+  }
+  // Every issued copy lands before shared memory goes away (see attn_load_role).
+  if (lane == 0) {
+    w.drain(q_full, 0);
+    for (int s = 0; s < C::K_STAGES + C::V_STAGES; ++s)
       if (issued & (1u << s)) w.drain(smem_addr(&misc->kv_full[s]), (issued_phase >> s) & 1u);
   }
   __syncwarp();
@@ -513,6 +597,71 @@ __device__ void attn_mma_role(const AttnParams& p, const TileInfo t0, const Tile
   w.drain(smem_addr(&misc->drain), 0);
 }
 
+// MMA issue for split tiles with P in TMEM (BF16 P). Kept tiles alternate
+// between the softmax warpgroups (tile x = the keep-bit owner of u). Per kept
+// tile u of warpgroup x: its pending PV_x (P_x lives over S_x in TMEM, so it
+// must precede S_x(u)), then S_x(u) = Q K_u^T. A K slot is released when its
+// QK^T completes, a V slot when its PV completes.
+template <class C>
+__device__ void attn_mma_role_split(const AttnParams& p, const TileInfo t0, const TileInfo t1, uint8_t* sQ,
+                                    uint8_t* sK, uint8_t* sV, AttnMisc* misc, uint32_t tmem, const Waiter w) {
+  using namespace ptx;
+  constexpr uint32_t FULL = 0xffffffffu;
+  const bool leader = elect_one();
+  const uint32_t s_col[2] = {0u, 128u};
+  const uint32_t o_col[2] = {256u, 256u + C::DV};
+  const uint32_t hi = desc_hi(1024, 2);
+  const uint32_t q_lo = desc_lo(smem_addr(sQ), 16);
+  const uint32_t k_lo0 = desc_lo(smem_addr(sK), 16);
+  const uint32_t v_lo0 = desc_lo(smem_addr(sV), C::CHUNK_BYTES);
+  int pend[2] = {-1, -1};  // V slot of the warpgroup's pending PV
+  uint32_t pend_ph[2] = {0u, 0u};
+  int pv_cnt[2] = {0, 0};
+  int k_it = 0, v_it = 0;
+  const int n = t0.n_kv;
+  bool ok = __all_sync(FULL, w.wait(smem_addr(&misc->q_full), 0));
+  tc_fence_after();
+  auto issue_pending_pv = [&](int x) {
+    if (pend[x] < 0) return;
+    if (!(ok = __all_sync(FULL, w.wait(smem_addr(&misc->p_full[x]), pv_cnt[x] & 1)))) return;
+    if (!(ok = __all_sync(FULL, w.wait(smem_addr(&misc->kv_full[C::K_STAGES + pend[x]]), pend_ph[x])))) return;
+    tc_fence_after();
+    if (leader) {
+      issue_pv<C>(tmem + o_col[x], tmem + s_col[x], v_lo0 + pend[x] * (C::V_TILE >> 4), hi, pv_cnt[x] > 0);
+      tc_commit(smem_addr(&misc->kv_empty[C::K_STAGES + pend[x]]));  // V slot free once the PV finishes
+    }
+    __syncwarp();
+    ++pv_cnt[x];
+    pend[x] = -1;
+  };
+  for (int u = next_kept_tile<C>(p, misc, 3, t0.u0, n); u < n && ok; u = next_kept_tile<C>(p, misc, 3, u + 1, n)) {
+    const int x = keep_tile<C>(p, t1, u, misc) ? 1 : 0;
+    issue_pending_pv(x);
+    if (!ok) break;
+    const int ks = k_it % C::K_STAGES;
+    const uint32_t kph = (k_it / C::K_STAGES) & 1;
+    ++k_it;
+    if (!(ok = __all_sync(FULL, w.wait(smem_addr(&misc->kv_full[ks]), kph)))) break;
+    tc_fence_after();
+    if (leader) {
+      issue_qk<C>(tmem + s_col[x], q_lo, k_lo0 + ks * (C::K_TILE >> 4), hi);
+      tc_commit(smem_addr(&misc->s_full[x]));
+      tc_commit(smem_addr(&misc->kv_empty[ks]));  // K slot free once S_x(u) finishes
+    }
+    __syncwarp();
+    pend[x] = v_it % C::V_STAGES;
+    pend_ph[x] = (v_it / C::V_STAGES) & 1;
+    ++v_it;
+  }
+  for (int x = 0; x < 2 && ok; ++x) issue_pending_pv(x);
+  if (leader) {
+    if (ok) tc_commit(smem_addr(&misc->o_full));
+    tc_commit(smem_addr(&misc->drain));
+  }
+  __syncwarp();
+  w.drain(smem_addr(&misc->drain), 0);
+}
+
 // Shared-memory P: O += P V with P (A operand, K-major, 128-byte swizzle)
 // read from shared memory. K-steps of 32 keys advance 32 bytes in the row.
 template <class C>
@@ -522,6 +671,84 @@ __device__ __forceinline__ void issue_pv_ss(uint32_t tmem_o, uint32_t p_lo, uint
   for (int s = 0; s < C::PV_STEPS; ++s)
     ptx::mma_ss_f8_lean_acc(tmem_o, p_lo + ((s * 32) >> 4), hi, v_lo + ((s * C::PV_K * 128) >> 4), hi,
                             C::IDESC_PV, s > 0 ? 1u : accumulate);
+}
+
+// MMA issue for split tiles with P in shared memory (E4M3 P). Per pair of kept
+// tiles (a for warpgroup 0, b for warpgroup 1): QK^T of the NEXT pair as soon as
+// each softmax has loaded its current S (s_free), then PV_0(a), PV_1(b) once
+// their P is in shared memory (p_full), committed to pv_done[x].
+template <class C>
+__device__ void attn_mma_role_psmem_split(const AttnParams& p, const TileInfo t0, uint8_t* sQ, uint8_t* sP0,
+                                          uint8_t* sP1, uint8_t* sK, uint8_t* sV, AttnMisc* misc, uint32_t tmem,
+                                          const Waiter w) {
+  using namespace ptx;
+  constexpr uint32_t FULL = 0xffffffffu;
+  const bool leader = elect_one();
+  const uint32_t hi = desc_hi(1024, 2);
+  const uint32_t q_lo = desc_lo(smem_addr(sQ), 16);
+  const uint32_t p_lo[2] = {desc_lo(smem_addr(sP0), 16), desc_lo(smem_addr(sP1), 16)};
+  const uint32_t k_lo0 = desc_lo(smem_addr(sK), 16);
+  const uint32_t v_lo0 = desc_lo(smem_addr(sV), C::CHUNK_BYTES);
+  const uint32_t s_col[2] = {0u, 128u};
+  const uint32_t o_col[2] = {256u, 256u + C::DV};
+  const int n = t0.n_kv;
+  int s_cnt[2] = {0, 0}, pv_cnt[2] = {0, 0};
+  int k_it = 0, v_it = 0;
+  bool ok = __all_sync(FULL, w.wait(smem_addr(&misc->q_full), 0));
+  tc_fence_after();
+  auto next = [&](int from) { return next_kept_tile<C>(p, misc, 3, from, n); };
+  // S_x(u) into warpgroup x's S columns, from the next K slot.
+  auto issue_s = [&](int x) {
+    const int ks = k_it % C::K_STAGES;
+    const uint32_t kph = (k_it / C::K_STAGES) & 1;
+    ++k_it;
+    if (s_cnt[x] > 0) {  // the softmax must have loaded this warpgroup's previous S
+      if (!(ok = __all_sync(FULL, w.wait(smem_addr(&misc->s_free[x]), (s_cnt[x] - 1) & 1)))) return;
+    }
+    if (!(ok = __all_sync(FULL, w.wait(smem_addr(&misc->kv_full[ks]), kph)))) return;
+    tc_fence_after();
+    if (leader) {
+      issue_qk<C>(tmem + s_col[x], q_lo, k_lo0 + ks * (C::K_TILE >> 4), hi);
+      tc_commit(smem_addr(&misc->s_full[x]));
+      tc_commit(smem_addr(&misc->kv_empty[ks]));
+    }
+    __syncwarp();
+    ++s_cnt[x];
+  };
+  // O_x += P_x V from the next V slot, once the softmax has written P_x.
+  auto issue_pv = [&](int x) {
+    const int vs = v_it % C::V_STAGES;
+    const uint32_t vph = (v_it / C::V_STAGES) & 1;
+    ++v_it;
+    if (!(ok = __all_sync(FULL, w.wait(smem_addr(&misc->p_full[x]), pv_cnt[x] & 1)))) return;
+    if (!(ok = __all_sync(FULL, w.wait(smem_addr(&misc->kv_full[C::K_STAGES + vs]), vph)))) return;
+    tc_fence_after();
+    if (leader) {
+      issue_pv_ss<C>(tmem + o_col[x], p_lo[x], v_lo0 + vs * (C::V_TILE >> 4), hi, pv_cnt[x] > 0);
+      tc_commit(smem_addr(&misc->pv_done[x]));
+      tc_commit(smem_addr(&misc->kv_empty[C::K_STAGES + vs]));
+    }
+    __syncwarp();
+    ++pv_cnt[x];
+  };
+  int ua = next(t0.u0);
+  int ub = ua < n ? next(ua + 1) : n;
+  if (ua < n && ok) issue_s(0);
+  if (ub < n && ok) issue_s(1);
+  while (ua < n && ok) {
+    const int na = ub < n ? next(ub + 1) : n;
+    const int nb = na < n ? next(na + 1) : n;
+    if (na < n) issue_s(0);
+    if (nb < n && ok) issue_s(1);
+    if (!ok) break;
+    issue_pv(0);
+    if (ub < n && ok) issue_pv(1);
+    ua = na;
+    ub = nb;
+  }
+  if (leader) tc_commit(smem_addr(&misc->drain));
+  __syncwarp();
+  w.drain(smem_addr(&misc->drain), 0);
 }
 
 // MMA issue for the shared-memory-P pipeline. Per kept KV tile u (in order):
@@ -688,8 +915,8 @@ __device__ __forceinline__ void exp2_poly_x2(float& a, float& b) {
 // this tile's E4M3 P is stored was measured 10 % slower.)
 template <class C>
 __device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, int b, int hkv, uint8_t* sQx,
-                                  uint8_t* sPx, int n_turns, AttnMisc* misc, uint32_t tmem, const CUtensorMap* tmO,
-                                  const Waiter w) {
+                                  uint8_t* sPx, uint8_t* sX, int n_turns, AttnMisc* misc, uint32_t tmem,
+                                  const CUtensorMap* tmO, const Waiter w) {
   using namespace ptx;
   constexpr uint32_t FULL = 0xffffffffu;
   constexpr int NCH = C::BN / 32;  // 32-key chunks per tile (one TMEM load each)
@@ -977,6 +1204,69 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, 
   const float inv_l = l > 0.f ? sfv / l : 0.f;
   const uint32_t stage0 = smem_addr(sQx);
   constexpr uint32_t TILE_THREADS = 128;
+  if constexpr (C::SPLIT) {
+    // Split tiles: both warpgroups hold partial results (m, l, O) of the same
+    // rows over disjoint keys. Once both have seen their last PV finish, every
+    // MMA of the CTA is done and the K/V ring is free: (m, l) per row go
+    // through it, and warpgroup x merges and stores columns [64x, 64x + 64):
+    // O = (O_0 2^(m_0 - M) + O_1 2^(m_1 - M)) / (l_0 2^(m_0 - M) + l_1 2^(m_1 - M)).
+    named_bar_sync(3, 2 * TILE_THREADS);
+    float2* ex = reinterpret_cast<float2*>(sX);
+    ex[x * 128 + r] = make_float2(have_o ? m : -INFINITY, have_o ? l : -1.f);  // l < 0: no O
+    named_bar_sync(3, 2 * TILE_THREADS);
+    const float2 e0 = ex[r], e1 = ex[128 + r];
+    const bool h0 = e0.y > 0.f, h1 = e1.y > 0.f;
+    const float M = fmaxf(h0 ? e0.x : -INFINITY, h1 ? e1.x : -INFINITY);
+    const float c0 = h0 ? ex2(e0.x - M) : 0.f, c1 = h1 ? ex2(e1.x - M) : 0.f;
+    const float L = (h0 ? e0.y * c0 : 0.f) + (h1 ? e1.y * c1 : 0.f);
+    const float inv = L > 0.f ? sfv / L : 0.f;
+    // Columns [64x, 64x + 64) of both accumulators (a warpgroup without tiles
+    // left its O undefined: its values are selected away, never multiplied).
+    const uint32_t tO0 = tmem + lane_off + 256u + 64u * x, tO1 = tO0 + C::DV;
+    uint32_t o0[2][32], o1[2][32];
+    tmem_ld32(tO0, o0[0]);
+    tmem_ld32(tO0 + 32, o0[1]);
+    tmem_ld32(tO1, o1[0]);
+    tmem_ld32(tO1 + 32, o1[1]);
+    tmem_wait_ld();
+    reg_fence(o0[0]);
+    reg_fence(o0[1]);
+    reg_fence(o1[0]);
+    reg_fence(o1[1]);
+    auto out_val = [&](int col) {
+      const float a = h0 ? __uint_as_float(o0[col >> 5][col & 31]) * c0 : 0.f;
+      const float b2 = h1 ? __uint_as_float(o1[col >> 5][col & 31]) * c1 : 0.f;
+      float v = (a + b2) * inv;
+      if (C::PV == PV_E4M3 && p.sf_v_kind == FMHA_SF_PER_CHANNEL) v *= misc->sf_v[64 * x + col];
+      return v;
+    };
+    const uint32_t buf = stage0 + x * C::CHUNK_BYTES;
+    const uint32_t base = buf + r * 128;
+#pragma unroll
+    for (int sc = 0; sc < 2; ++sc) {
+      uint32_t pk[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) pk[j] = pack_bf16x2(out_val(32 * sc + 2 * j), out_val(32 * sc + 2 * j + 1));
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        const int k = 4 * sc + kk;
+        const uint32_t addr = base + ((k ^ (r & 7)) << 4);
+        asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(pk[4 * kk]), "r"(pk[4 * kk + 1]),
+                     "r"(pk[4 * kk + 2]), "r"(pk[4 * kk + 3])
+                     : "memory");
+      }
+    }
+    fence_proxy_async_smem();
+    named_bar_sync(1 + x, TILE_THREADS);
+    if (lead && ok) {
+      tma_store_4d(tmO, buf, 64 * x, t.h, t.q0, b);
+      bulk_commit();
+    }
+    if (x == 0 && p.lse != nullptr && row < p.Sq && ok)
+      p.lse[bhq * p.Sq + row] = L > 0.f ? (M + __log2f(L) - log2g) * 0.69314718055994531f : -INFINITY;
+    if (lead) bulk_wait0();
+    return;
+  }
   if constexpr (C::O8) {
     // E4M3 output: the whole 128-column row is 128 bytes, one swizzled
     // 128 x 128-byte chunk (the size and layout of a 64-column BF16 chunk),
@@ -1099,9 +1389,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
   // Q buffers, then E4M3 P buffers (shared-memory P), then the K/V ring. With one
   // query tile per CTA the second tile's pointers alias the first (never used).
   uint8_t* const sQ[2] = {smem, smem + (C::NQ - 1) * C::Q_TILE};
-  uint8_t* const sP[2] = {smem + C::NQ * C::Q_TILE, smem + C::NQ * C::Q_TILE + (C::NQ - 1) * (C::P_BYTES / C::NQ)};
-  uint8_t* sSlots = smem + C::NQ * C::Q_TILE + C::P_BYTES;
-  AttnMisc* misc = reinterpret_cast<AttnMisc*>(sSlots + C::STAGES * C::SLOT);
+  uint8_t* const sP[2] = {smem + C::NQ * C::Q_TILE, smem + C::NQ * C::Q_TILE + C::P_BYTES / 2};
+  uint8_t* sSlots = smem + C::NQ * C::Q_TILE + C::P_BYTES;  // the K/V ring (split: K ring, then V ring)
+  AttnMisc* misc = reinterpret_cast<AttnMisc*>(sSlots + C::RING_BYTES);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   // ---- work item -> (b, heads, query rows) ----
@@ -1188,15 +1478,14 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     }
   } else {
     int item = blockIdx.x;
-    if (C::NQ == 1) {  // SINGLE: one query block of one head; tile 1 stays empty
+    if (C::SPLIT) {  // SINGLE: one query block of one head, its kept KV tiles split between the warpgroups
       int qb = item % p.n_units;
       item /= p.n_units;
       const int h = item % p.Hq;
       b = item / p.Hq;
       if (p.causal) qb = p.n_units - 1 - qb;  // heaviest causal tiles first
       t[0].h = t[1].h = h;
-      t[0].qblk = qb;
-      t[1].qblk = p.n_q_blocks;  // past the end: not valid
+      t[0].qblk = t[1].qblk = qb;
     } else if (p.pair_mode == PAIR_ROWS) {
       int pr = item % p.n_units;
       item /= p.n_units;
@@ -1234,10 +1523,33 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       }
       t[x].n_kv = t[x].valid ? n : 0;
     }
+    // Split tiles: warp 2 gives the kept KV tiles (causal bound, block mask) of
+    // the query tile alternately to the two warpgroups: ranks 0, 2, 4, ... to
+    // warpgroup 0 and 1, 3, 5, ... to warpgroup 1. same_kept holds the number
+    // of tiles both have (exp turn-taking runs over those).
+    if (C::SPLIT && warp == 2) {
+      const int n_words = (t[0].n_kv + 31) >> 5;
+      const uint8_t* mrow = p.mask == nullptr ? nullptr
+                            : p.mask + b * p.mask_sb + hkv * p.mask_sh + static_cast<int64_t>(t[0].mrow) * p.n_kv_blocks;
+      int total = 0;
+      for (int wd = 0; wd < n_words; ++wd) {
+        const int u = (wd << 5) + lane;
+        const bool kept = u < t[0].n_kv && (mrow == nullptr || mrow[u] != 0);
+        const uint32_t kb = __ballot_sync(0xffffffffu, kept);
+        const int rank = total + __popc(kb & ((1u << lane) - 1u));
+        const uint32_t even = __ballot_sync(0xffffffffu, kept && (rank & 1) == 0);
+        if (lane == 0) {
+          misc->keep_bits[0][wd] = even;
+          misc->keep_bits[1][wd] = kb & ~even;
+        }
+        total += __popc(kb);
+      }
+      if (lane == 0) misc->same_kept = total >> 1;
+    }
     // Masked launch: warp 2 (otherwise idle) turns each query tile's block-mask
     // row into the keep-bit set (one coalesced 32-byte read per word), and
     // records whether both tiles keep the same KV tiles.
-    if (p.mask != nullptr && warp == 2) {
+    if (!C::SPLIT && p.mask != nullptr && warp == 2) {
       const int n_words = (max(t[0].n_kv, t[1].n_kv) + 31) >> 5;
       bool same = t[0].n_kv == t[1].n_kv;
       int count = 0;
@@ -1270,7 +1582,7 @@ __global__ void __launch_bounds__(C::THREADS, 1)
       mbar_init(smem_addr(&misc->pv_done[x]), 1);
       mbar_init(smem_addr(&misc->exp_done[x]), 4);  // one arrive per softmax warp
     }
-    for (int s = 0; s < C::STAGES; ++s) {
+    for (int s = 0; s < (C::SPLIT ? C::K_STAGES + C::V_STAGES : C::STAGES); ++s) {
       mbar_init(smem_addr(&misc->kv_full[s]), 1);
       mbar_init(smem_addr(&misc->kv_empty[s]), 1);
     }
@@ -1314,19 +1626,28 @@ __global__ void __launch_bounds__(C::THREADS, 1)
     // mask their common prefix [0, min n_kv); with a block mask only when both
     // tiles keep the same tiles (e.g. two query heads of one KV head).
     int n_turns = 0;
-    if (C::TURNS && !C::PACKED) n_turns = p.mask == nullptr ? min(t[0].n_kv, t[1].n_kv) : misc->same_kept;
+    if (C::TURNS && !C::PACKED)
+      n_turns = (C::SPLIT || p.mask != nullptr) ? misc->same_kept : min(t[0].n_kv, t[1].n_kv);
     if (tx.valid)
-      attn_softmax_role<C>(p, tx, x, b, hkv, x ? sQ[1] : sQ[0], x ? sP[1] : sP[0], n_turns, misc, tmem, &tmO,
-                           w);
+      attn_softmax_role<C>(p, tx, x, b, hkv, x ? sQ[1] : sQ[0], x ? sP[1] : sP[0], sSlots, n_turns, misc, tmem,
+                           &tmO, w);
   } else {
     regs_dec<C::CONTROL_REGS>();
+    uint8_t* const sV = sSlots + C::K_STAGES * C::K_TILE;  // split: the V ring
     if (warp == C::MMA_WARP) {  // the whole warp; one elected lane issues
-      if constexpr (C::PSMEM)
+      if constexpr (C::SPLIT && C::PSMEM)
+        attn_mma_role_psmem_split<C>(p, t[0], sQ[0], sP[0], sP[1], sSlots, sV, misc, tmem, w);
+      else if constexpr (C::SPLIT)
+        attn_mma_role_split<C>(p, t[0], t[1], sQ[0], sSlots, sV, misc, tmem, w);
+      else if constexpr (C::PSMEM)
         attn_mma_role_psmem<C>(p, t[0], t[1], b, hkv, sQ[0], sQ[1], sP[0], sP[1], sSlots, misc, tmem, w);
       else
         attn_mma_role<C>(p, t[0], t[1], b, hkv, sQ[0], sQ[1], sSlots, misc, tmem, w);
     } else if (warp == C::LOAD_WARP) {  // the whole warp
-      attn_load_role<C>(p, t[0], t[1], b, hkv, sQ[0], sQ[1], sSlots, misc, &tmQ, &tmK, &tmV, w);
+      if constexpr (C::SPLIT)
+        attn_load_role_split<C>(p, t[0], b, hkv, sQ[0], sSlots, sV, misc, &tmQ, &tmK, &tmV, w);
+      else
+        attn_load_role<C>(p, t[0], t[1], b, hkv, sQ[0], sQ[1], sSlots, misc, &tmQ, &tmK, &tmV, w);
     }
   }
 
