@@ -99,7 +99,11 @@ struct AttnCfg {
   static constexpr int STAGES_FIT = (SMEM_CAP - 1024 - MISC_BYTES - NQ * Q_TILE - P_BYTES) / SLOT;
   static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
   static_assert(SPLIT || STAGES >= 3, "the K/V ring needs at least three slots");
-  static constexpr int K_STAGES = 2, V_STAGES = 2;  // split rings
+  // Split rings: two K slots, and as many V slots (up to 4) as the rest holds.
+  static constexpr int K_STAGES = 2;
+  static constexpr int V_FIT = (SMEM_CAP - 1024 - MISC_BYTES - NQ * Q_TILE - P_BYTES - K_STAGES * K_TILE) / V_TILE;
+  static constexpr int V_STAGES = V_FIT > 4 ? 4 : V_FIT;
+  static_assert(!SPLIT || V_STAGES >= 2, "the V ring needs two slots");
   static constexpr int RING_BYTES = SPLIT ? K_STAGES * K_TILE + V_STAGES * V_TILE : STAGES * SLOT;
   static constexpr int SMEM_BYTES = 1024 + NQ * Q_TILE + P_BYTES + RING_BYTES + MISC_BYTES;
   static_assert(SMEM_BYTES <= SMEM_CAP, "shared memory");
@@ -372,46 +376,48 @@ __device__ void attn_load_role(const AttnParams& p, const TileInfo t0, const Til
   __syncwarp();
 }
 
-// TMA producer for split tiles (one query tile, two softmax warpgroups taking
-// alternate kept KV tiles): Q once, then per pair of kept tiles (a, b) their K
-// tiles into the K ring and then their V tiles into the V ring, so the next
-// pair's K is in flight while this pair's V waits for a free slot. Barriers:
-// kv_full/kv_empty [0, K_STAGES) for K, [K_STAGES, K_STAGES + V_STAGES) for V.
+// TMA producers for split tiles (one query tile, two softmax warpgroups taking
+// alternate kept KV tiles): one warp loads Q and then the kept K tiles into
+// the K ring (kv = 0), another the kept V tiles into the V ring (kv = 1), so
+// neither ring's free slots wait on the other's. Barriers: kv_full/kv_empty
+// [0, K_STAGES) for K, [K_STAGES, K_STAGES + V_STAGES) for V.
 template <class C>
-__device__ void attn_load_role_split(const AttnParams& p, const TileInfo t0, int b, int hkv, uint8_t* sQ,
-                                     uint8_t* sK, uint8_t* sV, AttnMisc* misc, const CUtensorMap* tmQ,
-                                     const CUtensorMap* tmK, const CUtensorMap* tmV, const Waiter w) {
+__device__ void attn_load_role_split(const AttnParams& p, const TileInfo t0, int b, int hkv, int kv_sel,
+                                     uint8_t* sQ, uint8_t* sK, uint8_t* sV, AttnMisc* misc,
+                                     const CUtensorMap* tmQ, const CUtensorMap* tmK, const CUtensorMap* tmV,
+                                     const Waiter w) {
   using namespace ptx;
   constexpr uint32_t FULL = 0xffffffffu;
   const int lane = threadIdx.x & 31;
   const uint32_t q_full = smem_addr(&misc->q_full);
-  if (lane == 0) mbar_arrive_expect_tx(q_full, C::Q_TILE);
-  __syncwarp();
-  if (lane < C::QK_CHUNKS)
-    tma_load_4d(smem_addr(sQ) + lane * C::CHUNK_BYTES, tmQ, q_full, lane * C::QK_CHUNK_ELEMS, t0.h, t0.q0, b);
+  if (kv_sel == 0) {
+    if (lane == 0) mbar_arrive_expect_tx(q_full, C::Q_TILE);
+    __syncwarp();
+    if (lane < C::QK_CHUNKS)
+      tma_load_4d(smem_addr(sQ) + lane * C::CHUNK_BYTES, tmQ, q_full, lane * C::QK_CHUNK_ELEMS, t0.h, t0.q0, b);
+  }
   const uint64_t pol = policy_evict_last();  // K/V tiles are re-read by every CTA of this head
-  uint32_t issued = 0u, issued_phase = 0u;    // per barrier: a load was issued / parity of its last phase
-  int it[2] = {0, 0};                         // K and V ring positions
+  const int ring = kv_sel ? C::K_STAGES : 0, stages = kv_sel ? C::V_STAGES : C::K_STAGES;
+  const int chunks = kv_sel == 0 ? C::QK_CHUNKS : C::V_CHUNKS;
+  const int chunk_elems = kv_sel == 0 ? C::QK_CHUNK_ELEMS : C::V_CHUNK_ELEMS;
+  const uint32_t tile_bytes = kv_sel == 0 ? C::K_TILE : C::V_TILE;
+  const CUtensorMap* tm = kv_sel == 0 ? tmK : tmV;
+  const uint32_t ring_base = smem_addr(kv_sel == 0 ? sK : sV);
+  int pos = 0;  // tiles issued into this ring
   bool ok = true;
   const int n = t0.n_kv;
   const int per = C::PAGED ? C::BN / p.page_size : 1;
-  // One K (kv = 0) or V (kv = 1) tile u into its ring: lane l issues copy l
-  // (page l / chunks, chunk l % chunks), the page entry read here.
-  auto load = [&](int kv, int u) {
-    const int ring = kv ? C::K_STAGES : 0, stages = kv ? C::V_STAGES : C::K_STAGES;
-    const int s = it[kv] % stages;
-    const uint32_t ph = (it[kv] / stages) & 1;
-    ++it[kv];
+  // One tile u into the ring: lane l issues copy l (page l / chunks, chunk
+  // l % chunks), the page entry read here.
+  auto load = [&](int u) {
+    const int s = pos % stages;
+    const uint32_t ph = (pos / stages) & 1;
     if (!(ok = __all_sync(FULL, w.wait(smem_addr(&misc->kv_empty[ring + s]), ph ^ 1)))) return;
+    ++pos;
     const uint32_t full = smem_addr(&misc->kv_full[ring + s]);
-    const int chunks = kv == 0 ? C::QK_CHUNKS : C::V_CHUNKS;
-    const int chunk_elems = kv == 0 ? C::QK_CHUNK_ELEMS : C::V_CHUNK_ELEMS;
-    const CUtensorMap* tm = kv == 0 ? tmK : tmV;
-    const uint32_t dst = kv == 0 ? smem_addr(sK + s * C::K_TILE) : smem_addr(sV + s * C::V_TILE);
-    if (lane == 0) mbar_arrive_expect_tx(full, kv == 0 ? C::K_TILE : C::V_TILE);
+    const uint32_t dst = ring_base + s * tile_bytes;
+    if (lane == 0) mbar_arrive_expect_tx(full, tile_bytes);
     __syncwarp();
-    issued |= 1u << (ring + s);
-    issued_phase = (issued_phase & ~(1u << (ring + s))) | (ph << (ring + s));
     if constexpr (!C::PAGED) {
       if (lane < chunks)
         tma_load_4d_hint(dst + lane * C::CHUNK_BYTES, tm, full, lane * chunk_elems, hkv, u * C::BN, b, pol);
@@ -429,19 +435,14 @@ __device__ void attn_load_role_split(const AttnParams& p, const TileInfo t0, int
                          pol);
     }
   };
-  for (int ua = next_kept_tile<C>(p, misc, 3, t0.u0, n); ua < n && ok;) {
-    const int ub = next_kept_tile<C>(p, misc, 3, ua + 1, n);
-    load(0, ua);
-    if (ok && ub < n) load(0, ub);
-    if (ok) load(1, ua);
-    if (ok && ub < n) load(1, ub);
-    ua = ub < n ? next_kept_tile<C>(p, misc, 3, ub + 1, n) : n;
-  }
-  // Every issued copy lands before shared memory goes away (see attn_load_role).
+  for (int u = next_kept_tile<C>(p, misc, 3, t0.u0, n); u < n && ok; u = next_kept_tile<C>(p, misc, 3, u + 1, n))
+    load(u);
+  // Every issued copy lands before shared memory goes away (see attn_load_role):
+  // the last `stages` tiles issued, one per slot.
   if (lane == 0) {
-    w.drain(q_full, 0);
-    for (int s = 0; s < C::K_STAGES + C::V_STAGES; ++s)
-      if (issued & (1u << s)) w.drain(smem_addr(&misc->kv_full[s]), (issued_phase >> s) & 1u);
+    if (kv_sel == 0) w.drain(q_full, 0);
+    for (int k = pos > stages ? pos - stages : 0; k < pos; ++k)
+      w.drain(smem_addr(&misc->kv_full[ring + k % stages]), (k / stages) & 1u);
   }
   __syncwarp();
 }
@@ -1223,30 +1224,26 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, 
     // Columns [64x, 64x + 64) of both accumulators (a warpgroup without tiles
     // left its O undefined: its values are selected away, never multiplied).
     const uint32_t tO0 = tmem + lane_off + 256u + 64u * x, tO1 = tO0 + C::DV;
-    uint32_t o0[2][32], o1[2][32];
-    tmem_ld32(tO0, o0[0]);
-    tmem_ld32(tO0 + 32, o0[1]);
-    tmem_ld32(tO1, o1[0]);
-    tmem_ld32(tO1 + 32, o1[1]);
-    tmem_wait_ld();
-    reg_fence(o0[0]);
-    reg_fence(o0[1]);
-    reg_fence(o1[0]);
-    reg_fence(o1[1]);
-    auto out_val = [&](int col) {
-      const float a = h0 ? __uint_as_float(o0[col >> 5][col & 31]) * c0 : 0.f;
-      const float b2 = h1 ? __uint_as_float(o1[col >> 5][col & 31]) * c1 : 0.f;
-      float v = (a + b2) * inv;
-      if (C::PV == PV_E4M3 && p.sf_v_kind == FMHA_SF_PER_CHANNEL) v *= misc->sf_v[64 * x + col];
-      return v;
-    };
     const uint32_t buf = stage0 + x * C::CHUNK_BYTES;
     const uint32_t base = buf + r * 128;
-#pragma unroll
-    for (int sc = 0; sc < 2; ++sc) {
+#pragma unroll 1
+    for (int sc = 0; sc < 2; ++sc) {  // 32 columns at a time
+      uint32_t o0[32], o1[32];
+      tmem_ld32(tO0 + 32 * sc, o0);
+      tmem_ld32(tO1 + 32 * sc, o1);
+      tmem_wait_ld();
+      reg_fence(o0);
+      reg_fence(o1);
+      auto out_val = [&](int j) {
+        const float a = h0 ? __uint_as_float(o0[j]) * c0 : 0.f;
+        const float b2 = h1 ? __uint_as_float(o1[j]) * c1 : 0.f;
+        float v = (a + b2) * inv;
+        if (C::PV == PV_E4M3 && p.sf_v_kind == FMHA_SF_PER_CHANNEL) v *= misc->sf_v[64 * x + 32 * sc + j];
+        return v;
+      };
       uint32_t pk[16];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) pk[j] = pack_bf16x2(out_val(32 * sc + 2 * j), out_val(32 * sc + 2 * j + 1));
+      for (int j = 0; j < 16; ++j) pk[j] = pack_bf16x2(out_val(2 * j), out_val(2 * j + 1));
 #pragma unroll
       for (int kk = 0; kk < 4; ++kk) {
         const int k = 4 * sc + kk;
@@ -1643,11 +1640,12 @@ __global__ void __launch_bounds__(C::THREADS, 1)
         attn_mma_role_psmem<C>(p, t[0], t[1], b, hkv, sQ[0], sQ[1], sP[0], sP[1], sSlots, misc, tmem, w);
       else
         attn_mma_role<C>(p, t[0], t[1], b, hkv, sQ[0], sQ[1], sSlots, misc, tmem, w);
+    } else if (C::SPLIT && (warp == C::LOAD_WARP || warp == C::LOAD_WARP + 2)) {
+      // split tiles: warp 1 loads Q and the K ring, warp 3 the V ring
+      attn_load_role_split<C>(p, t[0], b, hkv, warp == C::LOAD_WARP ? 0 : 1, sQ[0], sSlots, sV, misc, &tmQ,
+                              &tmK, &tmV, w);
     } else if (warp == C::LOAD_WARP) {  // the whole warp
-      if constexpr (C::SPLIT)
-        attn_load_role_split<C>(p, t[0], b, hkv, sQ[0], sSlots, sV, misc, &tmQ, &tmK, &tmV, w);
-      else
-        attn_load_role<C>(p, t[0], t[1], b, hkv, sQ[0], sQ[1], sSlots, misc, &tmQ, &tmK, &tmV, w);
+      attn_load_role<C>(p, t[0], t[1], b, hkv, sQ[0], sQ[1], sSlots, misc, &tmQ, &tmK, &tmV, w);
     }
   }
 
