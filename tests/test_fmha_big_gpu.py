@@ -55,7 +55,8 @@ def oracle_head(x_bf16, b, h, spec, full_x=None):
 def check_rows(mode, got_rows, ref_rows, sf_o=None, atol=Q8_ATOL):
     """got/ref: dict (b, h) -> [n, D] arrays. sf_o: the output scale of an E4M3
     output, whose rounding (2^-4 relative, 2^-10 sf_o absolute) adds to the
-    8-bit tolerance, with cos >= 0.998."""
+    8-bit tolerance; the per-head cosine bound stays Q8_COS (measured 1 - cos
+    about 7e-4 for the E4M3-output workload)."""
     for key in ref_rows:
         g, r = got_rows[key], ref_rows[key]
         assert np.all(np.isfinite(g)), f"non-finite output at {key}"
@@ -64,7 +65,7 @@ def check_rows(mode, got_rows, ref_rows, sf_o=None, atol=Q8_ATOL):
             worst = np.argmax(np.abs(g - r) - bound)
             assert np.all(np.abs(g - r) <= bound), f"{key}: err {np.abs(g - r).flat[worst]:.3e}"
             c = cos_per_head(g[None, :, None, :], r[None, :, None, :])[0]
-            assert c >= 0.998, f"{key}: cos {c:.6f}"
+            assert c >= Q8_COS, f"{key}: cos {c:.6f}"
             continue
         err = np.abs(g - r).max()
         if mode == "bf16":
