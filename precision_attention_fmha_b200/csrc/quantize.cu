@@ -162,6 +162,33 @@ __device__ __forceinline__ float block_reduce_max(float v, float* red) {
 // stay in flight through the block reduction and the encoding. Each thread
 // keeps up to kCache 16-byte vectors of an item in registers (HBM read once);
 // vectors past kThr * kCache (blocks larger than the cache) are re-read.
+// Position (b, token block, h) of a work item, in that order (h fastest), and
+// its advance by a fixed stride without a division per item: the stride is
+// decomposed once (dh heads, then dblk blocks and db batches with carries).
+struct ItemCursor {
+  int b, blk, h;
+  int dh, dblk, db;
+  __device__ ItemCursor(int64_t item, int64_t stride, int H, int nblk) {
+    h = static_cast<int>(item % H);
+    const int64_t bb = item / H;
+    blk = static_cast<int>(bb % nblk);
+    b = static_cast<int>(bb / nblk);
+    dh = static_cast<int>(stride % H);
+    const int64_t sb = stride / H;
+    dblk = static_cast<int>(sb % nblk);
+    db = static_cast<int>(sb / nblk);
+  }
+  __device__ __forceinline__ void advance(int H, int nblk) {
+    h += dh;
+    int carry = h >= H;
+    h -= carry ? H : 0;
+    blk += dblk + carry;
+    carry = blk >= nblk;
+    blk -= carry ? nblk : 0;
+    b += db + carry;
+  }
+};
+
 // CTAs per SM the register budget is set for: 64 registers a thread without a
 // shift; the shifted values need a few more (3 CTAs of 256, 1 of 512).
 constexpr int token_block_min_ctas(int threads, bool shift) {
@@ -176,15 +203,8 @@ __global__ void __launch_bounds__(kThr, token_block_min_ctas(kThr, kShift))
   auto shift_of = [&](int64_t bh, int c) -> const float* { return kShift ? shift_at(p, bh, c) : nullptr; };
   __shared__ float red[2][kThr / 32];  // alternating buffers: no barrier between items
   const int vpr = p.D >> 3;
-  auto locate = [&](int64_t item, int& b, int& h, int& blk) {
-    h = static_cast<int>(item % p.H);
-    const int64_t bb = item / p.H;
-    blk = static_cast<int>(bb % p.nblk);
-    b = static_cast<int>(bb / p.nblk);
-  };
-  auto load = [&](int64_t item, uint4 (&c)[kCache]) {
-    int b, h, blk;
-    locate(item, b, h, blk);
+  auto load = [&](const ItemCursor& ic, uint4 (&c)[kCache]) {
+    const int b = ic.b, h = ic.h, blk = ic.blk;
     const int s0 = blk * p.rpb;
     const int nvec = min(p.S - s0, p.rpb) * vpr;
     const uint16_t* src = p.src + b * p.s_sb + static_cast<int64_t>(s0) * p.s_ss + h * p.s_sh;
@@ -199,12 +219,13 @@ __global__ void __launch_bounds__(kThr, token_block_min_ctas(kThr, kShift))
   };
   uint4 cur[kCache], nxt[kCache];
   int64_t item = blockIdx.x;
-  if (item < n_items) load(item, cur);
+  ItemCursor ic(item, gridDim.x, p.H, p.nblk);
+  if (item < n_items) load(ic, cur);
   for (int it = 0; item < n_items; ++it) {
     const int64_t next = item + gridDim.x;
-    if (next < n_items) load(next, nxt);  // in flight while this item is reduced and encoded
-    int b, h, blk;
-    locate(item, b, h, blk);
+    const int b = ic.b, h = ic.h, blk = ic.blk;
+    ic.advance(p.H, p.nblk);
+    if (next < n_items) load(ic, nxt);  // in flight while this item is reduced and encoded
     const int s0 = blk * p.rpb;
     const int nvec = min(p.S - s0, p.rpb) * vpr;
     const uint16_t* src = p.src + b * p.s_sb + static_cast<int64_t>(s0) * p.s_ss + h * p.s_sh;
@@ -338,18 +359,10 @@ __global__ void __launch_bounds__(kThr) quant_token_block_tma_kernel(const __gri
   const int rstep = kThr >> lg;            // rows per pass
   const uint32_t box_bytes = static_cast<uint32_t>(p.rpb) * p.D * 2;  // zero-filled rows count too
   const uint32_t slots = smem_addr(qsm);
-  auto locate = [&](int64_t item, int& b, int& h, int& blk) {
-    h = static_cast<int>(item % p.H);
-    const int64_t bb = item / p.H;
-    blk = static_cast<int>(bb % p.nblk);
-    b = static_cast<int>(bb / p.nblk);
-  };
-  auto issue = [&](int slot, int64_t item) {  // thread 0
-    int b, h, blk;
-    locate(item, b, h, blk);
+  auto issue = [&](int slot, const ItemCursor& ic) {  // thread 0
     const uint32_t bar = smem_addr(&full[slot]);
     mbar_arrive_expect_tx(bar, box_bytes);
-    tma_load_4d(slots + slot * slot_bytes, &tm, bar, 0, h, blk * p.rpb, b);
+    tma_load_4d(slots + slot * slot_bytes, &tm, bar, 0, ic.h, ic.blk * p.rpb, ic.b);
   };
   // Bounded wait for a slot's copy; a timeout is recorded in the error word.
   auto wait_full = [&](int slot, uint32_t parity) {
@@ -371,16 +384,20 @@ __global__ void __launch_bounds__(kThr) quant_token_block_tma_kernel(const __gri
   }
   __syncthreads();
   int issued = 0;  // thread 0: items whose copies were started
+  ItemCursor ahead(blockIdx.x, gridDim.x, p.H, p.nblk);  // thread 0: the next item to copy
   if (threadIdx.x == 0)
-    for (int k = 0; k < stages && blockIdx.x + static_cast<int64_t>(k) * gridDim.x < n_items; ++k, ++issued)
-      issue(k, blockIdx.x + static_cast<int64_t>(k) * gridDim.x);
+    for (int k = 0; k < stages && blockIdx.x + static_cast<int64_t>(k) * gridDim.x < n_items; ++k, ++issued) {
+      issue(k, ahead);
+      ahead.advance(p.H, p.nblk);
+    }
 
   int it = 0;
+  ItemCursor ic(blockIdx.x, gridDim.x, p.H, p.nblk);
   for (int64_t item = blockIdx.x; item < n_items; item += gridDim.x, ++it) {
     const int slot = it % stages;
     if (!__syncthreads_and(wait_full(slot, (it / stages) & 1))) break;
-    int b, h, blk;
-    locate(item, b, h, blk);
+    const int b = ic.b, h = ic.h, blk = ic.blk;
+    ic.advance(p.H, p.nblk);
     const int s0 = blk * p.rpb;
     const int rows = min(p.S - s0, p.rpb);
     const uint8_t* tile = qsm + slot * slot_bytes + c * 16;
@@ -420,7 +437,8 @@ __global__ void __launch_bounds__(kThr) quant_token_block_tma_kernel(const __gri
     amax = block_reduce_max<kThr>(amax, red[it & 1]);  // every thread has read the slot
     if (threadIdx.x == 0 && item + static_cast<int64_t>(stages) * gridDim.x < n_items) {
       fence_proxy_async_smem();  // generic reads of the slot before the copy that rewrites it
-      issue(slot, item + static_cast<int64_t>(stages) * gridDim.x);
+      issue(slot, ahead);
+      ahead.advance(p.H, p.nblk);
       ++issued;
     }
     const Divisor dv(scale_from_amax<kE4M3>(amax));
