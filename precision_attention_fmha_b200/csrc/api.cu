@@ -424,6 +424,8 @@ fmha_status run_attention(const fmha_args* a, const uint8_t* mask, int64_t msb, 
     p.packed = 1;
     p.group_shift = group_shift;
     p.n_rows = Sq * group;
+    // At most 16 packed rows (all in one tile) with BF16 P: the 16-lane softmax pass.
+    p.narrow = (pv == PV_BF16 && sp.interleave && p.n_rows <= 16) ? 1 : 0;
     p.n_units = sp.n_units;
     p.n_splits = sp.n_splits;
     p.split_tiles = sp.split_tiles;

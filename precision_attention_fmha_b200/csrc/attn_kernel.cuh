@@ -902,6 +902,132 @@ __device__ __forceinline__ void exp2_poly_x2(float& a, float& b) {
   b = __int_as_float(__float_as_int(pb) + (__float_as_int(jb) << 23));
 }
 
+// ------------------------------------------------------- narrow softmax ----
+// Decode tiles whose packed rows are all in rows 0..15 (Sq * group <= 16, BF16
+// P in TMEM): only the first warp of the warpgroup (TMEM lanes 0..31) holds
+// valid rows. It loads S with the 16-lane shape, which spreads rows 0..7 and
+// 8..15 over all 32 threads (thread t: rows t/4 and 8 + t/4, key pairs
+// 8k + 2(t%4), k = 0..15), so each thread exponentiates 32 (or 64) scores
+// instead of a row of 128 of which only 8 or 16 rows are real. The row max
+// and sum are reduced over the four threads of a row; P goes back over S with
+// the 16-lane x 128-bit shape, whose column 4k + t%4 is exactly the pair of
+// keys thread t holds. The other three warps only keep the barrier count.
+// Returns, for the epilogue, m and l of row `lane` (lanes 0..15), and the
+// number of tiles processed.
+template <class C>
+__device__ void attn_softmax_narrow(const AttnParams& p, const TileInfo t, int x, AttnMisc* misc, uint32_t tmem,
+                                    float cq, const Waiter w, float& m_out, float& l_out, int& it_out, bool& ok_out) {
+  using namespace ptx;
+  constexpr uint32_t FULL = 0xffffffffu;
+  const int warp = (threadIdx.x >> 5) & 3;
+  const int lane = threadIdx.x & 31;
+  const int j = lane & 3, rr = lane >> 2;
+  const uint32_t tS = tmem + (x ? 128u : 0u);                 // lane quadrant 0
+  const uint32_t tO = tmem + (x ? 256u + C::DV : 256u);
+  const int nh = p.n_rows > 8 ? 2 : 1;                         // row halves with valid rows
+  constexpr float tau = 8.f;                                   // BF16 P
+  float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
+  int it = 0;
+  bool ok = true;
+  for (int u = next_kept_tile<C>(p, misc, 1 << t.x, t.u0, t.n_kv); u < t.n_kv;
+       u = next_kept_tile<C>(p, misc, 1 << t.x, u + 1, t.n_kv)) {
+    ok = __all_sync(FULL, w.wait(smem_addr(&misc->s_full[x]), it & 1)) && ok;
+    if (!ok) break;
+    tc_fence_after();
+    if (warp == 0) {
+      uint32_t sr[64];
+      tmem_ld_16x256b_x16(tS, sr);
+      tmem_wait_ld();
+#pragma unroll
+      for (int q = 0; q < 64; q += 32) {
+        uint32_t (&blk)[32] = *reinterpret_cast<uint32_t (*)[32]>(&sr[q]);
+        reg_fence(blk);
+      }
+      float alpha[2] = {1.f, 1.f};
+      bool resc = false;
+      uint32_t pk[32];  // P columns 4k + j of row rr (2k) and 8 + rr (2k + 1)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        // keys at or past lim are hidden for this row (ragged end, causal)
+        const int row = rr + 8 * h;
+        const int tok = t.tok0 + (row >> p.group_shift);
+        int lim = p.Skv - u * C::BN;
+        if (p.causal) lim = min(lim, tok + 1 + (p.Skv - p.Sq) - u * C::BN);
+        if (h >= nh || tok >= p.Sq) lim = 0;  // a padding row: all hidden
+        float f[32];
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          f[2 * k] = 8 * k + 2 * j < lim ? __uint_as_float(sr[4 * k + 2 * h]) : -INFINITY;
+          f[2 * k + 1] = 8 * k + 2 * j + 1 < lim ? __uint_as_float(sr[4 * k + 2 * h + 1]) : -INFINITY;
+        }
+        float mt = f[0];
+#pragma unroll
+        for (int i = 1; i < 32; ++i) mt = fmaxf(mt, f[i]);
+        mt = fmaxf(mt, __shfl_xor_sync(FULL, mt, 1));
+        mt = fmaxf(mt, __shfl_xor_sync(FULL, mt, 2));
+        mt *= cq;
+        const float m_new = fmaxf(m[h], mt);
+        if (it == 0) {
+          m[h] = m_new;
+        } else if (m_new > m[h] + tau) {
+          alpha[h] = ex2(m[h] - m_new);
+          resc = true;
+          m[h] = m_new;
+        }
+        const float nmb = -(m[h] == -INFINITY ? 0.f : m[h]);
+        float rs = 0.f;
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          float e0, e1;
+          ffma2(e0, e1, f[2 * k], f[2 * k + 1], cq, cq, nmb, nmb);
+          e0 = ex2(e0);
+          e1 = ex2(e1);
+          pk[2 * k + h] = pack_bf16x2(e0, e1);
+          rs += e0 + e1;
+        }
+        l[h] = l[h] * alpha[h] + rs;
+      }
+      // Lazy O correction (rows rr and 8 + rr of this thread), before P is
+      // released: the arrival of S proved the previous PV finished.
+      if (__any_sync(FULL, resc)) {
+        uint32_t o[64];
+        tmem_ld_16x256b_x16(tO, o);
+        tmem_wait_ld();
+#pragma unroll
+        for (int q = 0; q < 64; q += 32) {
+          uint32_t (&blk)[32] = *reinterpret_cast<uint32_t (*)[32]>(&o[q]);
+          reg_fence(blk);
+        }
+#pragma unroll
+        for (int k = 0; k < 16; ++k)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) o[4 * k + e] = __float_as_uint(__uint_as_float(o[4 * k + e]) * alpha[e >> 1]);
+        tmem_st_16x256b_x16(tO, o);
+      }
+      tmem_st_16x128b_x16(tS, pk);
+      tmem_wait_st();
+    }
+    tc_fence_before();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(smem_addr(&misc->p_full[x]));
+    ++it;
+  }
+  // Row totals (four threads per row), then row `lane` for the epilogue.
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    l[h] += __shfl_xor_sync(FULL, l[h], 1);
+    l[h] += __shfl_xor_sync(FULL, l[h], 2);
+  }
+  const int src = 4 * (lane & 7);
+  const float m0 = __shfl_sync(FULL, m[0], src), m1 = __shfl_sync(FULL, m[1], src);
+  const float l0 = __shfl_sync(FULL, l[0], src), l1 = __shfl_sync(FULL, l[1], src);
+  const bool mine = warp == 0 && lane < 8 * nh;
+  m_out = mine ? (lane < 8 ? m0 : m1) : -INFINITY;
+  l_out = mine ? (lane < 8 ? l0 : l1) : 0.f;
+  it_out = it;
+  ok_out = ok;
+}
+
 // --------------------------------------------------------------- softmax ----
 // One thread per query row (TMEM lane = row). Per kept KV tile: load S (128
 // fp32 or s32 per row) from TMEM, scale and mask, exponentiate with packed
@@ -966,7 +1092,14 @@ __device__ void attn_softmax_role(const AttnParams& p, const TileInfo t, int x, 
   float l = 0.f;        // running row sum of P (times g)
   int it = 0;
   bool ok = true;
-  for (int u = next_kept_tile<C>(p, misc, 1 << t.x, t.u0, t.n_kv); u < t.n_kv;
+  bool narrow = false;  // decode tiles of at most 16 rows: the narrow pass above
+  if constexpr (C::PACKED && C::PV == PV_BF16) {
+    if (p.narrow) {
+      attn_softmax_narrow<C>(p, t, x, misc, tmem, cq * ck_uniform, w, m, l, it, ok);
+      narrow = true;
+    }
+  }
+  for (int u = narrow ? t.n_kv : next_kept_tile<C>(p, misc, 1 << t.x, t.u0, t.n_kv); u < t.n_kv;
        u = next_kept_tile<C>(p, misc, 1 << t.x, u + 1, t.n_kv)) {
     float ck[NCH];
     load_ck(u, ck);  // issued before the wait: the loads overlap it

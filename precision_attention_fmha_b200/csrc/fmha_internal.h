@@ -61,6 +61,7 @@ struct AttnParams {
   // token r >> group_shift of head (hkv * group + (r & (group - 1))); n_units
   // then counts pairs of 128-row units of the Sq * group packed rows.
   int32_t packed, group_shift, n_rows;
+  int32_t narrow;  // packed, BF16 P, n_rows <= 16 in one tile: the 16-lane softmax pass
   // Split-KV (packed only): split j of a (b, kv head) takes the kept KV tiles
   // of ranks [j * per, (j + 1) * per), per = ceil(kept / n_splits). With several
   // partials each query tile writes O / l (fp32) and its lse to o_part / lse_part.
