@@ -579,8 +579,14 @@ def cpu_cores():
         return os.cpu_count()
 
 
-def cpu_baseline(W, rows=1024):
+def cpu_baseline(W, rows=1024, target_s=10.0):
+    """The oracle on a bounded sample, sized to about target_s seconds of CPU work:
+    a 1024-row probe, then as many query rows (up to Sq) as the probe says fit."""
     dt, fl = oracle_sample(W.host, W.kind, W.B, W.Hq, W.Hkv, W.S, W.D, W.causal, rows)
+    grow = min(W.host["q"].shape[1], int(rows * target_s / max(dt, 1e-3)) // 128 * 128)
+    if grow > rows:
+        rows = grow
+        dt, fl = oracle_sample(W.host, W.kind, W.B, W.Hq, W.Hkv, W.S, W.D, W.causal, rows)
     return {"value": round(fl / dt / 1e12, 6), "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
             "sample": f"query head 0, rows 0..{rows - 1} against all keys (with the workload's quantization of "
                       f"that head), float64 NumPy, {dt:.1f} s"}
