@@ -5,6 +5,13 @@
 //   sb   = E4M3((amax_blk / s_t) / 6)           (IEEE divisions, RN, satfinite)
 //   e    = decode(sb) * s_t
 //   code = E2M1(x / e), or E2M1(x * (1 / e)) on the fast path; 0 when e == 0
+// The exact path takes x / e as Markstein's FMA-corrected quotient (P.
+// Markstein, IBM J. Res. Dev. 34(1), 1990) from one correctly rounded
+// reciprocal per block: q0 = RN(x r), q = RN(q0 + (x - q0 e) r), with the
+// sign of x (so -0 keeps its code). It is the correctly rounded quotient, so
+// the codes equal the IEEE division's, while e >= 2^-60 keeps every quotient
+// that can reach a nonzero code (|q| >= 2^-2) and its residual in the normal
+// range; blocks with a smaller e divide.
 // One CTA per row. Each thread keeps its 16-element blocks in registers from
 // the amax pass to the quantize pass (the row is read from HBM once, as the
 // page's kernel caches its input on chip), so HBM sees 2 B read and
@@ -95,6 +102,17 @@ __global__ void __launch_bounds__(kThreads) nvfp4_quant_kernel(const Nvfp4Params
         const float r = __fdiv_rn(1.f, e);
 #pragma unroll
         for (int k = 0; k < 16; ++k) y[k] = __fmul_rn(x[k], r);
+      } else if (e >= 0x1p-60f) {
+        const float r = __frcp_rn(e);
+#pragma unroll
+        for (int k = 0; k < 16; k += 2) {
+          float q0a, q0b, ea, eb, qa, qb;
+          ptx::ffma2(q0a, q0b, x[k], x[k + 1], r, r, -0.f, -0.f);       // RN(x r)
+          ptx::ffma2(ea, eb, -q0a, -q0b, e, e, x[k], x[k + 1]);         // x - q0 e, one rounding
+          ptx::ffma2(qa, qb, ea, eb, r, r, q0a, q0b);                   // RN(q0 + res r)
+          y[k] = copysignf(qa, x[k]);
+          y[k + 1] = copysignf(qb, x[k + 1]);
+        }
       } else {
 #pragma unroll
         for (int k = 0; k < 16; ++k) y[k] = __fdiv_rn(x[k], e);

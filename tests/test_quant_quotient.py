@@ -164,3 +164,38 @@ def test_negative_zero_keeps_its_sign():
     q = kernel_quotient(np.array([-0.0, 0.0], dtype=np.float32), np.float32(0.01))
     assert np.signbit(q[0]) and not np.signbit(q[1])
     assert list(codes_of(q, "e4m3")) == [0x80, 0x00]
+
+
+def test_nvfp4_block_quotients_match_division():
+    """The exact NVFP4 path divides each 16-element block by e = decode(sb) * s_t
+    with the same corrected quotient: its E2M1 codes equal those of RN(x / e)
+    (oracle/nvfp4.py), on N(0,1) rows with outliers, values placed on and next
+    to every E2M1 rounding boundary, and rows small enough that e falls below
+    the guard."""
+    from oracle import e4m3
+    from oracle import nvfp4 as on
+
+    rng = np.random.default_rng(4242)
+    rows = [rng.standard_normal(4096).astype(np.float32) * np.where(rng.random(4096) < 0.01, 40.0, 1.0)]
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0], dtype=np.float64)
+    bound = np.concatenate([mids, np.nextafter(mids, 0), np.nextafter(mids, 10)])
+    for scale in (1.0, 3.0e-3, 7.0e5, 2.0 ** -70):
+        r = np.resize(np.concatenate([bound, -bound, [6.0, -6.0, 0.0, -0.0]]), 4096) * scale
+        rows.append(r.astype(np.float32))
+    x = np.stack(rows).astype(np.float32)
+    x = x.view(np.uint32) & np.uint32(0xFFFF0000)  # exact BF16 values
+    x = x.view(np.float32)
+    _, sb_codes, st = on.quantize_per_token(x)
+    checked = below = 0
+    for i in range(x.shape[0]):
+        for j in range(x.shape[1] // 16):
+            e = np.float32(np.float32(e4m3.decode(np.array([sb_codes[i, j]]))[0]) * st[i])
+            if e == 0:
+                continue
+            blk = x[i, 16 * j:16 * (j + 1)]
+            got = on.e2m1_encode(kernel_quotient(blk, e))
+            want = on.e2m1_encode((blk / e).astype(np.float32))
+            assert np.array_equal(got, want), (i, j, e)
+            checked += blk.size
+            below += int(e < GUARD)
+    assert checked > 20000 and below > 0
