@@ -28,6 +28,9 @@ namespace {
 // saw no key carry lse_j = -inf and weigh nothing; if every split is empty the
 // row is O = 0, lse = -inf.
 __global__ void __launch_bounds__(128) split_merge_kernel(const MergeParams m) {
+  // Launched as a programmatic dependent of the attention grid: wait here until
+  // that grid has finished and its partials are visible.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int lane = threadIdx.x & 31;
   const long long rowid = static_cast<long long>(blockIdx.x) * 4 + (threadIdx.x >> 5);
   const long long rows = static_cast<long long>(m.B) * m.Sq * m.Hq;
@@ -87,8 +90,19 @@ cudaError_t launch_split_merge(const MergeParams& m, cudaStream_t s) {
   const long long rows = static_cast<long long>(m.B) * m.Sq * m.Hq;
   const long long blocks = (rows + 3) / 4;
   if (blocks <= 0) return cudaSuccess;
-  split_merge_kernel<<<static_cast<unsigned>(blocks), 128, 0, s>>>(m);
-  return cudaGetLastError();
+  // Programmatic dependent launch: the merge grid is set up while the attention
+  // grid (which allows it at its start) still runs, instead of after it.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(blocks));
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, split_merge_kernel, m);
 }
 
 }  // namespace fmha

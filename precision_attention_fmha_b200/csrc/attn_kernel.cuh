@@ -1514,6 +1514,9 @@ __global__ void __launch_bounds__(C::THREADS, 1)
                     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmV,
                     const __grid_constant__ CUtensorMap tmO) {
   using namespace ptx;
+  // Decode: the split merge that follows may be launched now (it waits for
+  // this grid's completion itself); every CTA of this grid is resident by then.
+  if constexpr (C::PACKED) asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   // Q buffers, then E4M3 P buffers (shared-memory P), then the K/V ring. With one
