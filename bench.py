@@ -310,8 +310,6 @@ def roofline(W, args, attn_ms, achieved_tflops):
     r = {"bound": "tensor", "achieved": round(achieved_tflops, 2), "peak": round(W.peak, 1), "unit": "TFLOP/s",
          "frac": round(achieved_tflops / W.peak, 4), "traffic": TRAFFIC.get(args.workload),
          "peak_note": f"{W.peak_src}: {W.peak_note}", "kernel": "attn_fwd_kernel", "kernel_ms": round(attn_ms, 4)}
-    if args.workload == "dense_pv8_s32768":
-        r["traffic_note"] = "ncu DRAM bytes of the S = 16384 launch times two (all tensors scale with S)"
     return r
 
 
@@ -504,11 +502,18 @@ def run_ours(args):
 # The default S = 32768 launch is the S = 16384 capture times two (every tensor the
 # launch moves doubles with S); profiles/attn_fwd_pv8_dram_traffic.md has the numbers.
 TRAFFIC = {
-    "dense_pv8_s32768": 2 * (421.13e6 + 151.15e6),  # scaled from the S = 16384 capture
-    "dense_pv8_s16384": 421.13e6 + 151.15e6,
-    "all_fp8_s8192": 201.48e6 + 106.56e6,
-    "sage_s16384": 151.20e6 + 71.45e6,
-    "sparse_paged_s16384": 1344.55e6 + 1042.80e6,
+    # ncu dram__bytes_read.sum + dram__bytes_write.sum of one attention launch (the first
+    # timed one) of the current kernels, one-pass metrics on the full-size workload
+    "dense_pv8_s32768": 847.64e6 + 315.26e6,
+    "dense_pv8_s16384": 420.51e6 + 144.98e6,
+    "dense_bf16_s16384": 504.63e6 + 148.48e6,
+    "all_fp8_s8192": 201.43e6 + 103.67e6,
+    "sage_s16384": 151.21e6 + 71.01e6,
+    "sparse_paged_s16384": 1343.59e6 + 1041.93e6,
+    "wide_qk_bf16_s16384": 673.46e6 + 160.15e6,
+    "wide_qk_pv8_s16384": 587.59e6 + 153.48e6,
+    "wide_qk_fp8_s16384": 336.24e6 + 143.42e6,
+    "decode_paged_s16384": 69.26e6 + 1.02e6,  # the attention launch (the merge adds about 1 MB)
 }
 
 

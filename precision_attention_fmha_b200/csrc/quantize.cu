@@ -284,17 +284,18 @@ __global__ void __launch_bounds__(kThr, token_block_min_ctas(kThr, kShift))
 // The per-element work is cut to a few instructions so that the kernel stays
 // bound by HBM: D / 8 is a power of two, so a thread's column vector is fixed
 // and its rows are a shift away (no integer division); without a shift the
-// amax is taken on the BF16 bit patterns (|x| ordered as unsigned 16-bit
-// integers, two per instruction); the quotient's three operations run on
-// packed fp32 pairs; an INT8 code is rint(q) read from the low byte of
+// amax is taken on the BF16 pairs themselves (max of magnitudes, two per
+// instruction); the quotient's three operations run on packed fp32 pairs; an
+// INT8 code is rint(q) read from the low byte of
 // q + 1.5 * 2^23 (exact for |q| < 2^22; |q| <= 127 here), bytes gathered with
 // byte permutes; an E4M3 code takes the sign bit of x (so -0 keeps 0x80).
 constexpr int kMaxStages = 4;
 constexpr uint32_t kQuantWaitSleepNs = 500;
 
-__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
+// max(|a|, |b|) of BF16 pairs; the sign bits hold garbage (masked at the end).
+__device__ __forceinline__ uint32_t max_abs_bf16x2(uint32_t a, uint32_t b) {
   uint32_t d;
-  asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
   return d;
 }
 
@@ -417,7 +418,7 @@ __global__ void __launch_bounds__(kThr) quant_token_block_tma_kernel(const __gri
     };
     uint4 cache[kCache];
     float amax = 0.f;
-    uint32_t am2 = 0u;  // no shift: max of |x| as BF16 bit patterns, two per word
+    uint32_t am2 = 0u;  // no shift: max of |x| over BF16 pairs (magnitudes in bits 0-14, 16-30)
 #pragma unroll
     for (int i = 0; i < kCache; ++i) {
       const int r = r0 + i * rstep;
@@ -428,12 +429,12 @@ __global__ void __launch_bounds__(kThr) quant_token_block_tma_kernel(const __gri
           values(cache[i], x);
           amax = fmaxf(amax, amax8(x));
         } else {
-          am2 = max_u16x2(am2, max_u16x2(max_u16x2(cache[i].x & 0x7FFF7FFFu, cache[i].y & 0x7FFF7FFFu),
-                                         max_u16x2(cache[i].z & 0x7FFF7FFFu, cache[i].w & 0x7FFF7FFFu)));
+          am2 = max_abs_bf16x2(am2, max_abs_bf16x2(max_abs_bf16x2(cache[i].x, cache[i].y),
+                                                   max_abs_bf16x2(cache[i].z, cache[i].w)));
         }
       }
     }
-    if constexpr (!kShift) amax = __uint_as_float(max(am2 & 0xFFFFu, am2 >> 16) << 16);
+    if constexpr (!kShift) amax = __uint_as_float(max(am2 & 0x7FFFu, (am2 >> 16) & 0x7FFFu) << 16);
     amax = block_reduce_max<kThr>(amax, red[it & 1]);  // every thread has read the slot
     if (threadIdx.x == 0 && item + static_cast<int64_t>(stages) * gridDim.x < n_items) {
       fence_proxy_async_smem();  // generic reads of the slot before the copy that rewrites it
