@@ -126,7 +126,9 @@ typedef struct {
  * (E4M3, E4M3, E4M3, BF16) ("all-FP8", [BW-FP8]), (INT8, INT8, E4M3, BF16)
  * ("SageAttention", [DiT-Sage]). D must be 64 or 128 (128 for 8-bit Q/K),
  * or D = 192 with Dv = 128 for the BF16, QK-BF16/PV-FP8 and all-FP8 tuples
- * with one-term P and a BF16 o, not through fmha_fwd_decode: the QK head dim
+ * with one-term P and a BF16 o, not through fmha_fwd_decode (with BF16 Q/K
+ * also Skv <= 131072: a CTA deals its kept key blocks to two warpgroups
+ * through a 1024-bit set; FMHA_ERR_UNSUPPORTED otherwise): the QK head dim
  * that [BW-FP8]'s reviewer notes name as the case their shared-memory-P
  * schedule was gated off for (shared-memory capacity).
  * Any of these may instead write an E4M3 o (D = 128, not fmha_fwd_decode):

@@ -123,6 +123,16 @@ def test_wide_qk_head_dim_rules(lib, mutate):
     assert lib.fmha_last_error_message().decode()
 
 
+def test_wide_qk_bf16_key_limit(lib):
+    """D = 192 with BF16 Q/K deals key blocks through a 1024-bit set: Skv <= 131072."""
+    a = _wide_args()
+    a.Skv = 131072 + 1
+    for t in (a.k, a.v):
+        t.stride_b = (131072 + 1) * t.stride_s
+    assert lib.fmha_fwd(ctypes.byref(a), None) == 2
+    assert "131072" in lib.fmha_last_error_message().decode()
+
+
 def test_paged_argument_checks(lib):
     a = _args()
     assert lib.fmha_fwd_paged(ctypes.byref(a), 0x30000, 8, 48, 4, None, 0, 0, None) == 2  # page size
