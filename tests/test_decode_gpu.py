@@ -70,6 +70,10 @@ def decode_case(mode, B, Hq, Hkv, Sq, Skv, splits, causal, paged, masked, seed):
     ("bf16", 1, 4, 4, 33, 900, 2, False, False, True),     # G = 1 (MHA)
     ("bf16", 1, 128, 1, 2, 600, 2, False, False, False),   # G = 128: one token per unit
     ("bf16", 1, 8, 1, 1, 300, 8, False, False, False),     # more splits asked than KV tiles
+    # at most 16 packed rows: the 16-lane softmax pass, both row halves
+    ("bf16", 2, 32, 2, 1, 1500, 0, False, True, True),     # G = 16, one token: rows 0-15
+    ("bf16", 1, 8, 1, 2, 1000, 2, True, False, False),     # G = 8, two tokens, causal
+    ("bf16", 1, 4, 1, 3, 700, 0, True, False, True),      # G = 4, three tokens: rows 0-11
     ("pv8", 2, 16, 2, 4, 2000, 0, True, True, False),
     ("fp8", 2, 16, 2, 1, 3000, 5, False, True, True),
     ("fp8", 1, 8, 2, 9, 1200, 3, True, False, False),
