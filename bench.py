@@ -383,7 +383,7 @@ def run_nvfp4(args):
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         from oracle import nvfp4 as on
-        n = 64
+        n = 512  # about 10 s of the per-row oracle
         tt = time.perf_counter()
         on.quantize_per_token(xh[:n].to(torch.float32).numpy())
         dt = time.perf_counter() - tt
@@ -584,9 +584,10 @@ def cpu_cores():
         return os.cpu_count()
 
 
-def cpu_baseline(W, rows=1024, target_s=10.0):
-    """The oracle on a bounded sample, sized to about target_s seconds of CPU work:
-    a 1024-row probe, then as many query rows (up to Sq) as the probe says fit."""
+def cpu_baseline(W, rows=1024, target_s=20.0):
+    """The oracle on a bounded sample: a 1024-row probe, then as many query rows (up
+    to Sq) as the probe says fit in target_s seconds (larger samples run faster per
+    row, so the second run takes about half of it: 10 s or so)."""
     dt, fl = oracle_sample(W.host, W.kind, W.B, W.Hq, W.Hkv, W.S, W.D, W.causal, rows)
     grow = min(W.host["q"].shape[1], int(rows * target_s / max(dt, 1e-3)) // 128 * 128)
     if grow > rows:
@@ -733,9 +734,9 @@ def run_smooth(args):
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        dt, nbytes = smooth_oracle_sample(kh, heads=2, smooth=smooth)
+        dt, nbytes = smooth_oracle_sample(kh, heads=H, smooth=smooth)  # the whole K: well under a second
         line["cpu_baseline"] = {"value": round(nbytes / dt / 1e9, 6), "unit": "GB/s", "cores": cpu_cores(),
-                                "kind": "oracle", "sample": f"heads 0..1 of {H}, NumPy oracle, {dt:.2f} s"}
+                                "kind": "oracle", "sample": f"all {H} heads, NumPy oracle, {dt:.2f} s"}
     if rank == 0:
         print(json.dumps(line), flush=True)
     teardown(world)
