@@ -453,19 +453,49 @@ def run_ours(args):
     attn_ms = max_over_ranks(attn_ms, world)
 
     # ---- end-to-end: host (pinned) inputs, H2D + path + D2H of O each step ----
-    o_h = torch.empty(W.o.shape, dtype=W.o.dtype, pin_memory=True)
+    # Pipelined as a serving loop would run it: step i + 1's inputs are copied
+    # host -> device on one stream while step i computes on the current stream,
+    # and step i's O goes back on a third (two device buffers of each). Every
+    # step's inputs and its O still cross the host link inside the timed region.
     Ke = max(1, min(K, 10))
+    h2d, d2h = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    bufs = [{n: torch.empty(t.shape, dtype=t.dtype, device=dev) for n, t in W.host.items()} for _ in range(2)]
+    outs = [W.o, torch.empty_like(W.o)]
+    o_h = [torch.empty(W.o.shape, dtype=W.o.dtype, pin_memory=True) for _ in range(2)]
+    ev_in = [torch.cuda.Event() for _ in range(Ke)]
+    ev_comp = [torch.cuda.Event() for _ in range(Ke)]
+    ev_out = [torch.cuda.Event() for _ in range(Ke)]
+
+    def copy_in(i):
+        with torch.cuda.stream(h2d):
+            if i >= 2:  # compute of step i - 2 has read this buffer
+                h2d.wait_event(ev_comp[i - 2])
+            for n, t in W.host.items():
+                bufs[i % 2][n].copy_(t, non_blocking=True)
+            ev_in[i].record(h2d)
+
     barrier(world)
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(Ke):
-        inp = {n: t.to(dev, non_blocking=True) for n, t in W.host.items()}
-        W.prep(inp)
-        W.attn(inp)
-        o_h.copy_(W.o, non_blocking=True)
-    e1.record(stream)
+    e0.record(h2d)
+    copy_in(0)
+    for i in range(Ke):
+        if i + 1 < Ke:
+            copy_in(i + 1)
+        stream.wait_event(ev_in[i])
+        if i >= 2:  # the copy back of step i - 2 has read this O buffer
+            stream.wait_event(ev_out[i - 2])
+        W.o = outs[i % 2]
+        W.prep(bufs[i % 2])
+        W.attn(bufs[i % 2])
+        ev_comp[i].record(stream)
+        with torch.cuda.stream(d2h):
+            d2h.wait_event(ev_comp[i])
+            o_h[i % 2].copy_(outs[i % 2], non_blocking=True)
+            ev_out[i].record(d2h)
+    e1.record(d2h)  # after the last copy back, which waits for all the rest
     torch.cuda.synchronize()
+    W.o = outs[0]
     barrier(world)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / Ke, world)
     fmha.get_device_error()
@@ -484,6 +514,7 @@ def run_ours(args):
         "roofline": roofline(W, args, attn_ms, achieved),
         "e2e": {"value": round(world * W.flop / (e2e_ms * 1e-3) / 1e12, 2), "unit": UNIT,
                 "h2d_bytes_per_step": bytes_in, "d2h_bytes_per_step": W.o.numel() * W.o.element_size(),
+                "pipelined": "step i+1's H2D and step i's D2H run on their own streams, overlapping step i",
                 "steps": Ke},
         "gpu_launches": K * W.launches,
         "clocks": clk,
