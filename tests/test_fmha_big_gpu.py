@@ -161,14 +161,30 @@ def test_sage_full_size(p_terms):
     run_case("sage", w["q"], w["k"], w["v"], spec, heads=[(0, 0), (0, 11), (0, 23)], sf_p=sf_p, p_terms=p_terms)
 
 
+@pytest.mark.parametrize("mode", ["bf16", "pv8", "fp8"])
+def test_wide_qk_full_size(mode):
+    """D_qk = 192 / D_v = 128, B1 H40 S16384, quantized as bench.py's wide_qk workloads."""
+    w = workloads.wide_qk(outliers=mode == "fp8")
+    spec = {"bf16": {}, "pv8": {"v": ("e4m3", "per_tensor", None)},
+            "fp8": {n: ("e4m3", "per_head", None) for n in "qkv"}}[mode]
+    run_case(mode, w["q"], w["k"], w["v"], spec, heads=[(0, 0), (0, 19), (0, 39)])
+
+
 def test_sparse_paged_full_size():
+    """The paged block-sparse workload against the oracle, and its contiguous-K/V
+    control (bench.py's sparse_contig workload) equal to it bit for bit."""
     w = workloads.sparse_paged()
     B, S, Hq, D = w["q"].shape
     Hkv = w["k"].shape[2]
     group = Hq // Hkv
-    o = fmha.fmha_fwd_paged(w["q"].to(DEV), w["k_pool"].to(DEV), w["v_pool"].to(DEV), w["page_table"].to(DEV), S,
-                            mask=w["mask"].to(DEV), softmax_scale=w["scale"])
+    q, dmask = w["q"].to(DEV), w["mask"].to(DEV)
+    o = fmha.fmha_fwd_paged(q, w["k_pool"].to(DEV), w["v_pool"].to(DEV), w["page_table"].to(DEV), S,
+                            mask=dmask, softmax_scale=w["scale"])
     fmha.get_device_error()
+    oc = fmha.fmha_fwd_block_sparse(q, w["k"].to(DEV), w["v"].to(DEV), dmask, softmax_scale=w["scale"])
+    fmha.get_device_error()
+    assert torch.equal(o, oc), "paged and contiguous K/V must give identical bits"
+    del oc
     mask = w["mask"].numpy()
     got, ref = {}, {}
     heads = [(0, 0), (1, 21), (3, 63)]
@@ -181,3 +197,23 @@ def test_sparse_paged_full_size():
         ref[(b, h)] = ro
         got[(b, h)] = f64(o[b, rows, h, :])
     check_rows("bf16", got, ref)
+
+
+def test_decode_paged_full_size():
+    """The decode workload (Sq = 1, B4 Hq64 Hkv8 Skv16384, 64-token pages, 25 % of the
+    128-key blocks kept) with automatic splits, as bench.py launches it: every output
+    row and its LSE against the oracle (the whole output is 256 rows)."""
+    from tests.helpers import assert_close_bf16
+
+    w = workloads.decode_paged()
+    B, Sq, Hq, D = w["q"].shape
+    S = w["k"].shape[1]
+    lse = torch.full((B, Hq, Sq), float("nan"), device=DEV)
+    o = fmha.fmha_fwd_decode(w["q"].to(DEV), w["k_pool"].to(DEV), w["v_pool"].to(DEV),
+                             page_table=w["page_table"].to(DEV), Skv=S, mask=w["mask"].to(DEV),
+                             softmax_scale=w["scale"], lse=lse)
+    fmha.get_device_error()
+    ref, ref_lse = oa.attention(f64(w["q"]), f64(w["k"]), f64(w["v"]), w["scale"], False, w["mask"].numpy())
+    assert_close_bf16(f64(o), ref)
+    got = f64(lse)
+    assert np.all(np.isfinite(got)) and np.abs(got - ref_lse).max() < 2e-2
