@@ -468,9 +468,12 @@ fmha_status run_attention(const fmha_args* a, const uint8_t* mask, int64_t msb, 
   return ok_status();
 }
 
-// Token rows one CTA of the channel-mean kernel sums: 128 KB of BF16 input
-// (few partials for the final sum; still several CTAs per SM at 16 K tokens).
-int mean_rows_per_cta(int D) { return D >= 8 ? 65536 / D : 1; }
+// Token rows one CTA of the channel-mean kernel sums: 256 KB of BF16 input, 64
+// rows per thread. At 48 registers a thread, 5 CTAs of 256 fit an SM; 128 KB
+// chunks gave the Sage workload's K (B1 H24 S16384) 768 CTAs, a second wave of
+// 28 on 148 SMs, while 256 KB chunks give 384 CTAs in one wave (2-3 per SM,
+// 64-96 KB of loads in flight each) and half the partials for the final sum.
+int mean_rows_per_cta(int D) { return D >= 8 ? 131072 / D : 1; }
 
 fmha_status quantize_impl(const fmha_tensor* src, const float* shift, const fmha_tensor* dst, const fmha_sf* sf,
                           int32_t B, int32_t S, int32_t H, int32_t D, void* workspace, size_t workspace_bytes,

@@ -190,19 +190,19 @@ def test_k_smoothing_entry_points_on_host(lib):
     names = declared_functions()
     for n in ("fmha_channel_mean", "fmha_channel_mean_workspace_bytes", "fmha_quantize_blockwise_shifted"):
         assert n in names and hasattr(lib, n)
-    # 512 rows of D = 128 per CTA: fp64 partial sums [B, H, chunks, D]
+    # 1024 rows of D = 128 per CTA: fp64 partial sums [B, H, chunks, D]
     assert fmha.channel_mean_workspace_bytes(2, 100, 3, 128) == 2 * 3 * 1 * 128 * 8
-    assert fmha.channel_mean_workspace_bytes(2, 1300, 3, 128) == 2 * 3 * 3 * 128 * 8
+    assert fmha.channel_mean_workspace_bytes(2, 2100, 3, 128) == 2 * 3 * 3 * 128 * 8
     assert fmha.channel_mean_workspace_bytes(2, 0, 3, 128) == 0
-    src = _bf16_tensor(2, 1300, 3, 128)
+    src = _bf16_tensor(2, 2100, 3, 128)
     mean, ws, need = 0x40000, 0x80000, 2 * 3 * 3 * 128 * 8
     f = lib.fmha_channel_mean
-    assert f(ctypes.byref(_bf16_tensor(2, 1300, 3, 96)), mean, 2, 1300, 3, 96, ws, need, None) == 2  # D not 2^k
-    assert f(ctypes.byref(src), mean + 2, 2, 1300, 3, 128, ws, need, None) == 1   # mean misaligned
-    assert f(ctypes.byref(src), None, 2, 1300, 3, 128, ws, need, None) == 1       # mean NULL
-    assert f(ctypes.byref(src), mean, 2, 1300, 3, 128, ws, need - 8, None) == 1   # workspace too small
-    assert f(ctypes.byref(src), mean, 2, 1300, 3, 128, ws + 4, need, None) == 1   # workspace misaligned
-    assert f(ctypes.byref(src), mean, 0, 1300, 3, 128, None, 0, None) == 0        # nothing to do
+    assert f(ctypes.byref(_bf16_tensor(2, 2100, 3, 96)), mean, 2, 2100, 3, 96, ws, need, None) == 2  # D not 2^k
+    assert f(ctypes.byref(src), mean + 2, 2, 2100, 3, 128, ws, need, None) == 1   # mean misaligned
+    assert f(ctypes.byref(src), None, 2, 2100, 3, 128, ws, need, None) == 1       # mean NULL
+    assert f(ctypes.byref(src), mean, 2, 2100, 3, 128, ws, need - 8, None) == 1   # workspace too small
+    assert f(ctypes.byref(src), mean, 2, 2100, 3, 128, ws + 4, need, None) == 1   # workspace misaligned
+    assert f(ctypes.byref(src), mean, 0, 2100, 3, 128, None, 0, None) == 0        # nothing to do
     g = lib.fmha_quantize_blockwise_shifted
     dst = _bf16_tensor(2, 300, 3, 128, ptr=0x100000)
     dst.dtype = fmha.INT8
