@@ -646,7 +646,7 @@ cudaError_t launch_quantize_t(const QuantParams& p, const CUtensorMap* tm, cudaS
 // of (b, h) per channel in fp64. Each thread owns one column vector (256 is a
 // multiple of D / 8) and a fixed set of rows; the threads of a column vector
 // are then added in thread order, so the partial sums do not depend on timing.
-__global__ void __launch_bounds__(kThreads) channel_mean_partial_kernel(const QuantParams p) {
+__global__ void __launch_bounds__(kThreads, 3) channel_mean_partial_kernel(const QuantParams p) {
   __shared__ double red[kThreads * 8];
   const int chunk = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
   const int s0 = chunk * p.rows_per_cta;
@@ -655,12 +655,24 @@ __global__ void __launch_bounds__(kThreads) channel_mean_partial_kernel(const Qu
   const int cv = threadIdx.x % vpr, row_step = kThreads / vpr;
   const uint16_t* src = p.src + b * p.s_sb + static_cast<int64_t>(s0) * p.s_ss + h * p.s_sh + cv * 8;
   double acc[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
-#pragma unroll 8
-  for (int r = threadIdx.x / vpr; r < rows; r += row_step) {
-    float x[8];
-    unpack8(ld16(src + r * p.s_ss), x);
+  // kU row vectors in flight per thread (3 CTAs of 256 fit an SM at this
+  // register count); the thread's rows are still added in ascending order.
+  constexpr int kU = 10;
+  for (int r0 = threadIdx.x / vpr; r0 < rows; r0 += kU * row_step) {
+    uint4 w[kU];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] += static_cast<double>(x[i]);
+    for (int u = 0; u < kU; ++u)  // unpredicated: rows past the end reload the last row
+      w[u] = ld16(src + static_cast<int64_t>(min(r0 + u * row_step, rows - 1)) * p.s_ss);
+    asm volatile("" ::: "memory");  // every load of the batch is issued before the first use
+#pragma unroll
+    for (int u = 0; u < kU; ++u) {
+      if (r0 + u * row_step < rows) {
+        float x[8];
+        unpack8(w[u], x);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] += static_cast<double>(x[i]);
+      }
+    }
   }
 #pragma unroll
   for (int i = 0; i < 8; ++i) red[threadIdx.x * 8 + i] = acc[i];
@@ -676,8 +688,8 @@ __global__ void __launch_bounds__(kThreads) channel_mean_partial_kernel(const Qu
 
 // Token mean, pass 2: one thread per (b, h, d) adds the chunks in order,
 // divides by S in fp64 and rounds once to fp32. The partials are loaded 16 at a
-// time before any is added (one memory round trip per 16 chunks instead of a
-// chain of dependent batches); the additions keep the chunk order.
+// time before any is added (one memory round trip per 16 chunks); the additions
+// keep the chunk order.
 __global__ void __launch_bounds__(kThreads) channel_mean_final_kernel(const QuantParams p) {
   constexpr int kBatch = 16;
   const int64_t i = static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x;
@@ -688,8 +700,9 @@ __global__ void __launch_bounds__(kThreads) channel_mean_final_kernel(const Quan
   for (int c0 = 0; c0 < p.n_chunks; c0 += kBatch) {
     double v[kBatch];
 #pragma unroll
-    for (int j = 0; j < kBatch; ++j)
-      v[j] = c0 + j < p.n_chunks ? part[static_cast<int64_t>(c0 + j) * p.D] : 0.0;
+    for (int j = 0; j < kBatch; ++j)  // unpredicated: past the last chunk, reload the last one
+      v[j] = part[static_cast<int64_t>(min(c0 + j, p.n_chunks - 1)) * p.D];
+    asm volatile("" ::: "memory");  // every load of the batch is issued before the first add
 #pragma unroll
     for (int j = 0; j < kBatch; ++j)
       if (c0 + j < p.n_chunks) a += v[j];
