@@ -40,9 +40,9 @@ the pages are silent is listed in the module that takes it.
 
 Parity pins: every function here is pinned by ``tests/test_oracle_*.py``
 against brute force, closed forms, invariants or an independent library
-routine. The one thing left unpinned is the GPU's internal quantization of
-the softmax output P (not an operand, so not modelled here): "parity
-unpinned" beyond the stated tolerance.
+routine. The attention runs on the dequantized operands; the kernels'
+internal cast of the softmax output P to E4M3 (P is not an operand) is not
+modelled here, so its effect is bounded only by the stated 8-bit tolerance.
 """
 
 from . import e4m3, quant, attention  # noqa: F401
