@@ -237,3 +237,16 @@ def test_sampled_rows_equal_full_attention(causal):
     assert np.allclose(o2, o[0, rows, 0], atol=1e-14)
     fin = np.isfinite(lse[0, 0, rows])
     assert np.array_equal(np.isfinite(lse2), fin) and np.allclose(lse2[fin], lse[0, 0, rows][fin], atol=1e-13)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_probabilities_times_v_equals_brute_force(causal):
+    """The invariant tests' helper: its P times V is the brute-force output."""
+    rng = np.random.default_rng(23)
+    Sq, Skv, D, blk = 9, 13, 6, 4
+    q, k, v = _rand(rng, 1, Sq, 1, D), _rand(rng, 1, Skv, 1, D), _rand(rng, 1, Skv, 1, D)
+    bm = rng.random((1, 1, -(-Sq // blk), -(-Skv // blk))) < 0.7
+    bm[..., -1] = True
+    p = A.probabilities(q[0, :, 0], k[0, :, 0], 0.7, causal, bm[0, 0], blk)
+    o_ref, _ = _brute(q, k, v, 0.7, causal, bm, blk)
+    assert np.allclose(p @ v[0, :, 0], o_ref[0, :, 0], atol=1e-13)

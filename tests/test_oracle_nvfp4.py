@@ -113,3 +113,20 @@ def test_packing_order():
     x[0, 0], x[0, 1] = 6.0, -3.0  # amax 6: e ~ 1, codes 7 and 13
     packed, sb, st = nvfp4.quantize_per_token(x)
     assert packed[0, 0] == (7 | (13 << 4))
+
+
+def test_every_block_maps_its_amax_to_six():
+    """The block scale is E4M3((amax_blk / s_t) / 6), so each block's largest
+    element lands on E2M1's largest magnitude: amax_blk / e = 6 q / decode(E4M3(q))
+    lies within 6 (1 +- 2^-4) whenever E4M3(q) is normal, which rounds (or
+    saturates) to 6. Blocks whose scale falls into E4M3's subnormal range have
+    coarser steps and are left out."""
+    x = rows_bf16(4, 16, 1024)
+    x *= np.exp2(np.random.default_rng(5).integers(-6, 4, size=(16, 64))).repeat(16, axis=1).astype(np.float32)
+    packed, sb, st = nvfp4.quantize_per_token(x)
+    codes = np.zeros(x.shape, dtype=np.uint8)
+    codes[:, 0::2], codes[:, 1::2] = packed & 0xF, packed >> 4
+    mags = np.abs(nvfp4.e2m1_decode(codes)).reshape(16, 64, 16).max(axis=2)
+    normal = e4m3.decode(sb) >= 2.0 ** -6
+    assert normal.sum() > 500
+    assert np.all(mags[normal] == 6.0)

@@ -10,6 +10,8 @@ granularities that must coincide.
 import numpy as np
 import pytest
 
+from fractions import Fraction
+
 from oracle import e4m3, quant
 
 
@@ -133,3 +135,43 @@ def test_e4m3_division_matches_torch_rounding():
     q = (x / scales[0]).astype(np.float32)
     ref = torch.from_numpy(q).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
     assert np.array_equal(codes, ref)
+
+
+def _rn32(fr):
+    """The float32 nearest to a positive rational, ties to even, exactly."""
+    f = np.float32(float(fr))
+    cands = [np.nextafter(f, np.float32(0)), f, np.nextafter(f, np.float32(np.inf))]
+    return min(cands, key=lambda c: (abs(Fraction(float(c)) - fr), int(np.float32(c).view(np.uint32)) & 1))
+
+
+@pytest.mark.parametrize("out", ["int8", "e4m3"])
+def test_scale_is_the_correctly_rounded_quotient(out):
+    """scale = RN(amax / R): for every positive finite BF16 amax, the float32
+    nearest to the exact rational amax / R (a multiplication by a rounded
+    reciprocal differs on some of them)."""
+    amax = (np.arange(1, 0x7F80, dtype=np.uint32) << 16).view(np.float32)
+    R = int(quant.RANGE[out])
+    got = quant.scale_from_amax(amax, out)
+    want = np.array([_rn32(Fraction(float(a)) / R) for a in amax], dtype=np.float32)
+    assert np.array_equal(got.view(np.uint32), want.view(np.uint32))
+
+
+@pytest.mark.parametrize("first_dominates", [True, False])
+def test_token_block_extent(first_dominates):
+    """Each token block covers exactly its rows: every block holds a spike in its
+    first and in its last row, and the dominant spike grows (first rows) or
+    shrinks (last rows) from block to block, so a block that reaches one row
+    into a neighbour, or stops one row short, takes a different amax. S = 200
+    with 64-row blocks leaves a ragged last block of 8 rows."""
+    rng = np.random.default_rng(6)
+    S, rpb, nblk = 200, 64, 4
+    x = (rng.uniform(-1.0, 1.0, size=(1, S, 2, 8))).astype(np.float32)
+    want = np.zeros((1, 2, nblk), dtype=np.float32)
+    for i in range(nblk):
+        first, last = i * rpb, min(S, (i + 1) * rpb) - 1
+        big = np.float32(10.0 * 4.0 ** i) if first_dominates else np.float32(10.0 * 4.0 ** (nblk - i))
+        x[0, first, :, 3] = big if first_dominates else big / 2
+        x[0, last, :, 5] = -(big / 2) if first_dominates else -big
+        want[0, :, i] = big
+    codes, scales = quant.quantize_blockwise(x, "int8", "per_token_block", rpb)
+    assert np.array_equal(scales, quant.scale_from_amax(want, "int8"))
