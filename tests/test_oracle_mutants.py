@@ -55,6 +55,10 @@ MUTANTS = [
      "p = e", ATT),
     ("probabilities_scale_dropped", oattn, "probabilities", "s = softmax_scale * (q @ k.T)", "s = q @ k.T", ATT),
     ("rows_scale_dropped", oattn, "attention_rows", "s = softmax_scale * (q @ k.T)", "s = q @ k.T", ATT),
+    ("row_chunk_drops_a_row", oattn, "attention", "r1 = min(Sq, r0 + ROW_CHUNK)",
+     "r1 = min(Sq, r0 + ROW_CHUNK - 1)", ATT),
+    ("row_chunk_mask_from_first_chunk", oattn, "attention", "vis = vis_full[r0:r1]", "vis = vis_full[:r1 - r0]",
+     ATT),
     # attention: paged gather
     ("page_row_off_by_one", oattn, "gather_paged", "(t % page_size)[None, :]", "((t + 1) % page_size)[None, :]",
      ATT),
@@ -78,6 +82,8 @@ MUTANTS = [
      QUANT),
     ("mean_over_s_minus_one", oquant, "channel_mean", "(total / np.float64(S))", "(total / np.float64(max(S - 1, 1)))",
      QUANT),
+    ("mean_summed_in_float32", oquant, "channel_mean", "total = x.astype(np.float64).sum(axis=1)",
+     "total = x.sum(axis=1, dtype=np.float32).astype(np.float64)", QUANT),
     ("dequant_next_block_scale", oquant, "dequantize", "idx = np.arange(S) // rows_per_block",
      "idx = np.minimum(np.arange(S) // rows_per_block + 1, sc.shape[2] - 1)", QUANT),
     # E4M3 codec

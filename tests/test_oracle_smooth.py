@@ -67,6 +67,22 @@ def test_channel_mean_axis_is_tokens():
                 assert m[b, h, d] == 100 * b + 10 * h + d
 
 
+def test_channel_mean_keeps_small_terms_next_to_large_ones():
+    """The sum is taken in float64: +-2^20 around 2^-10 terms (30 binades apart,
+    exact in float64, lost in a float32 running sum) leave the small terms' mean,
+    the correctly rounded fsum over S."""
+    S = 40
+    col = np.full(S, 2.0 ** -10, dtype=np.float32)
+    col[0], col[-1] = 2.0 ** 20, -(2.0 ** 20)  # first and last: a running sum holds 2^20 throughout
+    col[7] = np.float32(3.0 * 2.0 ** -9)
+    x = np.zeros((1, S, 1, 2), dtype=np.float32)
+    x[0, :, 0, 0] = col
+    x[0, :, 0, 1] = -col
+    want = np.float32(math.fsum(float(c) for c in col) / S)
+    m = quant.channel_mean(x)[0, 0]
+    assert m[0] == want and m[1] == -want and want > 0
+
+
 def test_channel_mean_empty():
     assert np.all(quant.channel_mean(np.zeros((1, 0, 2, 8), np.float32)) == 0)
 
