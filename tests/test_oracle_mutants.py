@@ -53,6 +53,9 @@ MUTANTS = [
     ("max_added", oattn, "attention", "e = np.exp(s - m_safe)", "e = np.exp(s + m_safe)", ATT),
     ("normaliser_dropped", oattn, "attention", "p = np.divide(e, l, out=np.zeros_like(e), where=l > 0)",
      "p = e", ATT),
+    ("lse_without_max", oattn, "attention", "m[:, 0] + np.log(np.where(", "np.log(np.where(", ATT),
+    ("hidden_rows_divided_by_zero", oattn, "attention", "p = np.divide(e, l, out=np.zeros_like(e), where=l > 0)",
+     "p = e / l", ATT),
     ("probabilities_scale_dropped", oattn, "probabilities", "s = softmax_scale * (q @ k.T)", "s = q @ k.T", ATT),
     ("rows_scale_dropped", oattn, "attention_rows", "s = softmax_scale * (q @ k.T)", "s = q @ k.T", ATT),
     ("row_chunk_drops_a_row", oattn, "attention", "r1 = min(Sq, r0 + ROW_CHUNK)",
@@ -67,6 +70,8 @@ MUTANTS = [
     # quantizer
     ("scale_by_reciprocal", oquant, "scale_from_amax", "scale = (amax_f32 / r).astype(np.float32)",
      "scale = (amax_f32 * np.float32(np.float32(1.0) / r)).astype(np.float32)", QUANT),
+    ("zero_amax_zero_scale", oquant, "scale_from_amax",
+     "np.where(amax_f32 == 0, np.float32(1.0), scale)", "scale", QUANT),
     ("int8_ties_away", oquant, "codes_with_scale", "np.clip(np.rint(q), -127, 127)",
      "np.clip(np.trunc(q + np.copysign(np.float32(0.5), q)), -127, 127)", QUANT),
     ("int8_range_128", oquant, None, "RANGE", {"int8": 128.0, "e4m3": 448.0}, QUANT),
@@ -95,11 +100,16 @@ MUTANTS = [
      (pins_e4m3,)),
     ("e4m3_subnormal_step_halved", oe4m3, "encode", "e = np.maximum(e, -6)", "e = np.maximum(e, -7)",
      (pins_e4m3,)),
+    ("e4m3_nan_code_finite", oe4m3, "decode", "val = np.where((exp_field == 0xF) & ((c & 0x7) == 0x7), np.nan, val)",
+     "val = val", (pins_e4m3,)),
     ("e4m3_negative_zero_unsigned", oe4m3, "encode", "neg = np.signbit(x)", "neg = x < 0", (pins_e4m3,)),
     # NVFP4
     ("nvfp4_token_scale_448", onvfp4, None, "ROW_RANGE", np.float32(448.0), (pins_nvfp4,)),
     ("e2m1_ties_down", onvfp4, "e2m1_encode", "better = (d < best) | ((d == best) & (c % 2 == 0))",
      "better = (d < best)", (pins_nvfp4,)),
+    ("zero_row_token_scale_zero", onvfp4, "quantize_per_token",
+     "s_t = np.float32(1.0) if amax == 0 else np.float32(amax / ROW_RANGE)", "s_t = np.float32(amax / ROW_RANGE)",
+     (pins_nvfp4,)),
     ("nibbles_swapped", onvfp4, "quantize_per_token", "packed = (codes4[:, 0::2] | (codes4[:, 1::2] << 4))",
      "packed = (codes4[:, 1::2] | (codes4[:, 0::2] << 4))", (pins_nvfp4,)),
     ("block_scale_without_e2m1_max", onvfp4, "quantize_per_token",
