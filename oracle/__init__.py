@@ -20,6 +20,11 @@ What it computes (plain, slow, obviously correct):
 * ``attention`` -- scaled-dot-product attention in float64 on dequantized
                    operands, with causal / 128x128 block masks, GQA and a
                    paged-KV gather.
+* ``online_softmax`` -- the same attention through the tiled online softmax
+                   (128-key tiles, lazy rescale past 2^tau) with P rounded as
+                   the kernels store it (BF16, one or two E4M3 terms with the P
+                   scale): a model of the approximation, for checks finer than
+                   the stated tolerance.
 
 Sources (page titles; sections):
 
@@ -27,7 +32,9 @@ Sources (page titles; sections):
   kernels" (flashinfer PR #2711), sections 2 (SageAttention scale factors) and
   "Why" item 2 (block-wise scaling beats per-tensor for outlier-heavy maps).
 * "FlashInfer FP8/BF16 mixed-precision attention for Blackwell" (flashinfer
-  PR #5900), introduction (dense context FMHA, QK-BF16/PV-FP8 and all-FP8).
+  PR #5900), introduction (dense context FMHA, QK-BF16/PV-FP8 and all-FP8),
+  sections 1 (P in FP8 staged for the PV product) and 3 (the row max moved
+  lazily, past a 2^8 jump).
 * "FlashInfer block-sparse attention with PrimTS" (flashinfer PR #4474),
   section 2 (block-sparse API over contiguous and paged K/V).
 * "FlashInfer per-token NVFP4 quantization kernel" (flashinfer PR #3237),
@@ -40,9 +47,11 @@ the pages are silent is listed in the module that takes it.
 
 Parity pins: every function here is pinned by ``tests/test_oracle_*.py``
 against brute force, closed forms, invariants or an independent library
-routine. The attention runs on the dequantized operands; the kernels'
-internal cast of the softmax output P to E4M3 (P is not an operand) is not
-modelled here, so its effect is bounded only by the stated 8-bit tolerance.
+routine. ``attention`` is the definition the tolerances are stated against
+(on the dequantized operands). The kernels' internal rounding of the softmax
+output P (not an operand) is modelled by ``online_softmax``, which is pinned to
+``attention`` when P is kept unrounded and to the formats' rounding bounds
+when it is not.
 """
 
-from . import e4m3, quant, attention  # noqa: F401
+from . import e4m3, quant, attention, online_softmax  # noqa: F401

@@ -1,0 +1,160 @@
+"""Attention through the tiled online softmax with P rounded as the kernels store it.
+
+TEST INFRASTRUCTURE ONLY (see ``oracle/__init__.py``).
+
+``attention.attention`` is the exact definition on dequantized operands. This
+module takes the steps of the method that approximate it, in the pages' order:
+the scores of one query row are taken 128 keys at a time; the running row max
+moves lazily, only when a tile's max exceeds it by more than tau (log2 units),
+and then O and the row sum are rescaled ("FlashInfer FP8/BF16 mixed-precision
+attention for Blackwell", section 3, with tau = 8 there); P is cast to BF16, or
+to E4M3 after multiplication by g = 1 / sf_p, the P scale factor of
+"FlashInfer DiT optimization: SageAttention and Int8/FP8 mixed-precision
+kernels", section 2; O accumulates P V; the epilogue divides by the row sum.
+
+Readings where the pages are silent (the same the kernels take):
+
+* Scores are in log2 units: s2 = softmax_scale * log2(e) * <q, k>.
+* The first tile in which a row sees a key sets its max; later tiles move it
+  (with O and l scaled by 2^(m_old - m_new)) only when their max exceeds it
+  by more than tau.
+* p = 2^(s2 - m) * g is formed in float32 (here: exactly, then rounded once
+  to float32; the "exact" mode keeps it in float64), so a stale max gives
+  p <= 2^tau * g.
+* tau = 8 for BF16 P; for E4M3 P, tau = floor(log2(448 * sf_p)) clamped to
+  [0, 8], so 2^tau * g <= 448. sf_p is one value, or one per (b, h_q,
+  128-row query block); without one, sf_p = 2^-4.
+* BF16 P: stored = RN_bf16(p); the row sum adds the unrounded p.
+* One E4M3 term: stored = E4M3(p) (RN-even, saturating); the row sum adds
+  the unrounded p plus, per tile, E4M3(p_max) - p_max for the tile's largest
+  p (so a dominant key's weight is normalised by its stored value).
+* Two E4M3 terms: hi = E4M3(p), lo = E4M3(RN_f16(RN_f16(p) - hi)), stored =
+  hi + lo; the row sum adds the unrounded p.
+* O = (sum over tiles of stored P V) / l; lse = (m + log2(l / g)) * ln 2;
+  a row with no visible key has O = 0 and lse = -inf.
+
+Not modelled: the exp2 unit's own error (here 2^x is exact before the float32
+rounding), and the order of the float32 additions of the row sum (here float64).
+These move a stored code only where p sits on an E4M3 or BF16 rounding
+boundary. The D_qk = 192 kernels with one query tile per CTA split the KV tiles
+of a row between two running states and merge them at the end; this module
+follows the single-state pass.
+"""
+
+import math
+
+import numpy as np
+
+from . import e4m3
+from .attention import visible_mask
+
+TILE = 128
+LOG2E = 1.0 / math.log(2.0)
+
+
+def _round_bf16(x32):
+    """float32 array -> nearest BF16 value (ties to even), as float32."""
+    u = np.asarray(x32, dtype=np.float32).view(np.uint32).astype(np.uint64)
+    u = (u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000
+    return u.astype(np.uint32).view(np.float32)
+
+
+def _round_e4m3(x):
+    return e4m3.decode(e4m3.encode(x))
+
+
+def _round_f16(x):
+    return np.asarray(x, dtype=np.float64).astype(np.float16).astype(np.float64)
+
+
+def tau_for(p_mode, sf_p):
+    """Lazy-rescale threshold in log2 units for one P scale."""
+    if p_mode == "bf16":
+        return 8.0
+    return float(min(8.0, max(0.0, math.floor(math.log2(448.0 * sf_p)))))
+
+
+def attention_rounded_p(q, k, v, softmax_scale, causal=False, block_mask=None, p_mode="e4m3", sf_p=None,
+                        p_block=128, block=128, tile=TILE, tau=None, stats=None):
+    """q [B, Sq, Hq, D], k [B, Skv, Hkv, D], v [B, Skv, Hkv, Dv] (dequantized values).
+
+    p_mode: "bf16", "e4m3" (one term), "e4m3x2" (two terms) or "exact" (P kept
+    unrounded: the online pass alone, which must equal ``attention.attention``).
+    sf_p: None (2^-4 for the E4M3 modes), a number, or an array [B, Hq,
+    ceil(Sq / p_block)] of per-query-block scales. tau: None (the reading's
+    threshold) or a number (the "exact" mode's rescale logic can then be
+    exercised at any threshold). stats: optional dict that receives the
+    largest stored P and the number of rescales.
+    Returns (o [B, Sq, Hq, Dv] float64, lse [B, Hq, Sq] float64).
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    B, Sq, Hq, D = q.shape
+    _, Skv, Hkv, Dv = v.shape
+    group = Hq // Hkv
+    if sf_p is None:
+        sf_p = 2.0 ** -4
+    sfp_arr = np.asarray(sf_p, dtype=np.float64)
+    o = np.zeros((B, Sq, Hq, Dv))
+    lse = np.full((B, Hq, Sq), -np.inf)
+    max_stored, rescales = 0.0, 0
+    for b in range(B):
+        for h in range(Hq):
+            hk = h // group
+            bm = None if block_mask is None else block_mask[b, hk]
+            vis = visible_mask(Sq, Skv, causal, bm, block)
+            s2 = (softmax_scale * LOG2E) * (q[b, :, h, :] @ k[b, :, hk, :].T)
+            s2 = np.where(vis, s2, -np.inf)
+            for r0 in range(0, Sq, p_block):  # rows of one P-scale block
+                r1 = min(Sq, r0 + p_block)
+                sfp = float(sfp_arr) if sfp_arr.ndim == 0 else float(sfp_arr[b, h, r0 // p_block])
+                g = 1.0 if p_mode in ("bf16", "exact") else 1.0 / sfp
+                tau_r = (tau_for(p_mode, sfp) if p_mode != "exact" else 8.0) if tau is None else float(tau)
+                n = r1 - r0
+                m = np.full(n, -np.inf)
+                l = np.zeros(n)
+                acc = np.zeros((n, Dv))
+                for c0 in range(0, Skv, tile):
+                    c1 = min(Skv, c0 + tile)
+                    st = s2[r0:r1, c0:c1]
+                    m_tile = st.max(axis=1)
+                    seen = np.isfinite(m_tile)
+                    first = seen & ~np.isfinite(m)
+                    move = seen & np.isfinite(m) & (m_tile > m + tau_r)
+                    alpha = np.exp2(np.where(move, m - np.where(move, m_tile, 0.0), 0.0))
+                    acc *= alpha[:, None]
+                    l *= alpha
+                    rescales += int(move.sum())
+                    m = np.where(first | move, m_tile, m)
+                    m_use = np.where(np.isfinite(m), m, 0.0)
+                    p = np.exp2(st - m_use[:, None]) * g  # 0 where hidden
+                    if p_mode != "exact":  # the kernels form p in float32
+                        p = p.astype(np.float32).astype(np.float64)
+                    if p_mode == "exact":
+                        stored, corr = p, 0.0
+                    elif p_mode == "bf16":
+                        stored, corr = _round_bf16(p).astype(np.float64), 0.0
+                    elif p_mode == "e4m3":
+                        stored = _round_e4m3(p)
+                        pmax = np.where(seen, (np.exp2(np.where(seen, m_tile - m_use, 0.0)) * g), 0.0)
+                        pmax = pmax.astype(np.float32).astype(np.float64)
+                        corr = np.where(seen, _round_e4m3(pmax) - pmax, 0.0)
+                    elif p_mode == "e4m3x2":
+                        hi = _round_e4m3(p)
+                        lo = _round_e4m3(_round_f16(_round_f16(p) - hi))
+                        stored, corr = hi + lo, 0.0
+                    else:
+                        raise ValueError(p_mode)
+                    if stored.size:
+                        max_stored = max(max_stored, float(stored.max()))
+                    l += p.sum(axis=1) + corr
+                    acc += stored @ v[b, c0:c1, hk, :]
+                alive = l > 0
+                o[b, r0:r1, h, :] = np.where(alive[:, None], acc / np.where(alive, l, 1.0)[:, None], 0.0)
+                lse[b, h, r0:r1] = np.where(alive, (m + np.log2(np.where(alive, l, 1.0) / g)) * math.log(2.0),
+                                            -np.inf)
+    if stats is not None:
+        stats["max_stored"] = max_stored
+        stats["rescales"] = rescales
+    return o, lse

@@ -23,10 +23,12 @@ import pytest
 from oracle import attention as oattn
 from oracle import e4m3 as oe4m3
 from oracle import nvfp4 as onvfp4
+from oracle import online_softmax as oonline
 from oracle import quant as oquant
 from tests import test_oracle_attention as pins_attention
 from tests import test_oracle_e4m3 as pins_e4m3
 from tests import test_oracle_nvfp4 as pins_nvfp4
+from tests import test_oracle_online_softmax as pins_online
 from tests import test_oracle_quant as pins_quant
 from tests import test_oracle_smooth as pins_smooth
 
@@ -103,6 +105,25 @@ MUTANTS = [
     ("e4m3_nan_code_finite", oe4m3, "decode", "val = np.where((exp_field == 0xF) & ((c & 0x7) == 0x7), np.nan, val)",
      "val = val", (pins_e4m3,)),
     ("e4m3_negative_zero_unsigned", oe4m3, "encode", "neg = np.signbit(x)", "neg = x < 0", (pins_e4m3,)),
+    # online softmax with rounded P
+    ("rescale_on_every_rise", oonline, "attention_rounded_p", "& (m_tile > m + tau_r)", "& (m_tile > m)",
+     (pins_online,)),
+    ("rescale_skips_row_sum", oonline, "attention_rounded_p", "l *= alpha", "l *= 1.0", (pins_online,)),
+    ("rescale_skips_o", oonline, "attention_rounded_p", "acc *= alpha[:, None]", "acc *= 1.0", (pins_online,)),
+    ("row_sum_correction_dropped", oonline, "attention_rounded_p", "l += p.sum(axis=1) + corr",
+     "l += p.sum(axis=1)", (pins_online,)),
+    ("p_scale_not_applied", oonline, "attention_rounded_p",
+     'g = 1.0 if p_mode in ("bf16", "exact") else 1.0 / sfp', "g = 1.0", (pins_online,)),
+    ("low_term_dropped", oonline, "attention_rounded_p", "stored, corr = hi + lo, 0.0", "stored, corr = hi, 0.0",
+     (pins_online,)),
+    ("bf16_truncates", oonline, "_round_bf16", "u = (u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000",
+     "u = u & 0xFFFF0000", (pins_online,)),
+    ("tau_rounded_up", oonline, "tau_for", "math.floor(math.log2(448.0 * sf_p))",
+     "math.ceil(math.log2(448.0 * sf_p))", (pins_online,)),
+    ("lse_without_p_scale", oonline, "attention_rounded_p", "np.log2(np.where(alive, l, 1.0) / g)",
+     "np.log2(np.where(alive, l, 1.0))", (pins_online,)),
+    ("p_scale_of_first_block", oonline, "attention_rounded_p", "sfp_arr[b, h, r0 // p_block]", "sfp_arr[b, h, 0]",
+     (pins_online,)),
     # NVFP4
     ("nvfp4_token_scale_448", onvfp4, None, "ROW_RANGE", np.float32(448.0), (pins_nvfp4,)),
     ("e2m1_ties_down", onvfp4, "e2m1_encode", "better = (d < best) | ((d == best) & (c % 2 == 0))",
@@ -168,7 +189,7 @@ def install(monkeypatch, module, func, old, new):
 
 def test_unmutated_oracle_passes_every_pin():
     """The harness itself: the real oracle passes every case it runs."""
-    mods = (pins_attention, pins_quant, pins_smooth, pins_e4m3, pins_nvfp4)
+    mods = (pins_attention, pins_quant, pins_smooth, pins_e4m3, pins_nvfp4, pins_online)
     assert sum(1 for m in mods for _ in pin_cases(m)) > 60
     assert first_failure(mods) is None
 
