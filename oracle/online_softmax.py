@@ -74,8 +74,70 @@ def tau_for(p_mode, sf_p):
     return float(min(8.0, max(0.0, math.floor(math.log2(448.0 * sf_p)))))
 
 
+def _tile_pass(s2, vv, tiles, tile, p_mode, g, tau, counters):
+    """One running state over the KV tiles ``tiles`` (start columns, in order)
+    for the rows of s2 [rows, Skv] (log2 scores, -inf where hidden); vv [Skv, Dv].
+    Returns (acc [rows, Dv], l [rows], m [rows]): O before normalisation, the
+    row sum and the lazy max."""
+    n, Dv = s2.shape[0], vv.shape[1]
+    m = np.full(n, -np.inf)
+    l = np.zeros(n)
+    acc = np.zeros((n, Dv))
+    for c0 in tiles:
+        c1 = min(s2.shape[1], c0 + tile)
+        st = s2[:, c0:c1]
+        m_tile = st.max(axis=1)
+        seen = np.isfinite(m_tile)
+        first = seen & ~np.isfinite(m)
+        move = seen & np.isfinite(m) & (m_tile > m + tau)
+        alpha = np.exp2(np.where(move, m - np.where(move, m_tile, 0.0), 0.0))
+        acc *= alpha[:, None]
+        l *= alpha
+        counters["rescales"] += int(move.sum())
+        m = np.where(first | move, m_tile, m)
+        m_use = np.where(np.isfinite(m), m, 0.0)
+        p = np.exp2(st - m_use[:, None]) * g  # 0 where hidden
+        if p_mode != "exact":  # the kernels form p in float32
+            p = p.astype(np.float32).astype(np.float64)
+        if p_mode == "exact":
+            stored, corr = p, 0.0
+        elif p_mode == "bf16":
+            stored, corr = _round_bf16(p).astype(np.float64), 0.0
+        elif p_mode == "e4m3":
+            stored = _round_e4m3(p)
+            pmax = np.where(seen, (np.exp2(np.where(seen, m_tile - m_use, 0.0)) * g), 0.0)
+            pmax = pmax.astype(np.float32).astype(np.float64)
+            corr = np.where(seen, _round_e4m3(pmax) - pmax, 0.0)
+        elif p_mode == "e4m3x2":
+            hi = _round_e4m3(p)
+            lo = _round_e4m3(_round_f16(_round_f16(p) - hi))
+            stored, corr = hi + lo, 0.0
+        else:
+            raise ValueError(p_mode)
+        if stored.size:
+            counters["max_stored"] = max(counters["max_stored"], float(stored.max()))
+        l += p.sum(axis=1) + corr
+        acc += stored @ vv[c0:c1]
+    return acc, l, m
+
+
+def _kept_tiles(b, hk, qblk, Sq, Skv, causal, block_mask, tile):
+    """Start columns of the KV tiles a 128-row query tile keeps: within its
+    causal bound (its last row's) and kept by the block mask, in order."""
+    n = -(-Skv // tile)
+    if causal:
+        last = min(qblk * tile + tile - 1, Sq - 1) + (Skv - Sq)
+        n = 0 if last < 0 else min(n, last // tile + 1)
+    return [u * tile for u in range(n) if block_mask is None or block_mask[b, hk, qblk, u]]
+
+
+def _deal(kept):
+    """Kept tiles by rank: even ranks to the first state, odd to the second."""
+    return kept[0::2], kept[1::2]
+
+
 def attention_rounded_p(q, k, v, softmax_scale, causal=False, block_mask=None, p_mode="e4m3", sf_p=None,
-                        p_block=128, block=128, tile=TILE, tau=None, stats=None):
+                        p_block=128, block=128, tile=TILE, tau=None, split_kv=False, stats=None):
     """q [B, Sq, Hq, D], k [B, Skv, Hkv, D], v [B, Skv, Hkv, Dv] (dequantized values).
 
     p_mode: "bf16", "e4m3" (one term), "e4m3x2" (two terms) or "exact" (P kept
@@ -83,9 +145,14 @@ def attention_rounded_p(q, k, v, softmax_scale, causal=False, block_mask=None, p
     sf_p: None (2^-4 for the E4M3 modes), a number, or an array [B, Hq,
     ceil(Sq / p_block)] of per-query-block scales. tau: None (the reading's
     threshold) or a number (the "exact" mode's rescale logic can then be
-    exercised at any threshold). stats: optional dict that receives the
-    largest stored P and the number of rescales.
-    Returns (o [B, Sq, Hq, Dv] float64, lse [B, Hq, Sq] float64).
+    exercised at any threshold). split_kv: the kept KV tiles of each 128-row
+    query tile are dealt by rank to two running states (even ranks to one, odd
+    to the other), which are merged at the end:
+    O = (acc_0 2^(m_0 - M) + acc_1 2^(m_1 - M)) / (l_0 2^(m_0 - M) + l_1 2^(m_1 - M)),
+    M = max(m_0, m_1) (the one-query-tile schedule of the 192-wide QK kernels;
+    needs 128-key tiles, 128-row P blocks and a 128 x 128 block mask).
+    stats: optional dict that receives the largest stored P and the number of
+    rescales. Returns (o [B, Sq, Hq, Dv] float64, lse [B, Hq, Sq] float64).
     """
     q = np.asarray(q, dtype=np.float64)
     k = np.asarray(k, dtype=np.float64)
@@ -93,12 +160,14 @@ def attention_rounded_p(q, k, v, softmax_scale, causal=False, block_mask=None, p
     B, Sq, Hq, D = q.shape
     _, Skv, Hkv, Dv = v.shape
     group = Hq // Hkv
+    if split_kv and not (tile == p_block == block == TILE):
+        raise ValueError("split_kv follows the kernels' 128-row, 128-key tiles")
     if sf_p is None:
         sf_p = 2.0 ** -4
     sfp_arr = np.asarray(sf_p, dtype=np.float64)
     o = np.zeros((B, Sq, Hq, Dv))
     lse = np.full((B, Hq, Sq), -np.inf)
-    max_stored, rescales = 0.0, 0
+    counters = {"max_stored": 0.0, "rescales": 0}
     for b in range(B):
         for h in range(Hq):
             hk = h // group
@@ -106,55 +175,28 @@ def attention_rounded_p(q, k, v, softmax_scale, causal=False, block_mask=None, p
             vis = visible_mask(Sq, Skv, causal, bm, block)
             s2 = (softmax_scale * LOG2E) * (q[b, :, h, :] @ k[b, :, hk, :].T)
             s2 = np.where(vis, s2, -np.inf)
+            vv = v[b, :, hk, :]
             for r0 in range(0, Sq, p_block):  # rows of one P-scale block
                 r1 = min(Sq, r0 + p_block)
                 sfp = float(sfp_arr) if sfp_arr.ndim == 0 else float(sfp_arr[b, h, r0 // p_block])
                 g = 1.0 if p_mode in ("bf16", "exact") else 1.0 / sfp
                 tau_r = (tau_for(p_mode, sfp) if p_mode != "exact" else 8.0) if tau is None else float(tau)
-                n = r1 - r0
-                m = np.full(n, -np.inf)
-                l = np.zeros(n)
-                acc = np.zeros((n, Dv))
-                for c0 in range(0, Skv, tile):
-                    c1 = min(Skv, c0 + tile)
-                    st = s2[r0:r1, c0:c1]
-                    m_tile = st.max(axis=1)
-                    seen = np.isfinite(m_tile)
-                    first = seen & ~np.isfinite(m)
-                    move = seen & np.isfinite(m) & (m_tile > m + tau_r)
-                    alpha = np.exp2(np.where(move, m - np.where(move, m_tile, 0.0), 0.0))
-                    acc *= alpha[:, None]
-                    l *= alpha
-                    rescales += int(move.sum())
-                    m = np.where(first | move, m_tile, m)
+                if not split_kv:
+                    acc, l, m = _tile_pass(s2[r0:r1], vv, range(0, Skv, tile), tile, p_mode, g, tau_r, counters)
+                else:
+                    kept = _kept_tiles(b, hk, r0 // tile, Sq, Skv, causal, block_mask, tile)
+                    parts = [_tile_pass(s2[r0:r1], vv, half, tile, p_mode, g, tau_r, counters)
+                             for half in _deal(kept)]
+                    ms = np.stack([np.where(pl > 0, pm, -np.inf) for _, pl, pm in parts])
+                    m = ms.max(axis=0)
                     m_use = np.where(np.isfinite(m), m, 0.0)
-                    p = np.exp2(st - m_use[:, None]) * g  # 0 where hidden
-                    if p_mode != "exact":  # the kernels form p in float32
-                        p = p.astype(np.float32).astype(np.float64)
-                    if p_mode == "exact":
-                        stored, corr = p, 0.0
-                    elif p_mode == "bf16":
-                        stored, corr = _round_bf16(p).astype(np.float64), 0.0
-                    elif p_mode == "e4m3":
-                        stored = _round_e4m3(p)
-                        pmax = np.where(seen, (np.exp2(np.where(seen, m_tile - m_use, 0.0)) * g), 0.0)
-                        pmax = pmax.astype(np.float32).astype(np.float64)
-                        corr = np.where(seen, _round_e4m3(pmax) - pmax, 0.0)
-                    elif p_mode == "e4m3x2":
-                        hi = _round_e4m3(p)
-                        lo = _round_e4m3(_round_f16(_round_f16(p) - hi))
-                        stored, corr = hi + lo, 0.0
-                    else:
-                        raise ValueError(p_mode)
-                    if stored.size:
-                        max_stored = max(max_stored, float(stored.max()))
-                    l += p.sum(axis=1) + corr
-                    acc += stored @ v[b, c0:c1, hk, :]
+                    w = [np.where(pl > 0, np.exp2(np.where(pl > 0, pm - m_use, 0.0)), 0.0) for _, pl, pm in parts]
+                    acc = parts[0][0] * w[0][:, None] + parts[1][0] * w[1][:, None]
+                    l = parts[0][1] * w[0] + parts[1][1] * w[1]
                 alive = l > 0
                 o[b, r0:r1, h, :] = np.where(alive[:, None], acc / np.where(alive, l, 1.0)[:, None], 0.0)
                 lse[b, h, r0:r1] = np.where(alive, (m + np.log2(np.where(alive, l, 1.0) / g)) * math.log(2.0),
                                             -np.inf)
     if stats is not None:
-        stats["max_stored"] = max_stored
-        stats["rescales"] = rescales
+        stats.update(counters)
     return o, lse

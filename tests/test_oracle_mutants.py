@@ -106,15 +106,15 @@ MUTANTS = [
      "val = val", (pins_e4m3,)),
     ("e4m3_negative_zero_unsigned", oe4m3, "encode", "neg = np.signbit(x)", "neg = x < 0", (pins_e4m3,)),
     # online softmax with rounded P
-    ("rescale_on_every_rise", oonline, "attention_rounded_p", "& (m_tile > m + tau_r)", "& (m_tile > m)",
+    ("rescale_on_every_rise", oonline, "_tile_pass", "& (m_tile > m + tau)", "& (m_tile > m)",
      (pins_online,)),
-    ("rescale_skips_row_sum", oonline, "attention_rounded_p", "l *= alpha", "l *= 1.0", (pins_online,)),
-    ("rescale_skips_o", oonline, "attention_rounded_p", "acc *= alpha[:, None]", "acc *= 1.0", (pins_online,)),
-    ("row_sum_correction_dropped", oonline, "attention_rounded_p", "l += p.sum(axis=1) + corr",
+    ("rescale_skips_row_sum", oonline, "_tile_pass", "l *= alpha", "l *= 1.0", (pins_online,)),
+    ("rescale_skips_o", oonline, "_tile_pass", "acc *= alpha[:, None]", "acc *= 1.0", (pins_online,)),
+    ("row_sum_correction_dropped", oonline, "_tile_pass", "l += p.sum(axis=1) + corr",
      "l += p.sum(axis=1)", (pins_online,)),
     ("p_scale_not_applied", oonline, "attention_rounded_p",
      'g = 1.0 if p_mode in ("bf16", "exact") else 1.0 / sfp', "g = 1.0", (pins_online,)),
-    ("low_term_dropped", oonline, "attention_rounded_p", "stored, corr = hi + lo, 0.0", "stored, corr = hi, 0.0",
+    ("low_term_dropped", oonline, "_tile_pass", "stored, corr = hi + lo, 0.0", "stored, corr = hi, 0.0",
      (pins_online,)),
     ("bf16_truncates", oonline, "_round_bf16", "u = (u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000",
      "u = u & 0xFFFF0000", (pins_online,)),
@@ -124,6 +124,13 @@ MUTANTS = [
      "np.log2(np.where(alive, l, 1.0))", (pins_online,)),
     ("p_scale_of_first_block", oonline, "attention_rounded_p", "sfp_arr[b, h, r0 // p_block]", "sfp_arr[b, h, 0]",
      (pins_online,)),
+    ("merge_without_max_weights", oonline, "attention_rounded_p",
+     "w = [np.where(pl > 0, np.exp2(np.where(pl > 0, pm - m_use, 0.0)), 0.0) for _, pl, pm in parts]",
+     "w = [np.where(pl > 0, 1.0, 0.0) for _, pl, pm in parts]", (pins_online,)),
+    ("deal_by_halves", oonline, "_deal", "return kept[0::2], kept[1::2]",
+     "return kept[:(len(kept) + 1) // 2], kept[(len(kept) + 1) // 2:]", (pins_online,)),
+    ("kept_tiles_first_row_bound", oonline, "_kept_tiles",
+     "last = min(qblk * tile + tile - 1, Sq - 1) + (Skv - Sq)", "last = qblk * tile + (Skv - Sq)", (pins_online,)),
     # NVFP4
     ("nvfp4_token_scale_448", onvfp4, None, "ROW_RANGE", np.float32(448.0), (pins_nvfp4,)),
     ("e2m1_ties_down", onvfp4, "e2m1_encode", "better = (d < best) | ((d == best) & (c % 2 == 0))",

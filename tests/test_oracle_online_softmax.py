@@ -197,3 +197,55 @@ def test_sage_p_scale_reading():
            for mode in ("e4m3", "e4m3x2") for sfp in (1 / 16, 1 / 224)}
     assert err[("e4m3", 1 / 224)] < err[("e4m3", 1 / 16)]
     assert err[("e4m3x2", 1 / 224)] < err[("e4m3", 1 / 224)] / 8
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_split_states_merge_to_the_exact_attention(causal):
+    """Two running states over alternate kept tiles, merged with the
+    2^(m_x - M) weights: with P unrounded the merge is the exact attention,
+    whatever the thresholds (causal with Skv > Sq, a block mask with a hidden
+    query block, GQA)."""
+    rng = np.random.default_rng(38)
+    B, Sq, Skv, Hq, Hkv, D, Dv = 1, 300, 700, 2, 1, 8, 6
+    q, k, v = _rand(rng, B, Sq, Hq, D) * 2, _rand(rng, B, Skv, Hkv, D) * 2, _rand(rng, B, Skv, Hkv, Dv)
+    bm = rng.random((B, Hkv, 3, 6)) < 0.6
+    bm[0, 0, 1, :] = False
+    bm[0, 0, 2, :] = [True, False, True, True, False, True]
+    ref, ref_lse = A.attention(q, k, v, 0.9, causal, bm)
+    for tau in (0.0, 8.0):
+        o, lse = OS.attention_rounded_p(q, k, v, 0.9, causal, bm, p_mode="exact", tau=tau, split_kv=True)
+        assert np.allclose(o, ref, atol=1e-12, rtol=0)
+        fin = np.isfinite(ref_lse)
+        assert np.array_equal(np.isfinite(lse), fin) and np.allclose(lse[fin], ref_lse[fin], atol=1e-12)
+
+
+def test_split_dealing_and_kept_tiles():
+    """The tiles a query tile keeps (its last row's causal bound, the block mask)
+    and their dealing by rank parity."""
+    assert OS._kept_tiles(0, 0, 0, 300, 700, True, None, 128) == [0, 128, 256, 384, 512]  # last row 527
+    assert OS._kept_tiles(0, 0, 2, 300, 700, True, None, 128) == [0, 128, 256, 384, 512, 640]
+    assert OS._kept_tiles(0, 0, 0, 700, 300, True, None, 128) == []  # rows 0..127 see no key (bottom-right)
+    bm = np.zeros((1, 1, 3, 6), dtype=bool)
+    bm[0, 0, 1, [0, 2, 3, 5]] = True
+    assert OS._kept_tiles(0, 0, 1, 300, 700, False, bm, 128) == [0, 256, 384, 640]
+    assert OS._deal([0, 256, 384, 640, 768]) == ([0, 384, 768], [256, 640])
+
+
+@pytest.mark.parametrize("p_mode,rel", [("e4m3", None), ("bf16", 2.0 ** -8)])
+def test_split_states_within_the_rounding_bounds(p_mode, rel):
+    """The rounded modes through two states stay within the same format bounds
+    (each state's row sum carries its own tiles' corrections)."""
+    rng = np.random.default_rng(39)
+    S, D = 600, 16
+    q = rng.uniform(-1, 1, (1, S, 1, D))
+    k = rng.uniform(-1, 1, (1, S, 1, D))
+    v = _rand(rng, 1, S, 1, D)
+    o, _ = OS.attention_rounded_p(q, k, v, 0.2, True, p_mode=p_mode, sf_p=1 / 224, split_kv=True)
+    ref, _ = A.attention(q, k, v, 0.2, True)
+    _, spv, pmax = _bound_terms(q, k, v, 0.2, True)
+    r = ref[0, :, 0]
+    if rel is None:
+        bound = 2.0 ** -4 * (spv + np.abs(r) * pmax[:, None]) / (1 - 2.0 ** -4 * pmax[:, None])
+    else:
+        bound = rel * spv
+    assert np.all(np.abs(o[0, :, 0] - r) <= bound * (1 + 1e-6) + 1e-9)
