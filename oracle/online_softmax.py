@@ -200,3 +200,88 @@ def attention_rounded_p(q, k, v, softmax_scale, causal=False, block_mask=None, p
     if stats is not None:
         stats.update(counters)
     return o, lse
+
+
+def _split_groups(kept, n_splits, interleave):
+    """The KV tile groups of a decode tile's partials: split s takes the ranks
+    [s * per, (s + 1) * per) of the kept tiles, per = ceil(total / n_splits);
+    with interleave, two partials per split take the split's ranks alternately
+    (rank - s * per even, then odd)."""
+    total = len(kept)
+    per = -(-total // n_splits) if total else 0
+    groups = []
+    for s in range(n_splits):
+        mine = kept[s * per:min(total, (s + 1) * per)]
+        groups += [mine[0::2], mine[1::2]] if interleave else [mine]
+    return groups
+
+
+def decode_rounded_p(q, k, v, softmax_scale, causal=False, block_mask=None, p_mode="e4m3", sf_p=None, n_splits=1,
+                     tile=TILE, stats=None):
+    """The decode path's schedule with rounded P, for q [B, Sq, Hq, D] (a few
+    query tokens), k [B, Skv, Hkv, D], v [B, Skv, Hkv, Dv].
+
+    The Sq * G rows of one KV head (G = Hq / Hkv, a power of two) are packed
+    token-major, row r = (token r // G, head r % G), into 128-row tiles (the
+    query tile is the query block times the query heads per KV head, "FlashInfer
+    block-sparse attention with PrimTS", section 1). Each tile ranks the KV
+    tiles it keeps (its last token's causal bound, the block mask row of its
+    tokens); split s of n_splits takes ranks [s * per, (s + 1) * per), per =
+    ceil(total / n_splits). When all rows fit one tile, each split has two
+    partials taking its ranks alternately. Every partial is one running state
+    (the tiled pass with rounded P); the partials merge by their log-sum-exp:
+    lse = log sum_j exp(lse_j), O = sum_j exp(lse_j - lse) O_j, O_j = acc_j / l_j.
+    sf_p: None (2^-4 for the E4M3 modes) or one number. Returns (o, lse) as
+    ``attention_rounded_p`` does.
+    """
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    B, Sq, Hq, D = q.shape
+    _, Skv, Hkv, Dv = v.shape
+    G = Hq // Hkv
+    sfp = 2.0 ** -4 if sf_p is None else float(sf_p)
+    g = 1.0 if p_mode in ("bf16", "exact") else 1.0 / sfp
+    tau = tau_for(p_mode, sfp) if p_mode != "exact" else 8.0
+    n_rows = Sq * G
+    units = -(-n_rows // TILE)
+    interleave = units == 1
+    toks = TILE // G  # query tokens per 128-row tile
+    n_kv = -(-Skv // tile)
+    o = np.zeros((B, Sq, Hq, Dv))
+    lse = np.full((B, Hq, Sq), -np.inf)
+    counters = {"max_stored": 0.0, "rescales": 0}
+    for b in range(B):
+        for hk in range(Hkv):
+            bm = None if block_mask is None else block_mask[b, hk]
+            vis = visible_mask(Sq, Skv, causal, bm, TILE)  # per token
+            vv = v[b, :, hk, :]
+            for u in range(units):
+                rows = np.arange(u * TILE, min(n_rows, (u + 1) * TILE))
+                tok, head = rows // G, hk * G + rows % G
+                s2 = (softmax_scale * LOG2E) * np.einsum("rd,kd->rk", q[b, tok, head, :], k[b, :, hk, :])
+                s2 = np.where(vis[tok], s2, -np.inf)
+                tok0 = u * toks
+                n = n_kv
+                if causal:
+                    last = min(tok0 + toks - 1, Sq - 1) + (Skv - Sq)
+                    n = 0 if last < 0 else min(n_kv, last // tile + 1)
+                kept = [c * tile for c in range(n) if bm is None or bm[tok0 // TILE, c]]
+                parts = [_tile_pass(s2, vv, grp, tile, p_mode, g, tau, counters)
+                         for grp in _split_groups(kept, n_splits, interleave)]
+                # each partial: O_j = acc / l, lse_j; then the log-sum-exp merge
+                lse_j = np.stack([np.where(pl > 0, (pm + np.log2(np.where(pl > 0, pl, 1.0) / g)) * math.log(2.0),
+                                           -np.inf) for _, pl, pm in parts])
+                o_j = np.stack([np.where((pl > 0)[:, None], pa / np.where(pl > 0, pl, 1.0)[:, None], 0.0)
+                                for pa, pl, _ in parts])
+                mx = lse_j.max(axis=0)
+                alive = np.isfinite(mx)
+                w = np.where(np.isfinite(lse_j), np.exp(lse_j - np.where(alive, mx, 0.0)[None]), 0.0)
+                wsum = w.sum(axis=0)
+                o[b, tok, head, :] = np.where(alive[:, None], (w[:, :, None] * o_j).sum(axis=0)
+                                              / np.where(alive, wsum, 1.0)[:, None], 0.0)
+                lse[b, head, tok] = np.where(alive, np.where(alive, mx, 0.0) + np.log(np.where(alive, wsum, 1.0)),
+                                             -np.inf)
+    if stats is not None:
+        stats.update(counters)
+    return o, lse

@@ -131,6 +131,16 @@ MUTANTS = [
      "return kept[:(len(kept) + 1) // 2], kept[(len(kept) + 1) // 2:]", (pins_online,)),
     ("kept_tiles_first_row_bound", oonline, "_kept_tiles",
      "last = min(qblk * tile + tile - 1, Sq - 1) + (Skv - Sq)", "last = qblk * tile + (Skv - Sq)", (pins_online,)),
+    ("decode_per_rounded_down", oonline, "_split_groups", "per = -(-total // n_splits) if total else 0",
+     "per = max(1, total // n_splits) if total else 0", (pins_online,)),
+    ("decode_interleave_by_halves", oonline, "_split_groups", "groups += [mine[0::2], mine[1::2]] if interleave",
+     "groups += [mine[:len(mine) // 2], mine[len(mine) // 2:]] if interleave", (pins_online,)),
+    ("decode_merge_base_two", oonline, "decode_rounded_p", "np.exp(lse_j - np.where(alive, mx, 0.0)[None])",
+     "np.exp2(lse_j - np.where(alive, mx, 0.0)[None])", (pins_online,)),
+    ("decode_head_major_packing", oonline, "decode_rounded_p", "tok, head = rows // G, hk * G + rows % G",
+     "tok, head = rows % Sq, hk * G + rows // Sq", (pins_online,)),
+    ("decode_mask_row_by_tile", oonline, "decode_rounded_p", "bm[tok0 // TILE, c]", "bm[min(u, bm.shape[0] - 1), c]",
+     (pins_online,)),
     # NVFP4
     ("nvfp4_token_scale_448", onvfp4, None, "ROW_RANGE", np.float32(448.0), (pins_nvfp4,)),
     ("e2m1_ties_down", onvfp4, "e2m1_encode", "better = (d < best) | ((d == best) & (c % 2 == 0))",

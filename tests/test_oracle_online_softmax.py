@@ -249,3 +249,58 @@ def test_split_states_within_the_rounding_bounds(p_mode, rel):
     else:
         bound = rel * spv
     assert np.all(np.abs(o[0, :, 0] - r) <= bound * (1 + 1e-6) + 1e-9)
+
+
+@pytest.mark.parametrize("B,Sq,Hq,Hkv,Skv,causal,masked", [
+    (2, 1, 16, 2, 2000, False, True),   # one token, G = 8: all rows in one tile (two partials per split)
+    (1, 5, 8, 1, 1000, True, False),    # causal, ragged token tail
+    (2, 40, 32, 2, 1500, True, False),  # G = 16: 640 packed rows, five tiles
+    (1, 33, 4, 4, 900, False, True),    # G = 1
+    (1, 2, 128, 1, 600, False, False),  # G = 128: one token per tile
+    (1, 130, 2, 1, 700, True, True),    # tiles across a 128-token mask row
+])
+@pytest.mark.parametrize("n_splits", [1, 3, 8])
+def test_decode_schedule_merges_to_the_exact_attention(B, Sq, Hq, Hkv, Skv, causal, masked, n_splits):
+    """Packed rows, ranked and split KV tiles, interleaved partials and the
+    log-sum-exp merge: with P unrounded, the exact attention."""
+    rng = np.random.default_rng(40 + Sq + n_splits)
+    q, k, v = _rand(rng, B, Sq, Hq, 128) * 2, _rand(rng, B, Skv, Hkv, 128) * 2, _rand(rng, B, Skv, Hkv, 128)
+    bm = None
+    if masked:
+        bm = rng.random((B, Hkv, -(-Sq // 128), -(-Skv // 128))) < 0.5
+        bm[..., -1] = True
+    ref, ref_lse = A.attention(q, k, v, 0.1, causal, bm)
+    o, lse = OS.decode_rounded_p(q, k, v, 0.1, causal, bm, p_mode="exact", n_splits=n_splits)
+    assert np.allclose(o, ref, atol=1e-12, rtol=0)
+    fin = np.isfinite(ref_lse)
+    assert np.array_equal(np.isfinite(lse), fin) and np.allclose(lse[fin], ref_lse[fin], atol=1e-12)
+
+
+def test_decode_split_groups():
+    kept = list(range(7))
+    assert OS._split_groups(kept, 3, False) == [[0, 1, 2], [3, 4, 5], [6]]
+    assert OS._split_groups(kept, 3, True) == [[0, 2], [1], [3, 5], [4], [6], []]
+    assert OS._split_groups(kept, 8, False) == [[0], [1], [2], [3], [4], [5], [6], []]
+    assert OS._split_groups([], 2, True) == [[], [], [], []]
+
+
+@pytest.mark.parametrize("p_mode,rel", [("e4m3", None), ("bf16", 2.0 ** -8)])
+def test_decode_schedule_within_the_rounding_bounds(p_mode, rel):
+    """The partials' merge weights are their row sums, so the rounded decode
+    schedule keeps the single-pass bounds (one token, G = 8, three splits)."""
+    rng = np.random.default_rng(41)
+    Skv, D = 2000, 16
+    q = rng.uniform(-1, 1, (1, 1, 8, D))
+    k = rng.uniform(-1, 1, (1, Skv, 1, D))
+    v = _rand(rng, 1, Skv, 1, D)
+    o, _ = OS.decode_rounded_p(q, k, v, 0.2, False, None, p_mode=p_mode, sf_p=1 / 224, n_splits=3)
+    ref, _ = A.attention(q, k, v, 0.2, False)
+    for h in range(8):
+        qh = q[:, :, h:h + 1]
+        _, spv, pmax = _bound_terms(qh, k, v, 0.2, False)
+        r = ref[0, :, h]
+        if rel is None:
+            bound = 2.0 ** -4 * (spv + np.abs(r) * pmax[:, None]) / (1 - 2.0 ** -4 * pmax[:, None])
+        else:
+            bound = rel * spv
+        assert np.all(np.abs(o[0, :, h] - r) <= bound * (1 + 1e-6) + 1e-9)
