@@ -199,3 +199,22 @@ def test_nvfp4_block_quotients_match_division():
             checked += blk.size
             below += int(e < GUARD)
     assert checked > 20000 and below > 0
+
+
+def test_int8_code_from_the_low_byte_of_a_shifted_sum():
+    """The INT8 kernels read rint(q) from the low byte of RN(q + 1.5 * 2^23):
+    in [2^23, 2^24) the float32 step is 1, so the addition rounds q to an integer
+    (ties to even) and the low mantissa byte holds it in two's complement. Checked
+    on every half-integer in [-127.5, 127.5], its float32 neighbours, and a dense
+    sample of float32 values in that range; |q| <= 127 always holds there (s is
+    amax / 127 rounded to nearest, so |x| / s exceeds 127 by at most a few ulps)."""
+    halves = np.arange(-255, 256, dtype=np.float64) / 2.0
+    h32 = halves.astype(np.float32)
+    q = np.concatenate([h32, np.nextafter(h32, np.float32(-np.inf)), np.nextafter(h32, np.float32(np.inf)),
+                        np.random.default_rng(9).uniform(-127.5, 127.5, 2_000_000).astype(np.float32)])
+    q = q[np.abs(q) <= 127.5]
+    shifted = (q + np.float32(1.5 * 2 ** 23)).astype(np.float32)
+    low = (shifted.view(np.uint32) & 0xFF).astype(np.uint8).view(np.int8)
+    want = np.rint(q).astype(np.int64)
+    keep = np.abs(want) <= 127  # the 128s only arise beyond the range the kernels reach
+    assert np.array_equal(low[keep].astype(np.int64), want[keep])
