@@ -288,7 +288,9 @@ fmha_status fmha_fwd_paged(const fmha_args* args, const int32_t* page_table, int
  *     single partial: then workspace may be NULL). With several partials each
  *     writes O/l in fp32 and its log-sum-exp there, and a second kernel merges
  *     them: lse = log sum_j exp(lse_j), O = sum_j exp(lse_j - lse) O_j.
- *   Supported: D = 128, Skv <= 131072; Q/K/V BF16/BF16/BF16, BF16/BF16/E4M3
+ *   Supported: D = 128, Skv <= 131072, Sq * Hq / Hkv < 2^31 packed rows
+ *   (fmha_decode_num_splits and fmha_decode_workspace_bytes return 0 beyond
+ *   it); Q/K/V BF16/BF16/BF16, BF16/BF16/E4M3
  *   or E4M3/E4M3/E4M3 with the scale kinds of fmha_fwd; p_terms 0 or 1.
  *   Errors: FMHA_ERR_UNSUPPORTED for other shapes/dtypes, FMHA_ERR_INVALID_ARG
  *   for a missing or short workspace; device errors as in fmha_fwd_paged.   */

@@ -227,6 +227,11 @@ int sm_count() {
   return n;
 }
 
+// The decode path packs Sq * (Hq / Hkv) query rows per KV head, counted in 32 bits.
+bool packed_rows_fit(int Sq, int Hq, int Hkv) {
+  return static_cast<int64_t>(Sq) * (Hq / Hkv) <= INT32_MAX;
+}
+
 // Split plan of the decode path: KV tiles per split and the split count
 // (no trailing empty split). Automatic: about one CTA per SM, at least two KV
 // tiles per split.
@@ -304,6 +309,8 @@ fmha_status run_attention(const fmha_args* a, const uint8_t* mask, int64_t msb, 
     if (qk == QK_INT8) return fail(FMHA_ERR_UNSUPPORTED, "decode: INT8 Q/K not supported");
     if (a->p_terms == 2) return fail(FMHA_ERR_UNSUPPORTED, "decode: p_terms = 2 not supported");
     if (ceil_div(Skv, 128) > 1024) return fail(FMHA_ERR_UNSUPPORTED, "decode: Skv %d > 131072", Skv);
+    if (!packed_rows_fit(Sq, Hq, Hkv))
+      return fail(FMHA_ERR_UNSUPPORTED, "decode: Sq * Hq / Hkv packed rows exceed 2^31 - 1");
   }
 
   // scale factors
@@ -697,14 +704,14 @@ fmha_status fmha_quantize_nvfp4(const void* src, int64_t src_row_stride, int32_t
 
 size_t fmha_decode_workspace_bytes(const fmha_args* args, int32_t num_splits) {
   if (args == nullptr || args->B <= 0 || args->Hq <= 0 || args->Hkv <= 0 || args->Sq <= 0 || args->Skv < 0 ||
-      args->Hq % args->Hkv != 0)
+      args->Hq % args->Hkv != 0 || !packed_rows_fit(args->Sq, args->Hq, args->Hkv))
     return 0;
   return plan_splits(args->B, args->Hq, args->Hkv, args->Sq, args->Skv, args->D, num_splits).workspace_bytes;
 }
 
 int32_t fmha_decode_num_splits(const fmha_args* args, int32_t num_splits) {
   if (args == nullptr || args->B <= 0 || args->Hq <= 0 || args->Hkv <= 0 || args->Sq <= 0 || args->Skv < 0 ||
-      args->Hq % args->Hkv != 0)
+      args->Hq % args->Hkv != 0 || !packed_rows_fit(args->Sq, args->Hq, args->Hkv))
     return 0;
   return plan_splits(args->B, args->Hq, args->Hkv, args->Sq, args->Skv, args->D, num_splits).n_splits;
 }

@@ -177,6 +177,21 @@ def test_decode_plan_on_host(lib):
     assert lib.fmha_decode_num_splits(ctypes.byref(a), 1000) == 128
     a.Sq = 40  # 320 packed rows: no interleave; one split = one partial, no workspace
     assert lib.fmha_decode_workspace_bytes(ctypes.byref(a), 1) == 0
+    a.Sq = 2 ** 28  # x 8 query heads per KV head: 2^31 packed rows, beyond 32-bit row counts
+    assert lib.fmha_decode_num_splits(ctypes.byref(a), 4) == 0
+    assert lib.fmha_decode_workspace_bytes(ctypes.byref(a), 4) == 0
+    a.Sq = 2 ** 28 - 1
+    assert lib.fmha_decode_num_splits(ctypes.byref(a), 4) == 4
+
+
+def test_decode_rejects_packed_rows_beyond_32_bits(lib):
+    """Sq * Hq / Hkv >= 2^31 packed rows: FMHA_ERR_UNSUPPORTED before any launch."""
+    a = _args()
+    a.B, a.Hq, a.Hkv, a.Sq, a.Skv, a.D = 1, 16, 1, 2 ** 27, 1024, 128
+    for t, h in ((a.q, 16), (a.o, 16), (a.k, 1), (a.v, 1)):
+        t.stride_h, t.stride_s, t.stride_b = 128, h * 128, h * 128 * (2 ** 27)
+    st = lib.fmha_fwd_decode(ctypes.byref(a), None, 0, 0, 0, None, 0, 0, 0, None, 0, None)
+    assert st == 2 and "packed rows" in lib.fmha_last_error_message().decode()
 
 
 def _bf16_tensor(B, S, H, D, ptr=0x10000):
