@@ -93,6 +93,10 @@ MUTANTS = [
      "total = x.sum(axis=1, dtype=np.float32).astype(np.float64)", QUANT),
     ("dequant_next_block_scale", oquant, "dequantize", "idx = np.arange(S) // rows_per_block",
      "idx = np.minimum(np.arange(S) // rows_per_block + 1, sc.shape[2] - 1)", QUANT),
+    ("dequant_per_head_one_scale_per_batch", oquant, "dequantize", "return vals * sc[:, None, :, None]",
+     "return vals * sc.max(axis=1)[:, None, None, None]", QUANT),
+    ("dequant_per_channel_scales_by_token", oquant, "dequantize", "return vals * sc[:, None, :, :]",
+     "return vals * sc[:, :1, :, :]", QUANT),
     # E4M3 codec
     ("e4m3_bias_8", oe4m3, "decode", "np.exp2(exp_field.astype(np.float64) - 7.0)",
      "np.exp2(exp_field.astype(np.float64) - 8.0)", (pins_e4m3,)),
@@ -150,6 +154,8 @@ MUTANTS = [
      (pins_nvfp4,)),
     ("nibbles_swapped", onvfp4, "quantize_per_token", "packed = (codes4[:, 0::2] | (codes4[:, 1::2] << 4))",
      "packed = (codes4[:, 1::2] | (codes4[:, 0::2] << 4))", (pins_nvfp4,)),
+    ("nvfp4_dequant_nibbles_swapped", onvfp4, "dequantize", "c[:, 0::2] = packed & 0xF",
+     "c[:, 0::2] = packed >> 4", (pins_nvfp4,)),
     ("block_scale_without_e2m1_max", onvfp4, "quantize_per_token",
      "q = np.float32(np.float32(amax_b / s_t) / np.float32(6.0))", "q = np.float32(amax_b / s_t)", (pins_nvfp4,)),
 ]
